@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the batch-1 mixture-of-experts decode step on B200.
+
+Default workload ("layer"): one full-shape layer -- hidden 4096, 512 experts,
+top-4 renormalised + 1 shared expert, SwiGLU intermediate 1024, 4-bit group-64
+affine codes with bf16 scale/bias, bf16 router N(0, 0.02) -- decoding 1000
+seeded tokens x ~ N(0, 1) one at a time.  One step = one token through the
+whole hot path (router GEMV, softmax, top-K, K+1 dequantising SwiGLU experts,
+combine) = one fused kernel launch.  The weights stay resident in HBM; L2 is
+flushed (a 256 MB write) before every timed step, so the router and shared
+expert are read from HBM as they would be inside a multi-layer model; each
+step is timed with CUDA events on the launching stream and the flush is not.
+
+Other workloads: "stack4" (24 layers, 4-bit, RMSNorm + residual, 256 tokens)
+and "stack2" (60 layers, 2-bit), one step = one token through every layer
+(per-step weight traffic ~1 GB, far above L2, so no flush).
+
+``--impl reference`` times the plain double-precision CPU oracle on the same
+workload, metric and unit (the pages' own engine runs only on Apple Metal).
+
+Multi-GPU (torchrun): replicas only -- every rank decodes its own copy of the
+workload with no collective on the data path; ranks meet at a barrier and
+the step time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "decode_traffic.json")
+CSRC = os.path.join(ROOT, "quantised_expert_ffn_router_b200", "csrc")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(CSRC, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    try:
+        p = json.load(open(PEAKS_PATH))
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def layer_bytes(wl: synth.Workload) -> int:
+    """Algorithmic bytes of one token through one layer: router weights, K routed
+    + 1 shared expert blobs, norm weight, token in and out (bf16)."""
+    b = wl.n_experts * wl.hidden * 2 + (wl.top_k + 1) * wl.blob_bytes + 2 * wl.hidden * 2
+    if wl.norm:
+        b += wl.hidden * 2
+    return b
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler(threading.Thread):
+    """Samples SM clock and clock-event reasons through NVML every few ms."""
+
+    NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sync_boost", 0x40: "sw_thermal_slowdown",
+             0x80: "hw_thermal_slowdown", 0x100: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int):
+        super().__init__(daemon=True)
+        self.samples = []
+        self.stop_flag = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def run(self):
+        if not self.ok:
+            return
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM), int(get_reasons(self.h))))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def summary(self):
+        self.stop_flag.set()
+        self.join(timeout=1)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in self.NAMES.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+
+
+def oracle_tokens_per_s(wl: synth.Workload, n_tokens_max: int, budget_s: float):
+    """Times the CPU oracle on up to n_tokens_max tokens of the workload (first
+    layer for the single-layer workload, every layer for stacks), stopping after
+    budget_s seconds.  Returns (tokens/s, tokens done, threads, seconds)."""
+    import oracle
+    layers = wl.n_layers
+    cache = {}
+
+    def host_layer(l):
+        if l not in cache:
+            cache[l] = dict(router=synth.router_weight(wl, l), bias=synth.zipf_bias(wl, l),
+                            norm=synth.norm_weight(wl, l) if wl.norm else None, blobs={})
+        return cache[l]
+
+    def blob_of(l):
+        d = host_layer(l)
+
+        def get(e):
+            if e not in d["blobs"]:
+                d["blobs"][e] = synth.expert_blob(wl, l, e)
+            return d["blobs"][e]
+        return get
+
+    # routing pass (not timed) to pre-generate the experts the sample touches
+    n_tokens_max = max(1, n_tokens_max)
+    xs = [synth.token(wl, t) for t in range(n_tokens_max)]
+    if layers == 1:
+        d = host_layer(0)
+        for x in xs:
+            z = oracle.rmsnorm(x, d["norm"], wl.rms_eps) if d["norm"] is not None else x
+            idx, _, _ = oracle.topk(oracle.router_logits(d["router"], d["bias"], z), wl.top_k)
+            for e in list(idx) + [wl.n_experts]:
+                blob_of(0)(int(e))
+    threads = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    done = 0
+    for x in xs:
+        h = x
+        for l in range(layers):
+            d = host_layer(l)
+            r = oracle.layer_forward(h, router_w=d["router"], router_bias=d["bias"], norm_w=d["norm"],
+                                     eps=wl.rms_eps, top_k=wl.top_k, hidden=wl.hidden, inter=wl.inter, bits=wl.bits,
+                                     blob_of=blob_of(l))
+            h = r["out"]
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done / dt, done, threads, dt
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return 0
+    steps, warmup = args.steps, args.warmup
+    n = warmup + steps
+    tps_w, _, _, _ = oracle_tokens_per_s(wl, max(1, warmup), 1e9) if warmup else (0, 0, 0, 0)
+    tps, done, threads, dt = oracle_tokens_per_s(wl, steps, args.cpu_seconds * 4)
+    line = {
+        "impl": "reference",
+        "metric": metric_name(wl), "value": tps, "unit": "tokens/s", "n_gpus": args.gpus, "steps": done,
+        "warmup": warmup, "ms_per_step": 1e3 * dt / max(done, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, shaped like the pages' model)",
+        "config": config_dict(wl, flushed=False),
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{done} tokens of workload '{wl.name}' ({wl.n_layers} layer(s) each)"},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+
+def metric_name(wl):
+    return "MoE decode tokens/s and us/layer; expert+router HBM GB/s as fraction of peak"
+
+
+def config_dict(wl, flushed):
+    return {"workload": wl.name,
+            "shape": f"H{wl.hidden} E{wl.n_experts} top{wl.top_k}+1shared I{wl.inter} {wl.bits}-bit g64",
+            "layers": wl.n_layers, "tokens": wl.tokens, "batch": 1, "norm": wl.norm,
+            "l2": "flushed (256 MB write) before every timed step" if flushed else
+                  "per-step weight traffic far above L2 (no flush)",
+            "parallelism": "replicas"}
+
+
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(ws, value: float) -> float:
+    if ws == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_gpu(args, wl, ws, rank, local):
+    import torch
+
+    import quantised_expert_ffn_router_b200 as fm
+    from synth.gpu import DeviceWeights, tokens
+
+    torch.cuda.set_device(local)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    weights = DeviceWeights(wl)
+    descs = [fm.LayerDesc(**d) for d in weights.descs()]
+    cfg = fm.Config(wl.hidden, wl.n_experts, wl.top_k, wl.inter, wl.bits, 64, wl.n_layers, 1, wl.rms_eps, 0, 0)
+    _, ctx = fm.fmoe_create(cfg, descs, sp)
+    n_tok = wl.tokens
+    X = tokens(wl, range(n_tok))
+    OUT = torch.empty_like(X)
+    L = wl.n_layers
+    stacked = L > 1
+
+    def step(i, x_ptr=None, out_ptr=None):
+        x_ptr = X[i % n_tok].data_ptr() if x_ptr is None else x_ptr
+        out_ptr = OUT[i % n_tok].data_ptr() if out_ptr is None else out_ptr
+        if stacked:
+            fm.fmoe_stack_forward(ctx, 0, L, x_ptr, 1, out_ptr, sp)
+        else:
+            fm.fmoe_layer_forward(ctx, 0, x_ptr, 1, out_ptr, None, None, sp)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if not stacked else None
+
+    def maybe_flush(i):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+
+    steps, warmup = args.steps, args.warmup
+    for i in range(warmup):
+        maybe_flush(i)
+        step(i)
+    torch.cuda.synchronize()
+    st, word = fm.fmoe_poll_status(ctx, sp)
+    if st != 0:
+        raise RuntimeError(f"device status 0x{word:x} after warm-up")
+
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    sampler = ClockSampler(torch.cuda.current_device())
+    barrier(ws)
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(steps):
+        maybe_flush(i)
+        ev0[i].record(stream)
+        step(i)
+        ev1[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = sampler.summary()
+    step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    total_ms = max_over_ranks(ws, sum(step_ms))
+    st, word = fm.fmoe_poll_status(ctx, sp)
+    if st != 0:
+        raise RuntimeError(f"device status 0x{word:x} after timing")
+
+    # warm (no flush) reference number for the single layer
+    warm_us = None
+    if not stacked:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(steps):
+            step(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        warm_us = 1e3 * a.elapsed_time(b) / steps
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    e2e_steps = min(steps, args.e2e_steps)
+    x_host = X[:n_tok].cpu().pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    xd = torch.empty((1, wl.hidden), dtype=torch.bfloat16, device="cuda")
+    od = torch.empty_like(xd)
+    e2e_ms = []
+    for i in range(e2e_steps):
+        maybe_flush(i)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        xd.copy_(x_host[i % n_tok:i % n_tok + 1], non_blocking=True)
+        step(i, xd.data_ptr(), od.data_ptr())
+        out_host[i % n_tok:i % n_tok + 1].copy_(od, non_blocking=True)
+        b.record(stream)
+        stream.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_total = max_over_ranks(ws, sum(e2e_ms))
+    fm.fmoe_destroy(ctx)
+
+    if rank != 0:
+        return 0
+    ms_per_step = total_ms / steps
+    tps = ws * steps / (total_ms / 1e3)
+    us_layer = 1e3 * ms_per_step / L
+    bytes_launch = layer_bytes(wl)
+    achieved = bytes_launch / (us_layer * 1e-6) / 1e9
+    peak, peak_kind = hbm_peak()
+    traffic = None
+    try:
+        tr = json.load(open(TRAFFIC_PATH))
+        key = f"{wl.name}"
+        if tr.get("source_sha") == kernel_source_sha() and key in tr.get("bytes_per_launch", {}):
+            traffic = tr["bytes_per_launch"][key]
+    except Exception:
+        traffic = None
+    line = {
+        "metric": metric_name(wl), "value": tps, "unit": "tokens/s", "n_gpus": ws, "steps": steps,
+        "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp16 tensor-core MAC of exact integer codes, fp32 accumulate (bf16 I/O)",
+        "data": "synthetic (seeded, shaped like the pages' model; random weights)",
+        "config": config_dict(wl, flushed=not stacked),
+        "us_per_layer": us_layer, "hbm_gbs": achieved, "hbm_frac": achieved / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "peak_source": peak_kind, "kernel": f"decode_kernel<{wl.bits}>",
+                     "algorithmic_bytes_per_launch": bytes_launch},
+        "step_us_p10_p50_p90": [1e3 * q for q in statistics.quantiles(step_ms, n=10)[0::4]] if steps >= 10 else None,
+        "warm_l2_us_per_layer": warm_us,
+        "e2e": {"value": ws * e2e_steps / (e2e_total / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": wl.hidden * 2, "d2h_bytes_per_step": wl.hidden * 2},
+        "gpu_launches": steps * L,
+        "clocks": clocks,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        tps_cpu, done, threads, dt = oracle_tokens_per_s(wl, 400, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tps_cpu, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{done} tokens of workload '{wl.name}' ({L} layer(s) each), "
+                                          f"{dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["layer", "stack4", "stack2", "tiny"], default="layer")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    wl = synth.WORKLOADS[args.workload]
+    if args.steps is None:
+        args.steps = {"layer": 3000, "stack4": 256, "stack2": 256, "tiny": 1000}[args.workload]
+    args.warmup = max(args.warmup, 3)
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, wl, rank)
+    ws, rank, local = dist_setup(args)
+    try:
+        return run_gpu(args, wl, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

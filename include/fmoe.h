@@ -1,0 +1,186 @@
+/*
+ * fmoe.h -- C ABI of the quantised mixture-of-experts decode library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * One call runs one mixture-of-experts layer of the decode step that the
+ * Flash-MoE pages describe (page 5 "How the SSD expert streaming pipeline
+ * works": CMD2 runs the norm, the routing GEMV and the shared expert, the CPU
+ * takes softmax and top-K, CMD3 runs the expert forward pass plus combine; page
+ * 2 Key Takeaways: 512 experts per layer, K = 4 active; page 4 "The
+ * Architecture": 4-bit experts of about 6.75 MB dequantised by an FMA kernel).
+ * Here every step runs on the GPU and all expert weights stay resident in HBM.
+ *
+ * Conventions for every entry point
+ *  - Pointers named *_dev are device pointers the caller allocates and owns
+ *    (the library only borrows them); they must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls other than fmoe_create / fmoe_destroy / fmoe_poll_status only
+ *    enqueue work on `stream` and never synchronise the host.  Calls on one
+ *    context share its device workspace, so they must be ordered on one stream.
+ *  - bf16 tensors are raw bf16 bit patterns (uint16 storage).
+ *  - Every call validates its arguments before touching the GPU and returns an
+ *    fmoe_status; fmoe_last_error() gives a one-line reason.  CUDA launch
+ *    errors are reported as FMOE_ERR_CUDA.
+ */
+#ifndef FMOE_H
+#define FMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FMOE_API __attribute__((visibility("default")))
+#else
+#define FMOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct fmoe_ctx fmoe_ctx;
+
+typedef enum fmoe_status {
+  FMOE_OK = 0,
+  FMOE_ERR_INVALID_ARG = 1, /* bad value, NULL pointer, unknown/destroyed context */
+  FMOE_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement     */
+  FMOE_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned                  */
+  FMOE_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed               */
+  FMOE_ERR_OOM = 5,         /* device allocation failed                           */
+  FMOE_ERR_TIMEOUT = 6      /* a device-side bounded wait ran out (fmoe_poll_status) */
+} fmoe_status;
+
+/* fmoe_config.flags */
+#define FMOE_FLAG_FORCE_PER_TOKEN 0x1u /* T > 1: run the batch-1 kernel once per token  */
+#define FMOE_FLAG_FORCE_GROUPED 0x2u   /* T >= 1: always use the grouped batched path   */
+/* Fault injection for tests: the router step never publishes its completion,
+ * so every block's bounded wait for it runs out and the call reports
+ * FMOE_ERR_TIMEOUT through fmoe_poll_status (no GPU fault, no hang). */
+#define FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE 0x100u
+
+typedef struct fmoe_config {
+  int32_t hidden;      /* H: model width; multiple of 64, at most 4096          */
+  int32_t n_experts;   /* E: routed experts per layer (>= 1)                      */
+  int32_t top_k;       /* K: experts selected per token, 1 <= K <= min(E, 8)     */
+  int32_t inter;       /* I: SwiGLU intermediate width; multiple of 64, <= 4096  */
+  int32_t bits;        /* code width of expert weights: 4 or 2                    */
+  int32_t group;       /* quantisation group along the input dimension: must be 64 */
+  int32_t n_layers;    /* number of layer descriptors passed to fmoe_create      */
+  int32_t max_tokens;  /* largest T any call will pass (0 means 256)             */
+  float rms_eps;       /* RMSNorm epsilon (used by layers with norm_w != NULL)   */
+  uint32_t flags;      /* FMOE_FLAG_*                                             */
+  uint32_t wait_timeout_us; /* device-side bounded-wait limit; 0 means 1 second */
+} fmoe_config;
+
+/* Per-layer weights, all device pointers owned by the caller. */
+typedef struct fmoe_layer_desc {
+  const void* router_w_dev;    /* bf16 [E][H] row-major router GEMV weight            */
+  const float* router_bias_dev;/* fp32 [E] added to the logits, or NULL              */
+  void* experts_dev;           /* E routed + 1 shared expert blobs, contiguous: blob e
+                                  at byte offset e * fmoe_expert_bytes(H, I, bits), the
+                                  shared expert last (index E).  Given in the canonical
+                                  format below; fmoe_create rewrites it IN PLACE into
+                                  the library's packed tile layout (same size), and it
+                                  must stay allocated and unmodified until destroy.   */
+  const void* norm_w_dev;      /* bf16 [H] RMSNorm weight applied to the layer input
+                                  before routing and experts, or NULL for no norm.    */
+} fmoe_layer_desc;
+
+/*
+ * Canonical expert blob (input format of fmoe_create; output of
+ * fmoe_unpack_expert).  For each matrix in order gate [I][H], up [I][H],
+ * down [H][I] (rows x input columns):
+ *   codes : R*C*bits/8 bytes, row-major, 32/bits codes per little-endian
+ *           uint32; code c of a row is at bit bits*(c % (32/bits)) of word
+ *           c / (32/bits) of that row;
+ *   scales: bf16 [R][C/64];  biases: bf16 [R][C/64];
+ * weight w[r][c] = scale[r][c/64] * code[r][c] + bias[r][c/64].
+ * At H = 4096, I = 1024 a blob is 7,077,888 bytes at 4 bits (the pages' "about
+ * 6.75 MB" per expert) and 3,932,160 bytes at 2 bits.
+ */
+FMOE_API size_t fmoe_expert_bytes(int32_t hidden, int32_t inter, int32_t bits);
+
+/*
+ * Creates a context on the current CUDA device: validates `cfg` and the layer
+ * descriptors (copied; the weights they point to are borrowed), allocates the
+ * device workspace, and repacks every layer's experts_dev in place from the
+ * canonical to the packed layout on `stream` (then synchronises it).
+ * Errors: INVALID_ARG (NULL, bad shapes, K > E, bits not 2/4, group != 64),
+ * UNSUPPORTED (H or I above 4096 or a shape whose shared-memory plan does not
+ * fit), ALIGNMENT, OOM, CUDA.  On error *out is NULL.
+ */
+FMOE_API fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, void* stream, fmoe_ctx** out);
+
+/*
+ * Router step of layer `layer` for T tokens: z = RMSNorm(x) when the layer has
+ * a norm weight (else z = x), logits = W_r z (+ bias) in fp32, softmax, the K
+ * largest probabilities in descending order (equal values: lower expert index
+ * first) and their renormalised weights w_k = p_k / sum_j p_j.
+ *   x_dev   : bf16 [T][H];  idx_dev : int32 [T][K];  w_dev : fp32 [T][K].
+ * T == 0 is a no-op.  Errors: INVALID_ARG (layer or T out of range, NULL),
+ * ALIGNMENT, CUDA.
+ */
+FMOE_API fmoe_status fmoe_route(fmoe_ctx* ctx, int32_t layer, const void* x_dev, int32_t T, int32_t* idx_dev,
+                       float* w_dev, void* stream);
+
+/*
+ * One expert's SwiGLU feed-forward on the layer's (normed) input:
+ * y = W_down (silu(W_gate z) * (W_up z)), z as in fmoe_route.
+ *   expert  : 0..E-1 for a routed expert, -1 for the shared expert.
+ *   x_dev   : bf16 [T][H];  y_dev : fp32 [T][H].
+ * T == 0 is a no-op.  Errors: INVALID_ARG (expert, layer or T out of range),
+ * ALIGNMENT, CUDA.
+ */
+FMOE_API fmoe_status fmoe_expert_forward(fmoe_ctx* ctx, int32_t layer, int32_t expert, const void* x_dev, int32_t T,
+                                float* y_dev, void* stream);
+
+/*
+ * One full mixture-of-experts layer:
+ *   h_out = h_in + sum_k w_k * E_{idx_k}(z) + E_shared(z)
+ * with z, idx, w as in fmoe_route, accumulated in fp32 and rounded once to bf16.
+ *   h_in_dev, h_out_dev : bf16 [T][H], must not overlap;
+ *   idx_out_dev (int32 [T][K]) and w_out_dev (fp32 [T][K]) may be NULL.
+ * T == 1 runs the fused single-token kernel; T > 1 the grouped batched path
+ * (see FMOE_FLAG_*).  T == 0 is a no-op.  Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ */
+FMOE_API fmoe_status fmoe_layer_forward(fmoe_ctx* ctx, int32_t layer, const void* h_in_dev, int32_t T, void* h_out_dev,
+                               int32_t* idx_out_dev, float* w_out_dev, void* stream);
+
+/*
+ * Layers layer_begin .. layer_end-1 in sequence (a mixture-of-experts-only
+ * stack: each layer's output is the next layer's input), equivalent to
+ * chaining fmoe_layer_forward; intermediate activations live in the context
+ * workspace.  h_in_dev and h_out_dev (bf16 [T][H]) must not overlap.
+ */
+FMOE_API fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer_end, const void* h_in_dev,
+                               int32_t T, void* h_out_dev, void* stream);
+
+/*
+ * Writes expert `expert` (-1: shared) of `layer` back in the canonical format
+ * into dst_dev (fmoe_expert_bytes bytes).  Used to check the packed layout
+ * round trip.
+ */
+FMOE_API fmoe_status fmoe_unpack_expert(fmoe_ctx* ctx, int32_t layer, int32_t expert, void* dst_dev, void* stream);
+
+/*
+ * Synchronises `stream`, reads the device status word and clears it.
+ * *device_status (may be NULL) receives the raw word (0 = no fault).  Returns
+ * FMOE_ERR_TIMEOUT when a bounded wait ran out since the last poll (the
+ * workspace counters are then reset so the context stays usable), FMOE_OK
+ * otherwise.
+ */
+FMOE_API fmoe_status fmoe_poll_status(fmoe_ctx* ctx, void* stream, uint32_t* device_status);
+
+/* Releases the workspace; the context pointer is invalid afterwards (later
+ * calls with it return FMOE_ERR_INVALID_ARG).  Does not free caller memory. */
+FMOE_API fmoe_status fmoe_destroy(fmoe_ctx* ctx);
+
+/* One-line description of the last error on `ctx` (or of the last failed
+ * fmoe_create when ctx is NULL).  Valid until the next call on that context. */
+FMOE_API const char* fmoe_last_error(const fmoe_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FMOE_H */

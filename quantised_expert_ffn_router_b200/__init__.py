@@ -1,0 +1,153 @@
+"""Python binding of libfmoe.so, the C-ABI mixture-of-experts decode library.
+
+Argument marshalling only: every function forwards to the C entry point of
+the same name in ``include/fmoe.h`` (device pointers and a CUDA stream handle
+as plain integers).  All computation runs in the library's CUDA kernels; there
+is no Python or CPU fallback, and importing this package fails loudly when the
+library cannot be built or loaded.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+from . import build as _build
+
+__all__ = [
+    "FMOE_OK", "FMOE_ERR_INVALID_ARG", "FMOE_ERR_UNSUPPORTED", "FMOE_ERR_ALIGNMENT", "FMOE_ERR_CUDA",
+    "FMOE_ERR_OOM", "FMOE_ERR_TIMEOUT", "FMOE_FLAG_FORCE_PER_TOKEN", "FMOE_FLAG_FORCE_GROUPED",
+    "FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE", "Config", "LayerDesc", "FmoeError", "lib", "fmoe_expert_bytes",
+    "fmoe_create", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward", "fmoe_stack_forward",
+    "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error", "EXPORTED_SYMBOLS",
+]
+
+FMOE_OK, FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED, FMOE_ERR_ALIGNMENT = 0, 1, 2, 3
+FMOE_ERR_CUDA, FMOE_ERR_OOM, FMOE_ERR_TIMEOUT = 4, 5, 6
+FMOE_FLAG_FORCE_PER_TOKEN = 0x1
+FMOE_FLAG_FORCE_GROUPED = 0x2
+FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE = 0x100
+
+EXPORTED_SYMBOLS = ["fmoe_expert_bytes", "fmoe_create", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
+                    "fmoe_stack_forward", "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy",
+                    "fmoe_last_error"]
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("inter", ctypes.c_int32), ("bits", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("n_layers", ctypes.c_int32), ("max_tokens", ctypes.c_int32), ("rms_eps", ctypes.c_float),
+                ("flags", ctypes.c_uint32), ("wait_timeout_us", ctypes.c_uint32)]
+
+
+class LayerDesc(ctypes.Structure):
+    _fields_ = [("router_w_dev", ctypes.c_void_p), ("router_bias_dev", ctypes.c_void_p),
+                ("experts_dev", ctypes.c_void_p), ("norm_w_dev", ctypes.c_void_p)]
+
+
+class FmoeError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"fmoe status {status}: {message}")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib():
+    """The loaded libfmoe.so (built in-tree with nvcc when missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.LIB
+            if _build.stale():
+                path = _build.build()
+            if not os.path.exists(path):
+                raise ImportError(f"libfmoe.so not found at {path}")
+            L = ctypes.CDLL(path)
+            P, i32, u32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32
+            L.fmoe_expert_bytes.argtypes = [i32, i32, i32]
+            L.fmoe_expert_bytes.restype = ctypes.c_size_t
+            L.fmoe_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerDesc), P, ctypes.POINTER(P)]
+            L.fmoe_route.argtypes = [P, i32, P, i32, P, P, P]
+            L.fmoe_expert_forward.argtypes = [P, i32, i32, P, i32, P, P]
+            L.fmoe_layer_forward.argtypes = [P, i32, P, i32, P, P, P, P]
+            L.fmoe_stack_forward.argtypes = [P, i32, i32, P, i32, P, P]
+            L.fmoe_unpack_expert.argtypes = [P, i32, i32, P, P]
+            L.fmoe_poll_status.argtypes = [P, P, ctypes.POINTER(u32)]
+            L.fmoe_destroy.argtypes = [P]
+            L.fmoe_last_error.argtypes = [P]
+            L.fmoe_last_error.restype = ctypes.c_char_p
+            for name in ("fmoe_create", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
+                         "fmoe_stack_forward", "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy"):
+                getattr(L, name).restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _check(ctx, status: int) -> int:
+    if status != FMOE_OK:
+        raise FmoeError(status, fmoe_last_error(ctx))
+    return status
+
+
+def _vp(x):
+    return None if x is None or x == 0 else ctypes.c_void_p(int(x))
+
+
+def fmoe_last_error(ctx=None) -> str:
+    msg = lib().fmoe_last_error(_vp(ctx))
+    return msg.decode() if msg else ""
+
+
+def fmoe_expert_bytes(hidden: int, inter: int, bits: int) -> int:
+    return int(lib().fmoe_expert_bytes(hidden, inter, bits))
+
+
+def fmoe_create(cfg: Config, layers, stream: int = 0, *, check: bool = True):
+    """Returns (status, ctx handle as int or None)."""
+    arr = (LayerDesc * len(layers))(*layers)
+    out = ctypes.c_void_p()
+    st = lib().fmoe_create(ctypes.byref(cfg), arr, _vp(stream), ctypes.byref(out))
+    if check:
+        _check(None, st)
+    return st, out.value
+
+
+def fmoe_route(ctx, layer, x_dev, T, idx_dev, w_dev, stream=0, *, check=True) -> int:
+    st = lib().fmoe_route(_vp(ctx), layer, _vp(x_dev), T, _vp(idx_dev), _vp(w_dev), _vp(stream))
+    return _check(ctx, st) if check else st
+
+
+def fmoe_expert_forward(ctx, layer, expert, x_dev, T, y_dev, stream=0, *, check=True) -> int:
+    st = lib().fmoe_expert_forward(_vp(ctx), layer, expert, _vp(x_dev), T, _vp(y_dev), _vp(stream))
+    return _check(ctx, st) if check else st
+
+
+def fmoe_layer_forward(ctx, layer, h_in_dev, T, h_out_dev, idx_out_dev=None, w_out_dev=None, stream=0, *,
+                       check=True) -> int:
+    st = lib().fmoe_layer_forward(_vp(ctx), layer, _vp(h_in_dev), T, _vp(h_out_dev), _vp(idx_out_dev),
+                                  _vp(w_out_dev), _vp(stream))
+    return _check(ctx, st) if check else st
+
+
+def fmoe_stack_forward(ctx, layer_begin, layer_end, h_in_dev, T, h_out_dev, stream=0, *, check=True) -> int:
+    st = lib().fmoe_stack_forward(_vp(ctx), layer_begin, layer_end, _vp(h_in_dev), T, _vp(h_out_dev), _vp(stream))
+    return _check(ctx, st) if check else st
+
+
+def fmoe_unpack_expert(ctx, layer, expert, dst_dev, stream=0, *, check=True) -> int:
+    st = lib().fmoe_unpack_expert(_vp(ctx), layer, expert, _vp(dst_dev), _vp(stream))
+    return _check(ctx, st) if check else st
+
+
+def fmoe_poll_status(ctx, stream=0):
+    """Returns (status, raw device status word)."""
+    word = ctypes.c_uint32(0)
+    st = lib().fmoe_poll_status(_vp(ctx), _vp(stream), ctypes.byref(word))
+    return st, word.value
+
+
+def fmoe_destroy(ctx) -> int:
+    return lib().fmoe_destroy(_vp(ctx))

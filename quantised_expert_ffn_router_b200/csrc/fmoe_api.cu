@@ -1,0 +1,461 @@
+// fmoe_api.cu -- C ABI (include/fmoe.h): contexts, argument validation,
+// shared-memory plans and kernel launches.  No compute happens on the host.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <string>
+#include <vector>
+
+#include "fmoe_internal.h"
+
+using namespace fmoe;
+
+struct fmoe_ctx {
+  fmoe_config cfg;
+  std::vector<fmoe_layer_desc> layers;
+  int device = 0;
+  int n_sm = 0;
+  bool pdl_ok = true;
+  void* ws = nullptr;  // device workspace
+  size_t ws_bytes = 0;
+  WsHeader* hdr = nullptr;
+  float* logits = nullptr;
+  float* act = nullptr;
+  uint16_t* stack_buf[2] = {nullptr, nullptr};  // ping-pong activations, [max_tokens][H] bf16
+  DecodePlan plan[3];  // per mode: layer, expert, route (pointers filled per call)
+  std::string err;
+};
+
+namespace {
+
+std::mutex g_mu;
+std::set<const fmoe_ctx*> g_live;
+thread_local std::string g_create_err;
+
+bool alive(const fmoe_ctx* c) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return c != nullptr && g_live.count(c) != 0;
+}
+
+fmoe_status fail(fmoe_ctx* c, fmoe_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  if (c) c->err = buf;
+  else g_create_err = buf;
+  return st;
+}
+
+bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+// Shared-memory layout of the fused kernel for one mode; false if it does not fit.
+bool make_plan(const fmoe_config& c, int grid, int mode, int nstage, int max_smem, DecodePlan& P) {
+  memset(&P, 0, sizeof P);
+  P.H = c.hidden;
+  P.E = c.n_experts;
+  P.K = c.top_k;
+  P.I = c.inter;
+  P.bits = c.bits;
+  P.mode = mode;
+  P.n_slots = mode == kModeLayer ? c.top_k + 1 : (mode == kModeExpert ? 1 : 0);
+  P.grid = grid;
+  P.tb = tile_bytes(c.bits);
+  P.cb = tile_code_bytes(c.bits);
+  P.gu_tiles = c.hidden / kGroup;
+  P.gu_unit_bytes = P.gu_tiles * P.tb;
+  P.n_kr_gu = (c.hidden + 255) / 256;
+  P.teams_gu = kWarps / P.n_kr_gu;
+  P.units_per_slot = c.inter / 8;
+  P.total_units = P.n_slots * P.units_per_slot;
+  P.dn_tiles = c.inter / kGroup;
+  P.dn_job_bytes = P.dn_tiles * P.tb;
+  P.n_kr_dn = (c.inter + 255) / 256;
+  P.teams_dn = kWarps / P.n_kr_dn;
+  P.n_rb = c.hidden / 16;
+  P.rb_per_cta = P.n_slots > 0 ? (P.n_rb + grid - 1) / grid : 0;
+  const bool router = mode != kModeExpert;
+  P.router_rows = router ? (c.n_experts + grid - 1) / grid : 0;
+  P.router_chunks = (c.hidden + 255) / 256;
+  P.nstage = P.total_units > 0 ? nstage : 1;
+
+  uint32_t off = 0;
+  P.off_ring = off;
+  P.stage_bytes = P.total_units > 0 ? (uint32_t)(P.teams_gu * P.gu_unit_bytes) : 0;
+  off = align_up(off + P.nstage * P.stage_bytes, 128);
+  P.off_down = off;
+  const uint32_t down_bytes = (uint32_t)(P.n_slots * P.rb_per_cta * P.dn_job_bytes);
+  off = align_up(off + down_bytes, 128);
+  const uint32_t router_bytes = (uint32_t)(P.router_rows * c.hidden * 2);
+  const uint32_t routed_down = P.n_slots > 1 ? (uint32_t)((P.n_slots - 1) * P.rb_per_cta * P.dn_job_bytes) : 0;
+  if (router_bytes > 0 && routed_down >= router_bytes && mode == kModeLayer) {
+    P.off_router = P.off_down + (uint32_t)(P.rb_per_cta * P.dn_job_bytes);
+  } else {
+    P.off_router = off;
+    off = align_up(off + router_bytes, 128);
+  }
+  P.off_zfrag = off;
+  off = align_up(off + (uint32_t)c.hidden * 2, 128);
+  P.off_zinfo = off;
+  off = align_up(off + (uint32_t)(c.hidden / kGroup) * 8, 128);
+  P.afrag_bytes = align_up((uint32_t)c.inter * 2, 128);
+  P.ainfo_bytes = align_up((uint32_t)(c.inter / kGroup) * 8, 128);
+  P.off_afrag = off;
+  off += 2 * P.afrag_bytes;
+  P.off_ainfo = off;
+  off += 2 * P.ainfo_bytes;
+  P.off_z = off;
+  off = align_up(off + std::max<uint32_t>((uint32_t)c.hidden * 2, (uint32_t)c.n_experts * 4), 128);
+  P.off_gupart = off;
+  off += 2 * kWarps * 16 * 4;
+  P.off_dnpart = off;
+  off += kWarps * 16 * 4;
+  P.off_y = off;
+  off = align_up(off + (uint32_t)(std::max(P.rb_per_cta, 1) * std::max(P.n_slots, 1) * 16 * 4), 128);
+  P.off_rpart = off;
+  off = align_up(off + (uint32_t)(std::max(P.router_rows, 1) * kWarps * 4), 128);
+  P.off_misc = off;
+  off += 128;
+  P.off_bar = off;
+  off += (uint32_t)(P.nstage + kMaxSlots + 1) * 8;
+  P.smem_bytes = align_up(off, 128);
+  return (int)P.smem_bytes <= max_smem;
+}
+
+bool plan_all(fmoe_ctx* ctx, int max_smem) {
+  const int modes[3] = {kModeLayer, kModeExpert, kModeRoute};
+  for (int m = 0; m < 3; ++m) {
+    bool ok = false;
+    for (int ns = 3; ns >= 2 && !ok; --ns) ok = make_plan(ctx->cfg, ctx->n_sm, modes[m], ns, max_smem, ctx->plan[m]);
+    if (!ok) return false;
+  }
+  return true;
+}
+
+fmoe_status cuda_fail(fmoe_ctx* c, cudaError_t e, const char* what) {
+  return fail(c, FMOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+fmoe_status check_ctx_layer(fmoe_ctx* ctx, int32_t layer, int32_t T) {
+  if (layer < 0 || layer >= ctx->cfg.n_layers) return fail(ctx, FMOE_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (T < 0 || T > ctx->cfg.max_tokens)
+    return fail(ctx, FMOE_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, ctx->cfg.max_tokens);
+  return FMOE_OK;
+}
+
+// Fills the per-call pointers of a plan.
+DecodePlan bind(const fmoe_ctx* ctx, int mode, int layer) {
+  DecodePlan P = ctx->plan[mode];
+  const fmoe_layer_desc& L = ctx->layers[layer];
+  P.experts = static_cast<const uint8_t*>(L.experts_dev);
+  P.blob_bytes = expert_bytes(ctx->cfg.hidden, ctx->cfg.inter, ctx->cfg.bits);
+  P.router_w = static_cast<const uint16_t*>(L.router_w_dev);
+  P.router_bias = L.router_bias_dev;
+  P.norm_w = static_cast<const uint16_t*>(L.norm_w_dev);
+  P.eps = ctx->cfg.rms_eps;
+  P.ws = ctx->hdr;
+  P.ws_logits = ctx->logits;
+  P.ws_a = ctx->act;
+  P.flags = ctx->cfg.flags;
+  P.timeout_ns = (uint64_t)(ctx->cfg.wait_timeout_us ? ctx->cfg.wait_timeout_us : 1000000u) * 1000ull;
+  return P;
+}
+
+fmoe_status launch(fmoe_ctx* ctx, const DecodePlan& P, void* stream) {
+  int rc = launch_decode(P, stream, true, ctx->pdl_ok);
+  if (rc != 0 && ctx->pdl_ok) {
+    cudaGetLastError();
+    rc = launch_decode(P, stream, true, false);
+    if (rc == 0) ctx->pdl_ok = false;
+  }
+  if (rc != 0) {
+    cudaGetLastError();
+    return cuda_fail(ctx, (cudaError_t)rc, "decode launch");
+  }
+  return FMOE_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  auto x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fmoe_expert_bytes(int32_t hidden, int32_t inter, int32_t bits) {
+  if (hidden <= 0 || inter <= 0 || hidden % kGroup || inter % kGroup || (bits != 2 && bits != 4)) return 0;
+  return (size_t)expert_bytes(hidden, inter, bits);
+}
+
+const char* fmoe_last_error(const fmoe_ctx* ctx) {
+  if (ctx == nullptr) return g_create_err.c_str();
+  if (!alive(ctx)) return "invalid or destroyed context";
+  return ctx->err.c_str();
+}
+
+fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, void* stream, fmoe_ctx** out) {
+  if (out) *out = nullptr;
+  if (!cfg || !layers || !out) return fail(nullptr, FMOE_ERR_INVALID_ARG, "NULL argument");
+  fmoe_config c = *cfg;
+  if (c.max_tokens == 0) c.max_tokens = 256;
+  if (c.hidden <= 0 || c.hidden % kGroup)
+    return fail(nullptr, FMOE_ERR_INVALID_ARG, "hidden=%d must be a positive multiple of 64", c.hidden);
+  if (c.inter <= 0 || c.inter % kGroup)
+    return fail(nullptr, FMOE_ERR_INVALID_ARG, "inter=%d must be a positive multiple of 64", c.inter);
+  if (c.n_experts <= 0) return fail(nullptr, FMOE_ERR_INVALID_ARG, "n_experts=%d", c.n_experts);
+  if (c.top_k <= 0 || c.top_k > c.n_experts)
+    return fail(nullptr, FMOE_ERR_INVALID_ARG, "top_k=%d must be in [1, n_experts=%d]", c.top_k, c.n_experts);
+  if (c.bits != 2 && c.bits != 4) return fail(nullptr, FMOE_ERR_INVALID_ARG, "bits=%d must be 2 or 4", c.bits);
+  if (c.group != kGroup) return fail(nullptr, FMOE_ERR_INVALID_ARG, "group=%d must be 64", c.group);
+  if (c.n_layers <= 0) return fail(nullptr, FMOE_ERR_INVALID_ARG, "n_layers=%d", c.n_layers);
+  if (c.max_tokens < 0) return fail(nullptr, FMOE_ERR_INVALID_ARG, "max_tokens=%d", c.max_tokens);
+  if (!(c.rms_eps >= 0.f)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "rms_eps must be >= 0");
+  if (c.top_k > kMaxTopK) return fail(nullptr, FMOE_ERR_UNSUPPORTED, "top_k=%d above %d", c.top_k, kMaxTopK);
+  if (c.hidden > 4096 || c.inter > 4096)
+    return fail(nullptr, FMOE_ERR_UNSUPPORTED, "hidden=%d / inter=%d above 4096", c.hidden, c.inter);
+  if (c.n_experts > 65536) return fail(nullptr, FMOE_ERR_UNSUPPORTED, "n_experts=%d above 65536", c.n_experts);
+  for (int l = 0; l < c.n_layers; ++l) {
+    const fmoe_layer_desc& L = layers[l];
+    if (!L.router_w_dev || !L.experts_dev)
+      return fail(nullptr, FMOE_ERR_INVALID_ARG, "layer %d: NULL router or experts pointer", l);
+    if (misaligned(L.router_w_dev) || misaligned(L.experts_dev) || misaligned(L.router_bias_dev) ||
+        misaligned(L.norm_w_dev))
+      return fail(nullptr, FMOE_ERR_ALIGNMENT, "layer %d: pointer not 16-byte aligned", l);
+  }
+
+  fmoe_ctx* ctx = new fmoe_ctx();
+  ctx->cfg = c;
+  ctx->layers.assign(layers, layers + c.n_layers);
+  auto bail = [&](fmoe_status st) {
+    g_create_err = ctx->err;
+    if (ctx->ws) cudaFree(ctx->ws);
+    delete ctx;
+    return st;
+  };
+  cudaError_t e = cudaGetDevice(&ctx->device);
+  if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "cudaGetDevice"));
+  cudaDeviceGetAttribute(&ctx->n_sm, cudaDevAttrMultiProcessorCount, ctx->device);
+  int coop = 0;
+  cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, ctx->device);
+  if (!coop) return bail(fail(ctx, FMOE_ERR_UNSUPPORTED, "device lacks cooperative launch"));
+  const int max_smem = decode_max_smem_optin(ctx->device);
+  if (!plan_all(ctx, max_smem))
+    return bail(fail(ctx, FMOE_ERR_UNSUPPORTED, "shared-memory plan does not fit (%d bytes available)", max_smem));
+  for (int m = 0; m < 3; ++m) {
+    int blocks = 0;
+    int rc = decode_occupancy(c.bits, (int)ctx->plan[m].smem_bytes, &blocks);
+    if (rc != 0) return bail(cuda_fail(ctx, (cudaError_t)rc, "occupancy query"));
+    if (blocks < 1) return bail(fail(ctx, FMOE_ERR_UNSUPPORTED, "fused kernel cannot be resident"));
+  }
+
+  // workspace: header | logits [E] | activations [kMaxSlots][I] | 2 x [max_tokens][H] bf16
+  size_t off = 256;
+  size_t off_logits = off;
+  off += ((size_t)c.n_experts * 4 + 255) / 256 * 256;
+  size_t off_act = off;
+  off += ((size_t)kMaxSlots * c.inter * 4 + 255) / 256 * 256;
+  size_t off_stack = off;
+  size_t stack_bytes = ((size_t)std::max(c.max_tokens, 1) * c.hidden * 2 + 255) / 256 * 256;
+  off += 2 * stack_bytes;
+  ctx->ws_bytes = off;
+  e = cudaMalloc(&ctx->ws, ctx->ws_bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    ctx->ws = nullptr;
+    return bail(fail(ctx, FMOE_ERR_OOM, "workspace allocation of %zu bytes failed", ctx->ws_bytes));
+  }
+  uint8_t* base = static_cast<uint8_t*>(ctx->ws);
+  ctx->hdr = reinterpret_cast<WsHeader*>(base);
+  ctx->logits = reinterpret_cast<float*>(base + off_logits);
+  ctx->act = reinterpret_cast<float*>(base + off_act);
+  ctx->stack_buf[0] = reinterpret_cast<uint16_t*>(base + off_stack);
+  ctx->stack_buf[1] = reinterpret_cast<uint16_t*>(base + off_stack + stack_bytes);
+  cudaStream_t st = (cudaStream_t)stream;
+  e = cudaMemsetAsync(ctx->ws, 0, ctx->ws_bytes, st);
+  if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "workspace clear"));
+
+  // In-place repack, canonical -> packed, through a bounded staging buffer.
+  const size_t blob = (size_t)expert_bytes(c.hidden, c.inter, c.bits);
+  const int per_layer = c.n_experts + 1;
+  int chunk = (int)std::max<size_t>(1, std::min<size_t>((size_t)per_layer, (size_t)(256u << 20) / blob));
+  void* tmp = nullptr;
+  e = cudaMalloc(&tmp, (size_t)chunk * blob);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return bail(fail(ctx, FMOE_ERR_OOM, "repack staging allocation failed"));
+  }
+  for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
+    uint8_t* ex = static_cast<uint8_t*>(ctx->layers[l].experts_dev);
+    for (int e0 = 0; e0 < per_layer; e0 += chunk) {
+      int n = std::min(chunk, per_layer - e0);
+      e = cudaMemcpyAsync(tmp, ex + (size_t)e0 * blob, (size_t)n * blob, cudaMemcpyDeviceToDevice, st);
+      if (e != cudaSuccess) break;
+      int rc = launch_repack(static_cast<const uint8_t*>(tmp), ex + (size_t)e0 * blob, n, c.hidden, c.inter, c.bits,
+                             1, stream);
+      if (rc != 0) { e = (cudaError_t)rc; break; }
+    }
+  }
+  cudaError_t e2 = cudaStreamSynchronize(st);
+  cudaFree(tmp);
+  if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "expert repack"));
+  if (e2 != cudaSuccess) return bail(cuda_fail(ctx, e2, "expert repack (sync)"));
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_live.insert(ctx);
+  }
+  *out = ctx;
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_destroy(fmoe_ctx* ctx) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (ctx == nullptr || g_live.erase(ctx) == 0) {
+      g_create_err = "fmoe_destroy: invalid or destroyed context";
+      return FMOE_ERR_INVALID_ARG;
+    }
+  }
+  if (ctx->ws) cudaFree(ctx->ws);
+  delete ctx;
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_route(fmoe_ctx* ctx, int32_t layer, const void* x_dev, int32_t T, int32_t* idx_dev, float* w_dev,
+                       void* stream) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  fmoe_status s = check_ctx_layer(ctx, layer, T);
+  if (s != FMOE_OK) return s;
+  if (T == 0) return FMOE_OK;
+  if (!x_dev || !idx_dev || !w_dev) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL tensor");
+  if (misaligned(x_dev) || misaligned(idx_dev) || misaligned(w_dev))
+    return fail(ctx, FMOE_ERR_ALIGNMENT, "tensor not 16-byte aligned");
+  const int H = ctx->cfg.hidden, K = ctx->cfg.top_k;
+  for (int t = 0; t < T; ++t) {
+    DecodePlan P = bind(ctx, kModeRoute, layer);
+    P.h_in = static_cast<const uint16_t*>(x_dev) + (size_t)t * H;
+    P.idx_out = idx_dev + (size_t)t * K;
+    P.w_out = w_dev + (size_t)t * K;
+    s = launch(ctx, P, stream);
+    if (s != FMOE_OK) return s;
+  }
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_expert_forward(fmoe_ctx* ctx, int32_t layer, int32_t expert, const void* x_dev, int32_t T,
+                                float* y_dev, void* stream) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  fmoe_status s = check_ctx_layer(ctx, layer, T);
+  if (s != FMOE_OK) return s;
+  if (expert < -1 || expert >= ctx->cfg.n_experts)
+    return fail(ctx, FMOE_ERR_INVALID_ARG, "expert %d outside [-1, %d)", expert, ctx->cfg.n_experts);
+  if (T == 0) return FMOE_OK;
+  if (!x_dev || !y_dev) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL tensor");
+  if (misaligned(x_dev) || misaligned(y_dev)) return fail(ctx, FMOE_ERR_ALIGNMENT, "tensor not 16-byte aligned");
+  const int H = ctx->cfg.hidden;
+  for (int t = 0; t < T; ++t) {
+    DecodePlan P = bind(ctx, kModeExpert, layer);
+    P.expert_id = expert < 0 ? ctx->cfg.n_experts : expert;
+    P.h_in = static_cast<const uint16_t*>(x_dev) + (size_t)t * H;
+    P.y_out = y_dev + (size_t)t * H;
+    s = launch(ctx, P, stream);
+    if (s != FMOE_OK) return s;
+  }
+  return FMOE_OK;
+}
+
+static fmoe_status layer_tokens(fmoe_ctx* ctx, int32_t layer, const uint16_t* h_in, int32_t T, uint16_t* h_out,
+                                int32_t* idx, float* w, void* stream) {
+  const int H = ctx->cfg.hidden, K = ctx->cfg.top_k;
+  for (int t = 0; t < T; ++t) {
+    DecodePlan P = bind(ctx, kModeLayer, layer);
+    P.h_in = h_in + (size_t)t * H;
+    P.h_out = h_out + (size_t)t * H;
+    P.idx_out = idx ? idx + (size_t)t * K : nullptr;
+    P.w_out = w ? w + (size_t)t * K : nullptr;
+    fmoe_status s = launch(ctx, P, stream);
+    if (s != FMOE_OK) return s;
+  }
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_layer_forward(fmoe_ctx* ctx, int32_t layer, const void* h_in_dev, int32_t T, void* h_out_dev,
+                               int32_t* idx_out_dev, float* w_out_dev, void* stream) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  fmoe_status s = check_ctx_layer(ctx, layer, T);
+  if (s != FMOE_OK) return s;
+  if (T == 0) return FMOE_OK;
+  if (!h_in_dev || !h_out_dev) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL tensor");
+  if (misaligned(h_in_dev) || misaligned(h_out_dev) || misaligned(idx_out_dev) || misaligned(w_out_dev))
+    return fail(ctx, FMOE_ERR_ALIGNMENT, "tensor not 16-byte aligned");
+  const size_t bytes = (size_t)T * ctx->cfg.hidden * 2;
+  if (overlaps(h_in_dev, bytes, h_out_dev, bytes)) return fail(ctx, FMOE_ERR_INVALID_ARG, "h_out overlaps h_in");
+  return layer_tokens(ctx, layer, static_cast<const uint16_t*>(h_in_dev), T, static_cast<uint16_t*>(h_out_dev),
+                      idx_out_dev, w_out_dev, stream);
+}
+
+fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer_end, const void* h_in_dev, int32_t T,
+                               void* h_out_dev, void* stream) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  if (layer_begin < 0 || layer_end > ctx->cfg.n_layers || layer_begin >= layer_end)
+    return fail(ctx, FMOE_ERR_INVALID_ARG, "layer range [%d, %d) invalid", layer_begin, layer_end);
+  fmoe_status s = check_ctx_layer(ctx, layer_begin, T);
+  if (s != FMOE_OK) return s;
+  if (T == 0) return FMOE_OK;
+  if (!h_in_dev || !h_out_dev) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL tensor");
+  if (misaligned(h_in_dev) || misaligned(h_out_dev)) return fail(ctx, FMOE_ERR_ALIGNMENT, "tensor not 16-byte aligned");
+  const size_t bytes = (size_t)T * ctx->cfg.hidden * 2;
+  if (overlaps(h_in_dev, bytes, h_out_dev, bytes)) return fail(ctx, FMOE_ERR_INVALID_ARG, "h_out overlaps h_in");
+  const uint16_t* cur = static_cast<const uint16_t*>(h_in_dev);
+  for (int l = layer_begin; l < layer_end; ++l) {
+    uint16_t* dst = (l + 1 == layer_end) ? static_cast<uint16_t*>(h_out_dev) : ctx->stack_buf[(l - layer_begin) & 1];
+    s = layer_tokens(ctx, l, cur, T, dst, nullptr, nullptr, stream);
+    if (s != FMOE_OK) return s;
+    cur = dst;
+  }
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_unpack_expert(fmoe_ctx* ctx, int32_t layer, int32_t expert, void* dst_dev, void* stream) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  if (layer < 0 || layer >= ctx->cfg.n_layers) return fail(ctx, FMOE_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (expert < -1 || expert >= ctx->cfg.n_experts)
+    return fail(ctx, FMOE_ERR_INVALID_ARG, "expert %d outside [-1, %d)", expert, ctx->cfg.n_experts);
+  if (!dst_dev) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL destination");
+  if (misaligned(dst_dev)) return fail(ctx, FMOE_ERR_ALIGNMENT, "destination not 16-byte aligned");
+  const size_t blob = (size_t)expert_bytes(ctx->cfg.hidden, ctx->cfg.inter, ctx->cfg.bits);
+  const int e = expert < 0 ? ctx->cfg.n_experts : expert;
+  const uint8_t* src = static_cast<const uint8_t*>(ctx->layers[layer].experts_dev) + (size_t)e * blob;
+  int rc = launch_repack(src, static_cast<uint8_t*>(dst_dev), 1, ctx->cfg.hidden, ctx->cfg.inter, ctx->cfg.bits, 0,
+                         stream);
+  if (rc != 0) return cuda_fail(ctx, (cudaError_t)rc, "unpack");
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_poll_status(fmoe_ctx* ctx, void* stream, uint32_t* device_status) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  cudaStream_t st = (cudaStream_t)stream;
+  WsHeader h;
+  cudaError_t e = cudaMemcpyAsync(&h, ctx->hdr, sizeof h, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "status read");
+  if (device_status) *device_status = h.status;
+  if (h.status != 0) {
+    e = cudaMemsetAsync(ctx->hdr, 0, sizeof(WsHeader), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "status reset");
+    return fail(ctx, FMOE_ERR_TIMEOUT, "device-side wait timed out (status 0x%x)", h.status);
+  }
+  return FMOE_OK;
+}
+
+}  // extern "C"
