@@ -187,7 +187,7 @@ def run_reference(args, wl, rank):
         "metric": metric_name(wl), "value": tps, "unit": "tokens/s", "n_gpus": args.gpus, "steps": done,
         "warmup": warmup, "ms_per_step": 1e3 * dt / max(done, 1), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, shaped like the pages' model)",
-        "config": config_dict(wl, flushed=False),
+        "config": config_dict(wl, flushed=False, cpu=True),
         "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": f"{done} tokens of workload '{wl.name}' ({wl.n_layers} layer(s) each)"},
         "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -203,12 +203,12 @@ def metric_name(wl):
     return "MoE decode tokens/s and us/layer; expert+router HBM GB/s as fraction of peak"
 
 
-def config_dict(wl, flushed):
+def config_dict(wl, flushed, cpu=False):
     return {"workload": wl.name,
             "shape": f"H{wl.hidden} E{wl.n_experts} top{wl.top_k}+1shared I{wl.inter} {wl.bits}-bit g64",
             "layers": wl.n_layers, "tokens": wl.tokens, "batch": 1, "norm": wl.norm,
-            "l2": "flushed (256 MB write) before every timed step" if flushed else
-                  "per-step weight traffic far above L2 (no flush)",
+            "l2": "n/a (CPU oracle)" if cpu else ("flushed (256 MB write) before every timed step" if flushed else
+                                                  "per-step weight traffic far above L2 (no flush)"),
             "parallelism": "replicas"}
 
 

@@ -165,9 +165,10 @@ FMOE_API fmoe_status fmoe_unpack_expert(fmoe_ctx* ctx, int32_t layer, int32_t ex
 /*
  * Synchronises `stream`, reads the device status word and clears it.
  * *device_status (may be NULL) receives the raw word (0 = no fault).  Returns
- * FMOE_ERR_TIMEOUT when a bounded wait ran out since the last poll (the
- * workspace counters are then reset so the context stays usable), FMOE_OK
- * otherwise.
+ * FMOE_ERR_TIMEOUT when a bounded wait ran out since the last poll, FMOE_OK
+ * otherwise.  The context stays usable after a timeout: every launch tags its
+ * cross-block results with a fresh epoch, so nothing from the failed launch is
+ * read by the next one.
  */
 FMOE_API fmoe_status fmoe_poll_status(fmoe_ctx* ctx, void* stream, uint32_t* device_status);
 

@@ -24,8 +24,12 @@ struct fmoe_ctx {
   void* ws = nullptr;  // device workspace
   size_t ws_bytes = 0;
   WsHeader* hdr = nullptr;
-  float* logits = nullptr;
-  float* act = nullptr;
+  uint64_t* logits = nullptr;  // tagged
+  uint64_t* act = nullptr;     // tagged
+  uint64_t* asum = nullptr;    // tagged
+  uint64_t* amax = nullptr;    // tag-keyed maxima
+  uint32_t* tasks = nullptr;   // device [3 modes][grid][kMaxTasks]
+  int32_t* ntasks = nullptr;   // device [3 modes][grid]
   uint16_t* stack_buf[2] = {nullptr, nullptr};  // ping-pong activations, [max_tokens][H] bf16
   DecodePlan plan[3];  // per mode: layer, expert, route (pointers filled per call)
   std::string err;
@@ -58,7 +62,7 @@ bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) !
 uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
 // Shared-memory layout of the fused kernel for one mode; false if it does not fit.
-bool make_plan(const fmoe_config& c, int grid, int mode, int nstage, int max_smem, DecodePlan& P) {
+bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePlan& P) {
   memset(&P, 0, sizeof P);
   P.H = c.hidden;
   P.E = c.n_experts;
@@ -71,72 +75,104 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int nstage, int max_sme
   P.tb = tile_bytes(c.bits);
   P.cb = tile_code_bytes(c.bits);
   P.gu_tiles = c.hidden / kGroup;
-  P.gu_unit_bytes = P.gu_tiles * P.tb;
-  P.n_kr_gu = (c.hidden + 255) / 256;
-  P.teams_gu = kWarps / P.n_kr_gu;
+  P.gu_chunks = (P.gu_tiles + kChunkTiles - 1) / kChunkTiles;
+  P.dn_tiles = c.inter / kGroup;
+  P.dn_chunks = (P.dn_tiles + kChunkTiles - 1) / kChunkTiles;
   P.units_per_slot = c.inter / 8;
   P.total_units = P.n_slots * P.units_per_slot;
-  P.dn_tiles = c.inter / kGroup;
-  P.dn_job_bytes = P.dn_tiles * P.tb;
-  P.n_kr_dn = (c.inter + 255) / 256;
-  P.teams_dn = kWarps / P.n_kr_dn;
+  P.units_per_cta = (P.total_units + grid - 1) / grid;
   P.n_rb = c.hidden / 16;
   P.rb_per_cta = P.n_slots > 0 ? (P.n_rb + grid - 1) / grid : 0;
   const bool router = mode != kModeExpert;
   P.router_rows = router ? (c.n_experts + grid - 1) / grid : 0;
-  P.router_chunks = (c.hidden + 255) / 256;
-  P.nstage = P.total_units > 0 ? nstage : 1;
+  // up to 4 non-empty parts of whole 64-column groups
+  const int rgroups = c.hidden / kGroup, per_part = (rgroups + 3) / 4;
+  P.router_part_cols = per_part * kGroup;
+  P.router_parts = (rgroups + per_part - 1) / per_part;
+  const int max_tasks =
+      P.router_rows * P.router_parts + P.units_per_cta * P.gu_chunks + P.rb_per_cta * P.n_slots * P.dn_chunks;
+  if (max_tasks > kMaxTasks || P.units_per_cta > 32 || P.rb_per_cta * P.n_slots > 32 || P.router_rows > 16)
+    return false;
 
-  uint32_t off = 0;
-  P.off_ring = off;
-  P.stage_bytes = P.total_units > 0 ? (uint32_t)(P.teams_gu * P.gu_unit_bytes) : 0;
-  off = align_up(off + P.nstage * P.stage_bytes, 128);
-  P.off_down = off;
-  const uint32_t down_bytes = (uint32_t)(P.n_slots * P.rb_per_cta * P.dn_job_bytes);
-  off = align_up(off + down_bytes, 128);
-  const uint32_t router_bytes = (uint32_t)(P.router_rows * c.hidden * 2);
-  const uint32_t routed_down = P.n_slots > 1 ? (uint32_t)((P.n_slots - 1) * P.rb_per_cta * P.dn_job_bytes) : 0;
-  if (router_bytes > 0 && routed_down >= router_bytes && mode == kModeLayer) {
-    P.off_router = P.off_down + (uint32_t)(P.rb_per_cta * P.dn_job_bytes);
-  } else {
-    P.off_router = off;
-    off = align_up(off + router_bytes, 128);
+  uint32_t stage = 0;
+  if (P.total_units > 0) {
+    stage = std::max<uint32_t>(stage, (uint32_t)(std::min(kChunkTiles, P.gu_tiles) * P.tb));
+    stage = std::max<uint32_t>(stage, (uint32_t)(std::min(kChunkTiles, P.dn_tiles) * P.tb));
   }
-  P.off_zfrag = off;
-  off = align_up(off + (uint32_t)c.hidden * 2, 128);
-  P.off_zinfo = off;
-  off = align_up(off + (uint32_t)(c.hidden / kGroup) * 8, 128);
+  if (router) stage = std::max<uint32_t>(stage, (uint32_t)P.router_part_cols * 2);
+  P.stage_bytes = align_up(stage, 128);
+
+  // fixed regions after the ring
+  uint32_t off = 0;
+  uint32_t fixed = 0;
+  auto region = [&](uint32_t bytes) {
+    uint32_t o = fixed;
+    fixed = align_up(fixed + bytes, 128);
+    return o;
+  };
+  const uint32_t r_z = region((uint32_t)c.hidden * 2);
+  const uint32_t r_lg = region(router ? (uint32_t)c.n_experts * 4 : 4u);
+  const uint32_t r_zfrag = region((uint32_t)c.hidden * 2);
+  const uint32_t r_zinfo = region((uint32_t)(c.hidden / kGroup) * 8);
   P.afrag_bytes = align_up((uint32_t)c.inter * 2, 128);
   P.ainfo_bytes = align_up((uint32_t)(c.inter / kGroup) * 8, 128);
-  P.off_afrag = off;
-  off += 2 * P.afrag_bytes;
-  P.off_ainfo = off;
-  off += 2 * P.ainfo_bytes;
-  P.off_z = off;
-  off = align_up(off + std::max<uint32_t>((uint32_t)c.hidden * 2, (uint32_t)c.n_experts * 4), 128);
-  P.off_gupart = off;
-  off += 2 * kWarps * 16 * 4;
-  P.off_dnpart = off;
-  off += kWarps * 16 * 4;
-  P.off_y = off;
-  off = align_up(off + (uint32_t)(std::max(P.rb_per_cta, 1) * std::max(P.n_slots, 1) * 16 * 4), 128);
-  P.off_rpart = off;
-  off = align_up(off + (uint32_t)(std::max(P.router_rows, 1) * kWarps * 4), 128);
-  P.off_misc = off;
-  off += 128;
+  const uint32_t r_afrag = region((uint32_t)std::max(P.n_slots, 1) * P.afrag_bytes);
+  const uint32_t r_ainfo = region((uint32_t)std::max(P.n_slots, 1) * P.ainfo_bytes);
+  const uint32_t r_gupart = region((uint32_t)(std::max(P.units_per_cta, 1) * P.gu_chunks * 16 * 4));
+  const uint32_t r_dnpart = region((uint32_t)(std::max(P.rb_per_cta * P.n_slots, 1) * P.dn_chunks * 16 * 4));
+  const uint32_t r_y = region((uint32_t)(std::max(P.rb_per_cta, 1) * std::max(P.n_slots, 1) * 16 * 4));
+  const uint32_t r_tasks = region((uint32_t)kMaxTasks * 4);
+  const uint32_t r_misc = region((uint32_t)sizeof(Misc));
+  // ring: as many stages as fit (<= 64, <= tasks), each stage_bytes
+  int nstage = 0;
+  for (int ns = std::min(64, std::max(max_tasks, 1)); ns >= 1; --ns) {
+    uint32_t total = align_up((uint32_t)ns * P.stage_bytes, 128) + fixed + align_up((uint32_t)(2 * ns * 8), 128);
+    if ((int)total <= max_smem) {
+      nstage = ns;
+      break;
+    }
+  }
+  if (nstage < 1) return false;
+  // several issuing lanes (one copy instruction in flight per lane); keep the
+  // largest ring that divides evenly among 4..8 of them
+  int best_ni = 1, best_ns = nstage;
+  if (nstage >= 4) {
+    best_ns = 0;
+    for (int ni = std::min(8, nstage); ni >= 4; --ni)
+      if (nstage / ni * ni > best_ns) {
+        best_ns = nstage / ni * ni;
+        best_ni = ni;
+      }
+  } else {
+    best_ni = nstage;
+  }
+  nstage = best_ns;
+  P.n_issuers = best_ni;
+  P.nstage = nstage;
+  P.off_ring = off;
+  off = align_up((uint32_t)nstage * P.stage_bytes, 128);
+  P.off_z = off + r_z;
+  P.off_lg = off + r_lg;
+  P.off_zfrag = off + r_zfrag;
+  P.off_zinfo = off + r_zinfo;
+  P.off_afrag = off + r_afrag;
+  P.off_ainfo = off + r_ainfo;
+  P.off_gupart = off + r_gupart;
+  P.off_dnpart = off + r_dnpart;
+  P.off_y = off + r_y;
+  P.off_tasks = off + r_tasks;
+  P.off_misc = off + r_misc;
+  off += fixed;
   P.off_bar = off;
-  off += (uint32_t)(P.nstage + kMaxSlots + 1) * 8;
-  P.smem_bytes = align_up(off, 128);
+  off = align_up(off + (uint32_t)(2 * nstage * 8), 128);
+  P.smem_bytes = off;
   return (int)P.smem_bytes <= max_smem;
 }
 
 bool plan_all(fmoe_ctx* ctx, int max_smem) {
   const int modes[3] = {kModeLayer, kModeExpert, kModeRoute};
-  for (int m = 0; m < 3; ++m) {
-    bool ok = false;
-    for (int ns = 3; ns >= 2 && !ok; --ns) ok = make_plan(ctx->cfg, ctx->n_sm, modes[m], ns, max_smem, ctx->plan[m]);
-    if (!ok) return false;
-  }
+  for (int m = 0; m < 3; ++m)
+    if (!make_plan(ctx->cfg, ctx->n_sm, modes[m], max_smem, ctx->plan[m])) return false;
   return true;
 }
 
@@ -164,6 +200,10 @@ DecodePlan bind(const fmoe_ctx* ctx, int mode, int layer) {
   P.ws = ctx->hdr;
   P.ws_logits = ctx->logits;
   P.ws_a = ctx->act;
+  P.ws_asum = ctx->asum;
+  P.ws_amax = ctx->amax;
+  P.tasks = ctx->tasks + (size_t)mode * ctx->n_sm * kMaxTasks;
+  P.n_tasks = ctx->ntasks + (size_t)mode * ctx->n_sm;
   P.flags = ctx->cfg.flags;
   P.timeout_ns = (uint64_t)(ctx->cfg.wait_timeout_us ? ctx->cfg.wait_timeout_us : 1000000u) * 1000ull;
   return P;
@@ -189,6 +229,44 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 }
 
 }  // namespace
+
+namespace fmoe {
+
+// A block's ordered work list: its router row parts; the slot-0 expert's
+// gate/up K-chunks and down jobs (known before routing); then the routed
+// experts' gate/up chunks in unit order and their down jobs in slot order.
+// Routed down jobs wait for other blocks' activations, so they come last in
+// every consumer warp's queue: no gate/up chunk ever waits behind them.  The
+// slot-0 down jobs may wait, but only until the slot-0 units every block runs
+// first are done, while routed chunks cannot start anyway.
+int build_task_list(const DecodePlan& P, int cta, uint32_t* out) {
+  const int G = P.grid;
+  const int my_units = P.total_units > cta ? (P.total_units - cta + G - 1) / G : 0;
+  const int first_rb = G - 1 - cta;
+  const int my_rb = (P.n_slots > 0 && first_rb < P.n_rb) ? (P.n_rb - first_rb + G - 1) / G : 0;
+  const int my_rrows = (P.mode != kModeExpert && cta < P.E) ? (P.E - cta + G - 1) / G : 0;
+  int n = 0;
+  for (int j = 0; j < my_rrows; ++j)
+    for (int q = 0; q < P.router_parts; ++q) out[n++] = make_task(kTaskRouter, j, 0, q);
+  // the slot-0 expert (shared, or the single expert) needs no routing: its
+  // gate/up chunks and down jobs go first, ahead of every routed chunk
+  int j = 0;
+  for (; j < my_units && (cta + j * G) / P.units_per_slot == 0; ++j)
+    for (int c = 0; c < P.gu_chunks; ++c) out[n++] = make_task(kTaskGateUp, j, 0, c);
+  if (P.n_slots > 0)
+    for (int r = 0; r < my_rb; ++r)
+      for (int c = 0; c < P.dn_chunks; ++c) out[n++] = make_task(kTaskDown, r, 0, c);
+  for (; j < my_units; ++j) {
+    const int slot = (cta + j * G) / P.units_per_slot;
+    for (int c = 0; c < P.gu_chunks; ++c) out[n++] = make_task(kTaskGateUp, j, slot, c);
+  }
+  for (int d = 1; d < P.n_slots; ++d)
+    for (int r = 0; r < my_rb; ++r)
+      for (int c = 0; c < P.dn_chunks; ++c) out[n++] = make_task(kTaskDown, r, d, c);
+  return n;
+}
+
+}  // namespace fmoe
 
 extern "C" {
 
@@ -261,9 +339,17 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   // workspace: header | logits [E] | activations [kMaxSlots][I] | 2 x [max_tokens][H] bf16
   size_t off = 256;
   size_t off_logits = off;
-  off += ((size_t)c.n_experts * 4 + 255) / 256 * 256;
+  off += ((size_t)c.n_experts * 8 + 255) / 256 * 256;
   size_t off_act = off;
-  off += ((size_t)kMaxSlots * c.inter * 4 + 255) / 256 * 256;
+  off += ((size_t)kMaxSlots * c.inter * 8 + 255) / 256 * 256;
+  size_t off_asum = off;
+  off += ((size_t)kMaxSlots * (c.inter / 8) * 8 + 255) / 256 * 256;
+  size_t off_amax = off;
+  off += 256;
+  size_t off_tasks = off;
+  off += ((size_t)3 * ctx->n_sm * kMaxTasks * 4 + 255) / 256 * 256;
+  size_t off_ntasks = off;
+  off += ((size_t)3 * ctx->n_sm * 4 + 255) / 256 * 256;
   size_t off_stack = off;
   size_t stack_bytes = ((size_t)std::max(c.max_tokens, 1) * c.hidden * 2 + 255) / 256 * 256;
   off += 2 * stack_bytes;
@@ -276,13 +362,29 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   }
   uint8_t* base = static_cast<uint8_t*>(ctx->ws);
   ctx->hdr = reinterpret_cast<WsHeader*>(base);
-  ctx->logits = reinterpret_cast<float*>(base + off_logits);
-  ctx->act = reinterpret_cast<float*>(base + off_act);
+  ctx->logits = reinterpret_cast<uint64_t*>(base + off_logits);
+  ctx->act = reinterpret_cast<uint64_t*>(base + off_act);
+  ctx->asum = reinterpret_cast<uint64_t*>(base + off_asum);
+  ctx->amax = reinterpret_cast<uint64_t*>(base + off_amax);
+  ctx->tasks = reinterpret_cast<uint32_t*>(base + off_tasks);
+  ctx->ntasks = reinterpret_cast<int32_t*>(base + off_ntasks);
   ctx->stack_buf[0] = reinterpret_cast<uint16_t*>(base + off_stack);
   ctx->stack_buf[1] = reinterpret_cast<uint16_t*>(base + off_stack + stack_bytes);
   cudaStream_t st = (cudaStream_t)stream;
   e = cudaMemsetAsync(ctx->ws, 0, ctx->ws_bytes, st);
   if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "workspace clear"));
+  {
+    std::vector<uint32_t> tl((size_t)3 * ctx->n_sm * kMaxTasks, 0u);
+    std::vector<int32_t> nt((size_t)3 * ctx->n_sm, 0);
+    for (int m = 0; m < 3; ++m)
+      for (int b = 0; b < ctx->n_sm; ++b)
+        nt[(size_t)m * ctx->n_sm + b] =
+            build_task_list(ctx->plan[m], b, tl.data() + ((size_t)m * ctx->n_sm + b) * kMaxTasks);
+    e = cudaMemcpyAsync(ctx->tasks, tl.data(), tl.size() * 4, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ctx->ntasks, nt.data(), nt.size() * 4, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "task table upload"));
+  }
 
   // In-place repack, canonical -> packed, through a bounded staging buffer.
   const size_t blob = (size_t)expert_bytes(c.hidden, c.inter, c.bits);
@@ -450,7 +552,9 @@ fmoe_status fmoe_poll_status(fmoe_ctx* ctx, void* stream, uint32_t* device_statu
   if (e != cudaSuccess) return cuda_fail(ctx, e, "status read");
   if (device_status) *device_status = h.status;
   if (h.status != 0) {
-    e = cudaMemsetAsync(ctx->hdr, 0, sizeof(WsHeader), st);
+    // only the status word: the epoch must keep increasing so that values
+    // tagged by earlier launches are never mistaken for new ones
+    e = cudaMemsetAsync(&ctx->hdr->status, 0, sizeof(uint32_t), st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "status reset");
     return fail(ctx, FMOE_ERR_TIMEOUT, "device-side wait timed out (status 0x%x)", h.status);

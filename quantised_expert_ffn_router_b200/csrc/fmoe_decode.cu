@@ -1,26 +1,35 @@
 // fmoe_decode.cu -- fused single-token mixture-of-experts layer for sm_100a.
 //
-// One cooperative launch, one 512-thread block per SM, runs the whole decode
-// step the Flash-MoE pages split over CMD2, the CPU and CMD3 (page 5 "How the
-// SSD expert streaming pipeline works"):
-//   1. optional RMSNorm of the layer input (every block, redundantly);
-//   2. router GEMV: block b owns router rows b, b+G, ...; logits go to a global
-//      workspace and a release-counter announces them;
-//   3. softmax + top-K: every block waits (bounded) for all logits and selects
-//      the same K experts itself, so no second launch is needed;
-//   4. SwiGLU experts: the K routed experts and the shared expert are cut into
-//      units of 8 gate rows + 8 up rows over the full hidden width; units are
-//      striped over all blocks, their weights stream HBM -> shared memory by
-//      bulk-async (TMA) copies into a ring of stages, and each warp dequantises
-//      its 256-column slice into mma.sync fragments (codes are exact in fp16,
-//      the per-group scale and bias are applied as s*sum(q*x) + b*sum(x) after
-//      each 64-column group);  a = silu(g)*u goes to the workspace and a
-//      per-expert counter is released;
-//   5. down projection: block b owns output row blocks G-1-b, 2G-1-b, ... for
-//      every expert, preloads those weight tiles at the start, waits (bounded)
-//      for an expert's activations to be complete and folds them in;
-//   6. combine: h_out = h_in + y_shared + sum_k w_k y_k in fp32, one bf16
-//      rounding, written by the block that owns the rows (no atomics).
+// One cooperative launch, one block per SM, runs the whole decode step that the
+// Flash-MoE pages split over CMD2, the CPU and CMD3 (page 5 "How the SSD expert
+// streaming pipeline works"): optional RMSNorm, router GEMV, softmax + top-K,
+// the K routed and the shared SwiGLU experts with inline dequantisation, and the
+// weighted combine into the residual.
+//
+// Work split.  Every block owns (a) router rows b, b+G, ..., (b) gate/up units
+// (8 gate + 8 up rows over the full hidden width) u = b, b+G, ... striped over
+// the flattened list [shared expert | routed expert 1 | ... | routed expert K],
+// (c) output row blocks G-1-b, 2G-1-b, ... of every expert's down projection, so
+// the combine is local and needs no atomics.  These become an ordered list of
+// tasks of at most 16 tiles each (a router row, a 1024-column K-chunk of a
+// unit, a down job).
+//
+// Roles.  One producer warp walks the list and streams each task's weights
+// HBM -> shared memory with bulk-async (TMA) copies into a ring of stages
+// (full/empty mbarriers); it also waits (bounded) for every block's router
+// rows and runs softmax + top-K itself before the first task that needs a
+// routed expert.  Sixteen consumer warps take tasks round-robin and never wait
+// for each other: K-chunks of a unit are summed by whichever warp finishes
+// last (shared-memory counter, fixed order), which writes a = silu(g)*u and
+// publishes the unit with a release counter; a down job waits (bounded) for its
+// expert's activations to be published by every block, turns them into
+// fragments once per block and reduces its rows.
+//
+// Inner loop.  A tile is 16 rows x 64 columns (one quantisation group per
+// row); its codes go into mma.sync fragments exactly (lop3 into the mantissa
+// of 1024, sub.f16x2), the input is a power-of-two-scaled fp16 fragment, the
+// tensor pipe accumulates sum(q*x) in fp32, and s*sum(q*x) + b*sum(x) folds
+// in the group's scale and bias.
 // Every wait is bounded by %globaltimer; on a timeout the block records a status
 // bit, drains its outstanding copies and leaves.
 #include <cuda_bf16.h>
@@ -59,14 +68,6 @@ __device__ __forceinline__ uint64_t gtimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
-}
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
-  asm volatile("fence.acq_rel.gpu;\n red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t c) {
   uint32_t d;
@@ -145,74 +146,118 @@ __device__ __forceinline__ void tile_dot(const uint8_t* tile, const uint2 (&bf)[
   acc1 = fmaf(bf16lo(sb.y) * info.x, c[2], fmaf(bf16hi(sb.y), info.y, acc1));
 }
 
-// Input vector -> fp16 B fragments.  Group G of 64 values is scaled by 2^sh so
-// its largest magnitude lies in [2^14, 2^15); within slice s of the group the
-// values multiplying codes stored as 4^k * q are divided by 4^k.  Fragment
-// word for (group G, lane column t, slice s, half which) sits at uint32 index
-// ((G*4 + t)*4 + s)*2 + which; info[G] = (2^-sh, sum of the group's values).
-template <typename Load>
-__device__ __forceinline__ void build_frags(Load load, int C, int bits, uint32_t* frag, float2* info, int tid) {
-  const int lane = tid & 31;
-  for (int base = 0; base < C / 2; base += kThreads) {
-    int p = base + tid;
-    if (p - lane + 32 > C / 2) break;  // warp-uniform (C is a multiple of 64)
-    float v0 = load(2 * p), v1 = load(2 * p + 1);
-    uint32_t m = max(__float_as_uint(fabsf(v0)), __float_as_uint(fabsf(v1)));
-    m = __reduce_max_sync(0xffffffffu, m);
-    float sum = v0 + v1;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    int e = (int)((m >> 23) & 0xFF) - 127;  // exponent of the group maximum
-    int sh = (m == 0) ? 0 : 14 - max(e, -126);
-    sh = min(sh, 126);
-    int k = (2 * p) % kGroup, s = k / 16, kk = k % 16, which = kk / 8, t = (kk % 8) / 2;
-    int fs = (bits == 4) ? (which ? 4 : 0) : ((s & 1) ? 4 : 0) + (which ? 2 : 0);
-    float scl = exp2i(sh - fs);
-    __half2 h2 = __floats2half2_rn(v0 * scl, v1 * scl);
-    int G = (2 * p) / kGroup;
-    frag[((G * 4 + t) * 4 + s) * 2 + which] = *reinterpret_cast<uint32_t*>(&h2);
-    if (lane == 0) info[G] = make_float2(exp2i(-sh), sum);
-  }
-}
 
-__device__ __forceinline__ void load_frags(const uint32_t* frag, const float2* info, int kr, int n_groups, int lane,
-                                           uint2 (&bf)[4][4], float2 (&inf)[4]) {
-  const int t = lane & 3;
-#pragma unroll
-  for (int gg = 0; gg < 4; ++gg) {
-    int G = kr * 4 + gg;
-    if (G < n_groups) {
-      const uint4* src = reinterpret_cast<const uint4*>(frag + ((G * 4 + t) * 4) * 2);
-      uint4 x = src[0], y = src[1];
-      bf[gg][0] = make_uint2(x.x, x.y);
-      bf[gg][1] = make_uint2(x.z, x.w);
-      bf[gg][2] = make_uint2(y.x, y.y);
-      bf[gg][3] = make_uint2(y.z, y.w);
-      inf[gg] = info[G];
-    } else {
-      inf[gg] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int s = 0; s < 4; ++s) bf[gg][s] = make_uint2(0u, 0u);
-    }
-  }
+// Publishes {value, tag} with an atomic exchange: atomics are performed at L2,
+// so other SMs see the word within about a microsecond, whereas plain stores
+// were measured to linger for several microseconds under load.
+__device__ __forceinline__ void st_tagged(uint64_t* p, float v, uint32_t tag) {
+  const uint64_t w = (uint64_t)__float_as_uint(v) | ((uint64_t)tag << 32);
+  uint64_t old;
+  asm volatile("atom.relaxed.gpu.global.exch.b64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(w) : "memory");
 }
+__device__ __forceinline__ uint64_t ld_tagged(const uint64_t* p) {
+  uint64_t w;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+// Two tagged words (16-byte aligned); volatile so a polling loop re-reads them.
+__device__ __forceinline__ ulonglong2 ld_tagged2(const uint64_t* p) {
+  ulonglong2 w;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(w.x), "=l"(w.y) : "l"(p) : "memory");
+  return w;
+}
+__device__ __forceinline__ void atom_max_u64(uint64_t* p, uint64_t v) {
+  asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ float tagged_value(uint64_t w) { return __uint_as_float((uint32_t)w); }
+__device__ __forceinline__ uint32_t tagged_tag(uint64_t w) { return (uint32_t)(w >> 32); }
 
-// Bounded waits: true when satisfied, false after the time limit.
-__device__ __forceinline__ bool wait_counter(const uint32_t* p, uint32_t target, uint64_t limit) {
-  uint64_t t0 = gtimer();
+__device__ __forceinline__ void red_relaxed_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Bounded spin until a published count reaches its target (a hint only: the
+// values it counts carry their own tags and are re-checked by the reader).
+__device__ __forceinline__ bool wait_count(const uint32_t* p, uint32_t target, uint64_t limit,
+                                           const volatile int* abort_flag) {
+  const uint64_t t0 = gtimer();
   for (uint32_t it = 0;; ++it) {
-    if (ld_acquire(p) >= target) return true;
-    if ((it & 15) == 15 && gtimer() - t0 > limit) return false;
+    if (ld_relaxed(p) >= target) return true;
+    if ((it & 7) == 7 && (*abort_flag || gtimer() - t0 > limit)) return false;
+    __nanosleep(128);  // leave issue slots to warps with work
   }
 }
-__device__ __forceinline__ bool wait_mbar(uint32_t bar, uint32_t parity, uint64_t limit) {
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// fp16 B fragments of one 64-value group, built by one warp (lane holds values
+// 2*lane and 2*lane+1 of the group).  The group is scaled by 2^sh so its
+// largest magnitude lies in [2^14, 2^15); within slice s the values multiplying
+// codes stored as 4^k * q are divided by 4^k.  Fragment word for (group G, lane
+// column t, slice s, half which) sits at uint32 index ((G*4 + t)*4 + s)*2 +
+// which; info[G] = (2^-sh, sum of the group's values).
+__device__ __forceinline__ void frag_group(float v0, float v1, int G, int bits, uint32_t* frag, float2* info,
+                                           int lane) {
+  uint32_t m = max(__float_as_uint(fabsf(v0)), __float_as_uint(fabsf(v1)));
+  m = __reduce_max_sync(0xffffffffu, m);
+  float sum = v0 + v1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const int e = (int)((m >> 23) & 0xFF) - 127;  // exponent of the group maximum
+  int sh = (m == 0) ? 0 : 14 - max(e, -126);
+  sh = min(sh, 126);
+  const int k = 2 * lane, s = k / 16, kk = k % 16, which = kk / 8, t = (kk % 8) / 2;
+  const int fs = (bits == 4) ? (which ? 4 : 0) : ((s & 1) ? 4 : 0) + (which ? 2 : 0);
+  const float scl = exp2i(sh - fs);
+  __half2 h2 = __floats2half2_rn(v0 * scl, v1 * scl);
+  frag[((G * 4 + t) * 4 + s) * 2 + which] = *reinterpret_cast<uint32_t*>(&h2);
+  if (lane == 0) info[G] = make_float2(exp2i(-sh), sum);
+}
+
+// Dot products of n consecutive tiles (groups G0..G0+n-1 of the input) with the
+// fragments in shared memory.
+template <int BITS>
+__device__ __forceinline__ void chunk_dot(const uint8_t* tiles, int n, const uint32_t* frag, const float2* info,
+                                          int G0, int lane, float& acc0, float& acc1) {
+  constexpr int TB = 16 * kGroup * BITS / 8 + 64;
+  const int t = lane & 3;
+#pragma unroll 4
+  for (int tt = 0; tt < n; ++tt) {
+    const int G = G0 + tt;
+    const uint4* fp = reinterpret_cast<const uint4*>(frag + ((G * 4 + t) * 4) * 2);
+    const uint4 x = fp[0], y = fp[1];
+    const uint2 bf[4] = {make_uint2(x.x, x.y), make_uint2(x.z, x.w), make_uint2(y.x, y.y), make_uint2(y.z, y.w)};
+    tile_dot<BITS>(tiles + tt * TB, bf, info[G], lane, acc0, acc1);
+  }
+}
+
+// Bounded waits; they also give up when another warp of the block aborted.
+__device__ __forceinline__ bool wait_mbar(uint32_t bar, uint32_t parity, uint64_t limit,
+                                          const volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = gtimer();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (gtimer() - t0 > limit) return false;
+    if (*abort_flag || gtimer() - t0 > limit) return false;
   }
 }
+__device__ __forceinline__ bool wait_flag(const volatile int* f, int value, uint64_t limit,
+                                          const volatile int* abort_flag) {
+  uint64_t t0 = gtimer();
+  for (uint32_t it = 0;; ++it) {
+    if (*f == value) return true;
+    if ((it & 15) == 15 && (*abort_flag || gtimer() - t0 > limit)) return false;
+    __nanosleep(64);  // leave issue slots to warps with work
+  }
+}
+
+
 
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodePlan P) {
@@ -220,363 +265,531 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x, G = P.grid;
   constexpr int TB = 16 * kGroup * BITS / 8 + 64;
-
-  const uint32_t bar_base = smem_u32(smem + P.off_bar);
-  const uint32_t bar_router = bar_base + 8u * (P.nstage + kMaxSlots);
-  int* slot_e = reinterpret_cast<int*>(smem + P.off_misc);
-  float* slot_w = reinterpret_cast<float*>(smem + P.off_misc + 64);
+  Misc* misc = reinterpret_cast<Misc*>(smem + P.off_misc);
+  volatile int* abort_flag = &misc->abort;
+  uint32_t* tasks = reinterpret_cast<uint32_t*>(smem + P.off_tasks);
+  const uint32_t bar_full = smem_u32(smem + P.off_bar);
+  const uint32_t bar_empty = bar_full + 8u * P.nstage;
+  uint16_t* zs = reinterpret_cast<uint16_t*>(smem + P.off_z);
+  uint32_t* zfrag = reinterpret_cast<uint32_t*>(smem + P.off_zfrag);
+  float2* zinfo = reinterpret_cast<float2*>(smem + P.off_zinfo);
   float* gupart = reinterpret_cast<float*>(smem + P.off_gupart);
   float* dnpart = reinterpret_cast<float*>(smem + P.off_dnpart);
   float* ys = reinterpret_cast<float*>(smem + P.off_y);
-  float* rpart = reinterpret_cast<float*>(smem + P.off_rpart);
-  uint16_t* zs = reinterpret_cast<uint16_t*>(smem + P.off_z);
+  const uint64_t limit = P.timeout_ns;
 
   // this block's share of the work
-  const int my_units = P.total_units > cta ? (P.total_units - cta + G - 1) / G : 0;
-  const int my_stages = (my_units + P.teams_gu - 1) / P.teams_gu;
   const int first_rb = G - 1 - cta;
   const int my_rb = (P.n_slots > 0 && first_rb < P.n_rb) ? (P.n_rb - first_rb + G - 1) / G : 0;
   const bool has_router = P.mode != kModeExpert;
-  const int my_rrows = (has_router && cta < P.E) ? (P.E - cta + G - 1) / G : 0;
-  const uint64_t limit = P.timeout_ns;
+  float h_res = 0.f;  // residual input of the row this thread combines
 
-  auto unit_of = [&](int j) { return cta + j * G; };
-  // Units of a stage are increasing, so its last unit has its largest slot.
-  auto stage_max_slot = [&](int s) {
-    int j = min((s + 1) * P.teams_gu, my_units) - 1;
-    return unit_of(j) / P.units_per_slot;
-  };
-
-  if (tid == 0) {
-    for (int i = 0; i < P.nstage + kMaxSlots + 1; ++i) mbar_init(bar_base + 8u * i, 1);
+  // ---------------------------------------------------------------- set-up
+  if (warp == 0) {
+    for (int i = lane; i < 2 * P.nstage; i += 32) mbar_init(bar_full + 8u * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n fence.proxy.async.shared::cta;" ::: "memory");
-    if (P.mode == kModeLayer) { slot_e[0] = P.E; slot_w[0] = 1.f; }
-    if (P.mode == kModeExpert) { slot_e[0] = P.expert_id; slot_w[0] = 1.f; }
+  } else if (warp == 1) {
+    if (lane < 16) {
+      misc->rcnt[lane] = 0;
+      misc->aflag[lane] = 0;
+      misc->slot_e[lane] = (lane == 0) ? (P.mode == kModeExpert ? P.expert_id : P.E) : 0;
+      misc->slot_w[lane] = (lane == 0) ? 1.f : 0.f;
+    }
+    misc->unit_cnt[lane] = 0;
+    misc->dn_cnt[lane] = 0;
+    misc->last_task[lane] = -1;
+    misc->last_task[lane + 32] = -1;
+    if (lane == 0) misc->abort = 0;
+  } else if (warp == 2) {
+    // this block's ordered task list, global -> shared
+    const uint32_t* src = P.tasks + (int64_t)cta * kMaxTasks;
+    uint32_t v[kMaxTasks / 32];
+#pragma unroll
+    for (int k = 0; k < kMaxTasks / 32; ++k) v[k] = src[k * 32 + lane];
+#pragma unroll
+    for (int k = 0; k < kMaxTasks / 32; ++k) tasks[k * 32 + lane] = v[k];
+    if (lane == 0) misc->n_tasks = P.n_tasks[cta];
   }
   __syncthreads();
-
-  // ---------------------------------------------------------------- producer (thread 0)
-  int issued = 0;       // stages issued, in order
-  uint32_t dn_issued = 0;
-  bool router_issued = false;
-  auto issue_stage = [&](int s) {
-    const int buf = s % P.nstage;
-    const uint32_t dst = smem_u32(smem + P.off_ring + (uint32_t)buf * P.stage_bytes);
-    const uint32_t bar = bar_base + 8u * buf;
-    int n = min(P.teams_gu, my_units - s * P.teams_gu);
-    mbar_expect_tx(bar, (uint32_t)(n * P.gu_unit_bytes));
-    for (int tau = 0; tau < n; ++tau) {
-      int u = unit_of(s * P.teams_gu + tau);
-      int slot = u / P.units_per_slot, rb = u % P.units_per_slot;
-      const uint8_t* src = P.experts + (int64_t)slot_e[slot] * P.blob_bytes + (int64_t)rb * P.gu_unit_bytes;
-      tma_load(dst + (uint32_t)(tau * P.gu_unit_bytes), src, (uint32_t)P.gu_unit_bytes, bar);
-    }
-  };
-  auto issue_down = [&](int slot) {
-    if (my_rb == 0) return;
-    const uint32_t bar = bar_base + 8u * (P.nstage + slot);
-    mbar_expect_tx(bar, (uint32_t)(my_rb * P.dn_job_bytes));
-    const uint8_t* ex = P.experts + (int64_t)slot_e[slot] * P.blob_bytes + packed_gu_bytes(P.H, P.I, BITS);
-    for (int j = 0; j < my_rb; ++j) {
-      int rbg = first_rb + j * G;
-      uint32_t dst = smem_u32(smem + P.off_down + (uint32_t)((slot * P.rb_per_cta + j) * P.dn_job_bytes));
-      tma_load(dst, ex + (int64_t)rbg * P.dn_job_bytes, (uint32_t)P.dn_job_bytes, bar);
-    }
-    dn_issued |= 1u << slot;
-  };
-  auto issue_ready_stages = [&](int upto, bool routed) {
-    while (issued < my_stages && issued < upto && (routed || stage_max_slot(issued) == 0)) issue_stage(issued++);
-  };
-
-  if (tid == 0) {
-    if (my_rrows > 0) {
-      mbar_expect_tx(bar_router, (uint32_t)(my_rrows * P.H * 2));
-      for (int j = 0; j < my_rrows; ++j)
-        tma_load(smem_u32(smem + P.off_router + (uint32_t)(j * P.H * 2)), P.router_w + (int64_t)(cta + j * G) * P.H,
-                 (uint32_t)(P.H * 2), bar_router);
-      router_issued = true;
-    }
-    if (P.n_slots > 0) issue_down(0);
-    issue_ready_stages(P.nstage, P.mode == kModeExpert);
-  }
-
-  // Weights above do not depend on earlier kernels; everything below may.
-  if (P.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int n_tasks = misc->n_tasks;
+  // The next launch may start its weight prefetch as soon as blocks retire.
   if (P.pdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  int abort = 0;
-  int consumed = 0;         // stages consumed
-  bool router_consumed = false;
-  uint32_t dn_consumed = 0;
-
-  // ---------------------------------------------------------------- input: z and its fragments
-  {
-    const uint16_t* h = P.h_in;
-    if (P.norm_w != nullptr) {
-      float ss = 0.f;
-      for (int i = tid; i < P.H; i += kThreads) {
-        float v = bf16f(h[i]);
-        ss = fmaf(v, v, ss);
-      }
+  if (warp == kConsumerWarps) {
+    // ============================================================ producer warp
+    bool routed = false;
+    bool waited_grid = false;
+    auto do_routing = [&]() {
+      if (P.pdl && !waited_grid) asm volatile("griddepcontrol.wait;" ::: "memory");
+      waited_grid = true;
+      // Poll the tagged logits until every router row of this launch is
+      // published; each lane keeps experts lane, lane+32, ... in registers
+      // (up to 512 experts; beyond that the values are staged in shared memory).
+      const uint32_t tag = *reinterpret_cast<volatile uint32_t*>(&P.ws->epoch) + 1u;
+      constexpr int kRegE = 16;
+      const bool in_regs = P.E <= 32 * kRegE;
+      float vals[kRegE];
+      float* lg = reinterpret_cast<float*>(smem + P.off_lg);
+      const uint64_t t0 = gtimer();
+      for (;;) {
+        bool mine = true;
+        for (int base = 0; base < P.E; base += 32 * kRegE) {
+          uint64_t v[kRegE];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (lane == 0) dnpart[warp] = ss;
-      __syncthreads();
-      float tot = 0.f;
-      for (int w = 0; w < kWarps; ++w) tot += dnpart[w];
-      const float r = 1.0f / sqrtf(tot / (float)P.H + P.eps);
-      for (int i = tid; i < P.H; i += kThreads) zs[i] = f2bf16(bf16f(h[i]) * r * bf16f(P.norm_w[i]));
-    } else {
-      for (int i = tid; i < P.H; i += kThreads) zs[i] = h[i];
-    }
-    for (int i = tid; i < P.router_rows * kWarps; i += kThreads) rpart[i] = 0.f;
-    __syncthreads();
-    if (P.n_slots > 0)
-      build_frags([&](int i) { return bf16f(zs[i]); }, P.H, BITS, reinterpret_cast<uint32_t*>(smem + P.off_zfrag),
-                  reinterpret_cast<float2*>(smem + P.off_zinfo), tid);
-    __syncthreads();
-  }
-
-  // ---------------------------------------------------------------- router GEMV
-  if (my_rrows > 0) {
-    if (!wait_mbar(bar_router, 0, limit)) {
-      abort = 1;
-      atomicOr(&P.ws->status, kStatusTimeoutTma);
-    }
-    const int pairs = my_rrows * P.router_chunks;
-    for (int p = warp; p < pairs && !abort; p += kWarps) {
-      int j = p / P.router_chunks, ch = p % P.router_chunks;
-      int col = ch * 256 + lane * 8;
-      float acc = 0.f;
-      if (col < P.H) {
-        uint4 w = *reinterpret_cast<const uint4*>(smem + P.off_router + (uint32_t)(j * P.H * 2 + col * 2));
-        uint4 z = *reinterpret_cast<const uint4*>(zs + col);
-        acc = fmaf(bf16lo(w.x), bf16lo(z.x), acc);
-        acc = fmaf(bf16hi(w.x), bf16hi(z.x), acc);
-        acc = fmaf(bf16lo(w.y), bf16lo(z.y), acc);
-        acc = fmaf(bf16hi(w.y), bf16hi(z.y), acc);
-        acc = fmaf(bf16lo(w.z), bf16lo(z.z), acc);
-        acc = fmaf(bf16hi(w.z), bf16hi(z.z), acc);
-        acc = fmaf(bf16lo(w.w), bf16lo(z.w), acc);
-        acc = fmaf(bf16hi(w.w), bf16hi(z.w), acc);
-      }
+          for (int k = 0; k < kRegE; ++k) {
+            const int i = base + k * 32 + lane;
+            v[k] = i < P.E ? ld_tagged(P.ws_logits + i) : 0ull;
+          }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) rpart[j * kWarps + warp] = acc;
-    }
-    router_consumed = true;
-  }
-  abort = __syncthreads_or(abort);
-  if (!abort && tid < my_rrows) {
-    float l = 0.f;
-    for (int w = 0; w < kWarps; ++w) l += rpart[tid * kWarps + w];
-    int e = cta + tid * G;
-    if (P.router_bias) l += P.router_bias[e];
-    P.ws_logits[e] = l;
-  }
-  __syncthreads();
-  if (tid == 0 && has_router && !abort && !(P.flags & FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE))
-    red_release_add(&P.ws->router_arrive, 1u);
-
-  // ---------------------------------------------------------------- routing (softmax + top-K)
-  bool routed = (P.mode == kModeExpert);
-  auto do_routing = [&]() {
-    if (tid == 0 && !wait_counter(&P.ws->router_arrive, (uint32_t)G, limit)) {
-      atomicOr(&P.ws->status, kStatusTimeoutRouter);
-      abort = 1;
-    }
-    abort = __syncthreads_or(abort);
-    if (abort) return;
-    float* lg = reinterpret_cast<float*>(smem + P.off_z);  // z no longer needed
-    if (warp == 0) {
-      for (int i = lane; i < P.E; i += 32) {
-        float v = __ldcg(P.ws_logits + i);
-        lg[i] = (v != v) ? -INFINITY : v;
+          for (int k = 0; k < kRegE; ++k) {
+            const int i = base + k * 32 + lane;
+            float f = -INFINITY;
+            if (i < P.E) {
+              mine = mine && tagged_tag(v[k]) == tag;
+              f = tagged_value(v[k]);
+              f = (f != f) ? -INFINITY : f;
+              if (!in_regs) lg[i] = f;
+            }
+            vals[k] = f;
+          }
+        }
+        if (__all_sync(0xffffffffu, mine)) break;
+        __nanosleep(32);
+        if (__any_sync(0xffffffffu, *abort_flag != 0 || gtimer() - t0 > limit)) {
+          if (lane == 0) {
+            atomicOr(&P.ws->status, kStatusTimeoutRouter);
+            *abort_flag = 1;
+          }
+          return false;
+        }
       }
       __syncwarp();
-      float top[kMaxTopK];
-      int sel[kMaxTopK];
+      // K rounds of warp arg-max (ties: lower index).  Each lane keeps the best
+      // of its own values; a round is two warp reductions (max of an
+      // order-preserving key, then min index among lanes holding it) and only
+      // the winning lane rescans.  Lane k keeps result k in scalars.
+      float my_top = -INFINITY;
+      int my_sel = 0;
+      float lb = -INFINITY;
+      int li = P.E;
+      auto rescan = [&]() {
+        lb = -INFINITY;
+        li = P.E;
+        if (in_regs) {
+#pragma unroll
+          for (int kk = 0; kk < kRegE; ++kk) {
+            const int i = kk * 32 + lane;
+            const bool better = i < P.E && vals[kk] == vals[kk] && (li == P.E || vals[kk] > lb);
+            lb = better ? vals[kk] : lb;
+            li = better ? i : li;
+          }
+        } else {
+          for (int i = lane; i < P.E; i += 32) {
+            const float v = lg[i];
+            if (v == v && (li == P.E || v > lb)) { lb = v; li = i; }
+          }
+        }
+      };
+      rescan();
+#pragma unroll 1
       for (int k = 0; k < P.K; ++k) {
-        float bv = -INFINITY;
-        int bi = P.E;
-        for (int i = lane; i < P.E; i += 32) {
-          float v = lg[i];
-          if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+        uint32_t key = 0u;  // below every real entry
+        if (li < P.E) {
+          const uint32_t u = __float_as_uint(lb);
+          key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
         }
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        const uint32_t win = __reduce_min_sync(0xffffffffu, (key == kmax && li < P.E) ? (uint32_t)li : 0xFFFFFFFFu);
+        const int bi = win < (uint32_t)P.E ? (int)win : 0;
+        const float bv = __shfl_sync(0xffffffffu, lb, bi & 31);
+        if (lane == k) { my_top = bv; my_sel = bi; }
+        if (lane == (bi & 31) && win < (uint32_t)P.E) {
+          // taken entries become NaN (loaded NaNs were turned into -inf), so
+          // the rescan skips them even among -inf ties
+          if (in_regs) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-          if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            for (int kk = 0; kk < kRegE; ++kk) vals[kk] = (kk * 32 + lane == bi) ? __int_as_float(0x7fc00000) : vals[kk];
+          } else {
+            lg[bi] = __int_as_float(0x7fc00000);
+          }
+          rescan();
         }
-        if (bi >= P.E) bi = 0;  // only when every remaining logit is NaN/-inf
-        top[k] = bv;
-        sel[k] = bi;
-        __syncwarp();
-        if (lane == 0) lg[bi] = -INFINITY;
         __syncwarp();
       }
-      if (lane == 0) {
-        float den = 0.f;
-        float ex[kMaxTopK];
-        for (int k = 0; k < P.K; ++k) { ex[k] = expf(top[k] - top[0]); den += ex[k]; }
-        for (int k = 0; k < P.K; ++k) {
-          float w = ex[k] / den;
-          if (P.mode == kModeLayer) { slot_e[1 + k] = sel[k]; slot_w[1 + k] = w; }
-          if (cta == 0 && P.idx_out) P.idx_out[k] = sel[k];
-          if (cta == 0 && P.w_out) P.w_out[k] = w;
-        }
-      }
-    }
-    __syncthreads();
-    if (tid == 0) {
-      for (int s = 1; s < P.n_slots; ++s) issue_down(s);
-      issue_ready_stages(consumed + P.nstage, true);
-    }
-  };
-
-  // ---------------------------------------------------------------- down projections of one slot
-  const int n_ig = P.I / kGroup;
-  auto do_downs = [&](int d) {
-    if (tid == 0 && !wait_counter(&P.ws->h_arrive[d], (uint32_t)P.units_per_slot, limit)) {
-      atomicOr(&P.ws->status, kStatusTimeoutH);
-      abort = 1;
-    }
-    if (my_rb > 0 && !wait_mbar(bar_base + 8u * (P.nstage + d), 0, limit)) {
-      abort = 1;
-      atomicOr(&P.ws->status, kStatusTimeoutTma);
-    }
-    abort = __syncthreads_or(abort);
-    if (abort) return;
-    dn_consumed |= 1u << d;
-    uint32_t* af = reinterpret_cast<uint32_t*>(smem + P.off_afrag + (uint32_t)(d & 1) * P.afrag_bytes);
-    float2* ai = reinterpret_cast<float2*>(smem + P.off_ainfo + (uint32_t)(d & 1) * P.ainfo_bytes);
-    const float* act = P.ws_a + (int64_t)d * P.I;
-    build_frags([&](int i) { return __ldcg(act + i); }, P.I, BITS, af, ai, tid);
-    __syncthreads();
-    const int kr = warp % P.n_kr_dn, team = warp / P.n_kr_dn;
-    if (team < P.teams_dn) {
-      uint2 bf[4][4];
-      float2 inf[4];
-      load_frags(af, ai, kr, n_ig, lane, bf, inf);
-      for (int job = team; job < my_rb; job += P.teams_dn) {
-        const uint8_t* base = smem + P.off_down + (uint32_t)((d * P.rb_per_cta + job) * P.dn_job_bytes);
-        float acc0 = 0.f, acc1 = 0.f;
+      // renormalised weights over the K selected: p_k / sum_j p_j = e^(l_k - l_0) / sum_j e^(l_j - l_0)
+      const float top0 = __shfl_sync(0xffffffffu, my_top, 0);
+      const float ex = lane < P.K ? expf(my_top - top0) : 0.f;
+      float den = ex;
 #pragma unroll
-        for (int tt = 0; tt < 4; ++tt)
-          if (kr * 4 + tt < P.dn_tiles) tile_dot<BITS>(base + (kr * 4 + tt) * TB, bf[tt], inf[tt], lane, acc0, acc1);
-        if ((lane & 3) == 0) {
-          dnpart[warp * 16 + (lane >> 2)] = acc0;
-          dnpart[warp * 16 + 8 + (lane >> 2)] = acc1;
-        }
-        if (P.n_kr_dn > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(P.n_kr_dn * 32) : "memory");
-        else __syncwarp();
-        if (kr == 0 && lane < 16) {
-          float y = 0.f;
-          for (int k = 0; k < P.n_kr_dn; ++k) y += dnpart[(team * P.n_kr_dn + k) * 16 + lane];
-          ys[(job * P.n_slots + d) * 16 + lane] = y;
-        }
-        if (P.n_kr_dn > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(P.n_kr_dn * 32) : "memory");
-        else __syncwarp();
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      if (lane < P.K) {
+        const float w = ex / den;
+        if (P.mode == kModeLayer) { misc->slot_e[1 + lane] = my_sel; misc->slot_w[1 + lane] = w; }
+        if (cta == 0 && P.idx_out) P.idx_out[lane] = my_sel;
+        if (cta == 0 && P.w_out) P.w_out[lane] = w;
+      }
+      __syncwarp();
+      return true;
+    };
+
+    // Copies are issued by n_issuers lanes at once (one bulk copy in flight per
+    // lane, each lane refilling only its own stages), in rounds of n_issuers
+    // consecutive tasks.  Within a round, tasks that need no routing go first,
+    // so a round holding this block's own router rows never waits on routing.
+    const int NI = P.n_issuers;
+    auto issue = [&](int i, uint32_t t) -> int {
+      int s, fill;
+      task_stage(P.nstage, NI, i, s, fill);
+      if (fill > 0 && !wait_mbar(bar_empty + 8u * s, (uint32_t)((fill - 1) & 1), limit, abort_flag)) {
+        if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutTma);
+        *abort_flag = 1;
+        return 0;
+      }
+      const uint32_t dst = smem_u32(smem + P.off_ring + (uint32_t)s * P.stage_bytes);
+      const void* src;
+      uint32_t bytes;
+      const uint32_t ty = task_type(t), idx = task_idx(t), slot = task_slot(t), c = task_chunk(t);
+      if (ty == kTaskRouter) {
+        const int c0 = (int)c * P.router_part_cols;
+        src = P.router_w + (int64_t)(cta + (int)idx * G) * P.H + c0;
+        bytes = (uint32_t)min(P.router_part_cols, P.H - c0) * 2;
+      } else if (ty == kTaskGateUp) {
+        const int u = cta + (int)idx * G, rb = u % P.units_per_slot;
+        const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
+        src = P.experts + (int64_t)misc->slot_e[slot] * P.blob_bytes + ((int64_t)rb * P.gu_tiles + c * kChunkTiles) * TB;
+        bytes = (uint32_t)(n * TB);
+      } else {
+        const int rbg = first_rb + (int)idx * G;
+        const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
+        src = P.experts + (int64_t)misc->slot_e[slot] * P.blob_bytes + packed_gu_bytes(P.H, P.I, BITS) +
+              ((int64_t)rbg * P.dn_tiles + c * kChunkTiles) * TB;
+        bytes = (uint32_t)(n * TB);
+      }
+      mbar_expect_tx(bar_full + 8u * s, bytes);
+      tma_load(dst, src, bytes, bar_full + 8u * s);
+      // tells the consumer of task i that this fill is the one to wait for
+      reinterpret_cast<volatile int*>(misc->last_task)[s] = i;
+      return 1;
+    };
+    for (int r = 0; r * NI < n_tasks; ++r) {
+      if (__any_sync(0xffffffffu, *abort_flag)) break;
+      const int i = r * NI + lane;
+      const bool mine = lane < NI && i < n_tasks;
+      const uint32_t t = mine ? tasks[i] : 0u;
+      const bool needs_route =
+          mine && P.mode == kModeLayer && !routed && task_type(t) != kTaskRouter && task_slot(t) >= 1;
+      int ok = 1;
+      if (mine && !needs_route) ok = issue(i, t);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (__any_sync(0xffffffffu, needs_route)) {
+        if (!do_routing()) break;
+        routed = true;
+        if (needs_route) ok = issue(i, t);
+        if (!__all_sync(0xffffffffu, ok)) break;
       }
     }
-  };
-
-  // ---------------------------------------------------------------- gate/up stages, interleaved with downs
-  int next_down = 0;
-  const int n_zg = P.H / kGroup;
-  for (int s = 0; s < my_stages && !abort; ++s) {
-    if (!routed && stage_max_slot(s) > 0) {
+    // routing still owed for the output indices
+    if (!__any_sync(0xffffffffu, *abort_flag) && !routed && has_router && cta == 0 && (P.idx_out || P.w_out))
       do_routing();
-      routed = true;
-      if (abort) break;
-    }
-    const int buf = s % P.nstage;
-    if (!wait_mbar(bar_base + 8u * buf, (uint32_t)((s / P.nstage) & 1), limit)) {
-      abort = 1;
-      atomicOr(&P.ws->status, kStatusTimeoutTma);
-    }
-    const int kr = warp % P.n_kr_gu, team = warp / P.n_kr_gu;
-    const int j = s * P.teams_gu + team;
-    float* part = gupart + (s & 1) * (kWarps * 16);
-    if (!abort && team < P.teams_gu && j < my_units) {
-      uint2 bf[4][4];
-      float2 inf[4];
-      load_frags(reinterpret_cast<const uint32_t*>(smem + P.off_zfrag),
-                 reinterpret_cast<const float2*>(smem + P.off_zinfo), kr, n_zg, lane, bf, inf);
-      const uint8_t* base = smem + P.off_ring + (uint32_t)buf * P.stage_bytes + (uint32_t)(team * P.gu_unit_bytes);
-      float acc0 = 0.f, acc1 = 0.f;
+  } else {
+    // ============================================================ consumer warps
+    if (P.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+    const uint32_t tag = *reinterpret_cast<volatile uint32_t*>(&P.ws->epoch) + 1u;
+    if (tid == 0) misc->tag = tag;
+    // residual rows this block writes at the end
+    if (P.mode == kModeLayer && tid < my_rb * 16)
+      h_res = bf16f(P.h_in[(first_rb + (tid / 16) * G) * 16 + tid % 16]);
+    // ---- input: z = RMSNorm(h_in) or h_in (bf16, shared memory) and its fragments
+    {
+      const int c0 = tid * 8;
+      uint4 hv = make_uint4(0u, 0u, 0u, 0u);
+      if (c0 < P.H) hv = *reinterpret_cast<const uint4*>(P.h_in + c0);
+      if (P.norm_w != nullptr) {
+        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+        float ss = 0.f;
 #pragma unroll
-      for (int tt = 0; tt < 4; ++tt)
-        if (kr * 4 + tt < P.gu_tiles) tile_dot<BITS>(base + (kr * 4 + tt) * TB, bf[tt], inf[tt], lane, acc0, acc1);
-      if ((lane & 3) == 0) {
-        part[warp * 16 + (lane >> 2)] = acc0;
-        part[warp * 16 + 8 + (lane >> 2)] = acc1;
-      }
-    }
-    abort = __syncthreads_or(abort);
-    if (abort) break;
-    consumed = s + 1;
-    if (tid == 0) issue_ready_stages(consumed + P.nstage, routed);
-    // reduce the stage's units: a = silu(g) * u
-    const int nred = P.teams_gu * 8;
-    if (tid < nred) {
-      const int tau = tid / 8, i = tid % 8, jj = s * P.teams_gu + tau;
-      if (jj < my_units) {
-        float g = 0.f, u = 0.f;
-        for (int k = 0; k < P.n_kr_gu; ++k) {
-          g += part[(tau * P.n_kr_gu + k) * 16 + i];
-          u += part[(tau * P.n_kr_gu + k) * 16 + 8 + i];
+        for (int k = 0; k < 4; ++k) {
+          ss = fmaf(bf16lo(hw[k]), bf16lo(hw[k]), ss);
+          ss = fmaf(bf16hi(hw[k]), bf16hi(hw[k]), ss);
         }
-        const int uu = unit_of(jj), slot = uu / P.units_per_slot, rb = uu % P.units_per_slot;
-        const float a = g / (1.0f + expf(-g)) * u;
-        P.ws_a[(int64_t)slot * P.I + rb * 8 + i] = a;
-      }
-    }
-    if (nred <= 32) __syncwarp();
-    else if (tid < ((nred + 31) / 32) * 32) asm volatile("bar.sync 15, %0;" ::"r"(((nred + 31) / 32) * 32) : "memory");
-    if (tid == 0) {
-      // publish per slot (units of a stage have non-decreasing slots)
-      int n = min(P.teams_gu, my_units - s * P.teams_gu);
-      int cur = -1;
-      uint32_t cnt = 0;
-      for (int tau = 0; tau < n; ++tau) {
-        int slot = unit_of(s * P.teams_gu + tau) / P.units_per_slot;
-        if (slot != cur) {
-          if (cnt) red_release_add(&P.ws->h_arrive[cur], cnt);
-          cur = slot;
-          cnt = 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) misc->red[warp] = ss;
+        asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
+        float tot = 0.f;
+        for (int w = 0; w < kConsumerWarps; ++w) tot += misc->red[w];
+        const float r = 1.0f / sqrtf(tot / (float)P.H + P.eps);
+        if (c0 < P.H) {
+          const uint4 wv = *reinterpret_cast<const uint4*>(P.norm_w + c0);
+          const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+          uint32_t zz[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t lo = f2bf16(bf16lo(hw[k]) * r * bf16lo(ww[k]));
+            const uint32_t hi = f2bf16(bf16hi(hw[k]) * r * bf16hi(ww[k]));
+            zz[k] = lo | (hi << 16);
+          }
+          hv = make_uint4(zz[0], zz[1], zz[2], zz[3]);
         }
-        ++cnt;
       }
-      if (cnt) red_release_add(&P.ws->h_arrive[cur], cnt);
+      if (c0 < P.H) *reinterpret_cast<uint4*>(zs + c0) = hv;
+      asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
+      if (P.n_slots > 0) {
+        for (int Gi = warp; Gi < P.H / kGroup; Gi += kConsumerWarps) {
+          const uint32_t zz = *reinterpret_cast<const uint32_t*>(zs + Gi * kGroup + 2 * lane);
+          frag_group(bf16lo(zz), bf16hi(zz), Gi, BITS, zfrag, zinfo, lane);
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
     }
-    // downs of slot d once all of this block's units of slots <= d+1 are done
-    while (next_down < P.n_slots && !abort) {
-      bool last = (s + 1 == my_stages);
-      int next_slot = last ? 1 << 30 : unit_of((s + 1) * P.teams_gu) / P.units_per_slot;
-      if (next_slot <= next_down + 1) break;
-      if (!routed && next_down >= 1) { do_routing(); routed = true; if (abort) break; }
-      do_downs(next_down++);
+
+    // ---- task loop: warp w takes tasks w, w+16, ...
+    for (int i = warp; i < n_tasks; i += kConsumerWarps) {
+      int s, fill;
+      task_stage(P.nstage, P.n_issuers, i, s, fill);
+      // A stage's fills are consumed by different warps, so first make sure
+      // task i is the stage's current fill (all earlier fills consumed); only
+      // then is the parity wait unambiguous.  Every lane observes the phase,
+      // so the copied bytes are visible to it.
+      const bool issued = wait_flag(reinterpret_cast<volatile int*>(misc->last_task) + s, i, limit, abort_flag);
+      if (!__all_sync(0xffffffffu, issued && wait_mbar(bar_full + 8u * s, (uint32_t)(fill & 1), limit, abort_flag))) {
+        if (lane == 0) {
+          if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutTma);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      const uint8_t* stage = smem + P.off_ring + (uint32_t)s * P.stage_bytes;
+      const uint32_t t = tasks[i];
+      const uint32_t ty = task_type(t), idx = task_idx(t), slot = task_slot(t), c = task_chunk(t);
+      if (ty == kTaskRouter) {
+        const int c0 = (int)c * P.router_part_cols, width = min(P.router_part_cols, P.H - c0);
+        float acc = 0.f;
+        for (int col = lane * 8; col < width; col += 256) {
+          const uint4 w = *reinterpret_cast<const uint4*>(stage + col * 2);
+          const uint4 z = *reinterpret_cast<const uint4*>(zs + c0 + col);
+          acc = fmaf(bf16lo(w.x), bf16lo(z.x), acc);
+          acc = fmaf(bf16hi(w.x), bf16hi(z.x), acc);
+          acc = fmaf(bf16lo(w.y), bf16lo(z.y), acc);
+          acc = fmaf(bf16hi(w.y), bf16hi(z.y), acc);
+          acc = fmaf(bf16lo(w.z), bf16lo(z.z), acc);
+          acc = fmaf(bf16hi(w.z), bf16hi(z.z), acc);
+          acc = fmaf(bf16lo(w.w), bf16lo(z.w), acc);
+          acc = fmaf(bf16hi(w.w), bf16hi(z.w), acc);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+          // parts of a row are summed, in part order, by whichever warp ends last
+          misc->rpart[idx][c] = acc;
+          __threadfence_block();
+          const int old = atomicAdd(&misc->rcnt[idx], 1);
+          if (old == P.router_parts - 1) {
+            __threadfence_block();
+            const volatile float* rp = misc->rpart[idx];
+            float l = 0.f;
+            for (int q = 0; q < P.router_parts; ++q) l += rp[q];
+            const int e = cta + (int)idx * G;
+            if (P.router_bias) l += P.router_bias[e];
+            // fault injection publishes with a stale tag, so no reader accepts it
+            st_tagged(P.ws_logits + e, l, (P.flags & FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE) ? tag - 1u : tag);
+            red_relaxed_add(&P.ws->router_cnt, 1u);
+          }
+        }
+      } else if (ty == kTaskGateUp) {
+        const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
+        float acc0 = 0.f, acc1 = 0.f;
+        chunk_dot<BITS>(stage, n, zfrag, zinfo, (int)c * kChunkTiles, lane, acc0, acc1);
+        const int u = cta + (int)idx * G, rb = u % P.units_per_slot;
+        bool last = true;
+        if (P.gu_chunks > 1) {
+          float* part = gupart + ((int)idx * P.gu_chunks + (int)c) * 16;
+          if ((lane & 3) == 0) { part[lane >> 2] = acc0; part[8 + (lane >> 2)] = acc1; }
+          __syncwarp();
+          int old = 0;
+          if (lane == 0) {
+            __threadfence_block();
+            old = atomicAdd(&misc->unit_cnt[idx], 1);
+            __threadfence_block();
+          }
+          old = __shfl_sync(0xffffffffu, old, 0);
+          last = old == P.gu_chunks - 1;
+          if (last && lane < 8) {
+            acc0 = 0.f;
+            acc1 = 0.f;
+            for (int k = 0; k < P.gu_chunks; ++k) {
+              const volatile float* pk = gupart + ((int)idx * P.gu_chunks + k) * 16;
+              acc0 += pk[lane];
+              acc1 += pk[8 + lane];
+            }
+          }
+        }
+        if (last) {
+          // lanes 0..7 (gu_chunks > 1) or lanes 4g (gu_chunks == 1) hold row g
+          const int row = P.gu_chunks > 1 ? lane : (lane >> 2);
+          const bool writer = P.gu_chunks > 1 ? lane < 8 : (lane & 3) == 0;
+          const float av = writer ? acc0 / (1.0f + expf(-acc0)) * acc1 : 0.f;
+          if (writer) st_tagged(P.ws_a + (int64_t)slot * P.I + rb * 8 + row, av, tag);
+          // the unit's sum (fixed tree order) and max |a| (order-free) let
+          // readers scale and fold the bias without reducing 64 values each
+          float us = av;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) us += __shfl_xor_sync(0xffffffffu, us, o);
+          const uint32_t um = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(av)));
+          if (lane == 0) {
+            st_tagged(P.ws_asum + (int64_t)slot * P.units_per_slot + rb, us, tag);
+            atom_max_u64(P.ws_amax + slot, ((uint64_t)tag << 32) | um);
+            red_relaxed_add(&P.ws->h_cnt[slot], 1u);
+          }
+        }
+      } else {
+        // activations of this slot as fragments (built once per block)
+        uint32_t* af = reinterpret_cast<uint32_t*>(smem + P.off_afrag + slot * P.afrag_bytes);
+        float2* ai = reinterpret_cast<float2*>(smem + P.off_ainfo + slot * P.ainfo_bytes);
+        int claimed = 0;
+        if (lane == 0 && misc->aflag[slot] == 0 && atomicCAS(&misc->aflag[slot], 0, 1) == 0) claimed = 1;
+        claimed = __shfl_sync(0xffffffffu, claimed, 0);
+        int good = 1;
+        if (claimed) {
+          // poll the slot's tagged activations (published by every block's
+          // gate/up units), 8 groups at a time, and turn them into fragments
+          const uint64_t* act = P.ws_a + (int64_t)slot * P.I;
+          const int ng = P.I / kGroup;
+          const uint64_t t0 = gtimer();
+          good = __all_sync(0xffffffffu,
+                            wait_count(&P.ws->h_cnt[slot], (uint32_t)P.units_per_slot, limit, abort_flag));
+          if (!good && lane == 0) {
+            if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
+            *abort_flag = 1;
+          }
+          // One scale per slot, 2^sh with the slot's largest |a| in [2^14, 2^15)
+          // (from the producers' tag-keyed atomic max), and each group's sum from
+          // its 8 units' published sums (fixed order): no reductions here.
+          float scl_base = 0.f, inv = 1.f;
+          if (good) {
+            for (;;) {
+              const uint64_t mw = ld_tagged(P.ws_amax + slot);
+              if (__all_sync(0xffffffffu, tagged_tag(mw) == tag)) {
+                const uint32_t m = (uint32_t)mw;
+                const int e = (int)((m >> 23) & 0xFF) - 127;
+                int sh = (m == 0) ? 0 : 14 - max(e, -126);
+                sh = min(sh, 126);
+                scl_base = exp2i(sh);
+                inv = exp2i(-sh);
+                break;
+              }
+              __nanosleep(64);
+              if (__any_sync(0xffffffffu, *abort_flag != 0 || gtimer() - t0 > limit)) {
+                good = 0;
+                break;
+              }
+            }
+          }
+          // this lane's pair (2*lane, 2*lane+1) of every group sits at one
+          // position of the fragment layout
+          const int kq = 2 * lane, sq = kq / 16, kkq = kq % 16, whq = kkq / 8, tq = (kkq % 8) / 2;
+          const int fsq = (BITS == 4) ? (whq ? 4 : 0) : ((sq & 1) ? 4 : 0) + (whq ? 2 : 0);
+          const float scl = scl_base * exp2i(-fsq);
+          for (int g0 = 0; g0 < ng && good; g0 += 4) {
+            ulonglong2 v[4];
+            ulonglong2 su[4];
+            const int gs = g0 + lane;  // group whose sum this lane assembles
+            for (;;) {
+              bool mine = true;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                v[k] = (g0 + k < ng) ? ld_tagged2(act + (g0 + k) * kGroup + 2 * lane) : make_ulonglong2(0ull, 0ull);
+                if (g0 + k < ng) mine = mine && tagged_tag(v[k].x) == tag && tagged_tag(v[k].y) == tag;
+              }
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                su[k] = (lane < 4 && gs < ng) ? ld_tagged2(P.ws_asum + (int64_t)slot * P.units_per_slot + gs * 8 + 2 * k)
+                                              : make_ulonglong2(0ull, 0ull);
+                if (lane < 4 && gs < ng) mine = mine && tagged_tag(su[k].x) == tag && tagged_tag(su[k].y) == tag;
+              }
+              if (__all_sync(0xffffffffu, mine)) break;
+              __nanosleep(64);
+              if (__any_sync(0xffffffffu, *abort_flag != 0 || gtimer() - t0 > limit)) {
+                good = 0;
+                break;
+              }
+            }
+            if (!good) break;
+            if (lane < 4 && gs < ng) {
+              float gsum = 0.f;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) gsum += tagged_value(su[k].x) + tagged_value(su[k].y);
+              ai[gs] = make_float2(inv, gsum);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              if (g0 + k < ng) {
+                __half2 h2 = __floats2half2_rn(tagged_value(v[k].x) * scl, tagged_value(v[k].y) * scl);
+                af[(((g0 + k) * 4 + tq) * 4 + sq) * 2 + whq] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+            }
+          }
+          if (!good && lane == 0) {
+            if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
+            *abort_flag = 1;
+          }
+          if (good) {
+            __syncwarp();
+            if (lane == 0) {
+              __threadfence_block();
+              *reinterpret_cast<volatile int*>(&misc->aflag[slot]) = 2;
+            }
+          }
+        } else {
+          if (lane == 0 && !wait_flag(&misc->aflag[slot], 2, limit, abort_flag)) {
+            if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
+            *abort_flag = 1;
+            good = 0;
+          }
+          good = __shfl_sync(0xffffffffu, good, 0);
+          __threadfence_block();
+        }
+        if (!good) break;
+        const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
+        float acc0 = 0.f, acc1 = 0.f;
+        chunk_dot<BITS>(stage, n, af, ai, (int)c * kChunkTiles, lane, acc0, acc1);
+        float* y = ys + ((int)idx * P.n_slots + (int)slot) * 16;
+        if (P.dn_chunks == 1) {
+          if ((lane & 3) == 0) { y[lane >> 2] = acc0; y[8 + (lane >> 2)] = acc1; }
+        } else {
+          const int job = (int)idx * P.n_slots + (int)slot;
+          float* part = dnpart + (job * P.dn_chunks + (int)c) * 16;
+          if ((lane & 3) == 0) { part[lane >> 2] = acc0; part[8 + (lane >> 2)] = acc1; }
+          __syncwarp();
+          int old = 0;
+          if (lane == 0) {
+            __threadfence_block();
+            old = atomicAdd(&misc->dn_cnt[job], 1);
+            __threadfence_block();
+          }
+          old = __shfl_sync(0xffffffffu, old, 0);
+          if (old == P.dn_chunks - 1 && lane < 16) {
+            float v = 0.f;
+            for (int k = 0; k < P.dn_chunks; ++k) v += reinterpret_cast<volatile float*>(dnpart)[(job * P.dn_chunks + k) * 16 + lane];
+            y[lane] = v;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty + 8u * s);
     }
   }
-  // Routing still pending: needed for the output indices (block 0) and for the
-  // down projections of routed experts.
-  if (!abort && !routed && has_router && (cta == 0 || (P.mode == kModeLayer && my_rb > 0))) {
-    do_routing();
-    routed = true;
-  }
-  while (!abort && next_down < P.n_slots) do_downs(next_down++);
+  __syncthreads();
 
   // ---------------------------------------------------------------- combine + output
-  __syncthreads();
-  if (!abort) {
-    for (int r = tid; r < my_rb * 16; r += kThreads) {
+  const bool aborted = *abort_flag != 0;
+  if (!aborted && tid < kConsumerWarps * 32) {
+    for (int r = tid; r < my_rb * 16; r += kConsumerWarps * 32) {
       const int jb = r / 16, row = r % 16;
       const int out_row = (first_rb + jb * G) * 16 + row;
       if (P.mode == kModeLayer) {
-        float acc = bf16f(P.h_in[out_row]) + ys[(jb * P.n_slots + 0) * 16 + row];
-        for (int k = 1; k < P.n_slots; ++k) acc = fmaf(slot_w[k], ys[(jb * P.n_slots + k) * 16 + row], acc);
+        float acc = h_res + ys[(jb * P.n_slots + 0) * 16 + row];
+        for (int k = 1; k < P.n_slots; ++k) acc = fmaf(misc->slot_w[k], ys[(jb * P.n_slots + k) * 16 + row], acc);
         P.h_out[out_row] = f2bf16(acc);
       } else if (P.mode == kModeExpert) {
         P.y_out[out_row] = ys[(jb * P.n_slots + 0) * 16 + row];
@@ -585,26 +798,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   }
 
   // ---------------------------------------------------------------- drain + reset
-  if (tid == 0) {
-    // copies still in flight (only after an abort) must land before the block exits
-    for (int s = consumed; s < issued; ++s)
-      if (!wait_mbar(bar_base + 8u * (s % P.nstage), (uint32_t)((s / P.nstage) & 1), limit))
-        atomicOr(&P.ws->status, kStatusTimeoutTma);
-    if (router_issued && !router_consumed && !wait_mbar(bar_router, 0, limit))
-      atomicOr(&P.ws->status, kStatusTimeoutTma);
-    for (int d = 0; d < kMaxSlots; ++d)
-      if ((dn_issued >> d & 1) && !(dn_consumed >> d & 1) && !wait_mbar(bar_base + 8u * (P.nstage + d), 0, limit))
-        atomicOr(&P.ws->status, kStatusTimeoutTma);
+  if (tid == kConsumerWarps * 32) {
+    // After an abort the latest copy into every stage must land before the
+    // block exits (without one, every issued copy was consumed already).
+    for (int s = 0; s < P.nstage && aborted; ++s) {
+      const int i = misc->last_task[s];
+      if (i < 0) continue;
+      int s2, fill;
+      task_stage(P.nstage, P.n_issuers, i, s2, fill);
+      const uint64_t t0 = gtimer();
+      while (!mbar_try_wait(bar_full + 8u * s, (uint32_t)(fill & 1)))
+        if (gtimer() - t0 > limit) {
+          atomicOr(&P.ws->status, kStatusTimeoutTma);
+          break;
+        }
+    }
+    // the last block out advances the epoch for the next launch
     uint32_t old;
-    asm volatile("fence.acq_rel.gpu;\n atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                 : "=r"(old)
-                 : "l"(&P.ws->exit_count)
-                 : "memory");
+    asm volatile("atom.release.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&P.ws->exit_count) : "memory");
     if (old == (uint32_t)G - 1) {
-      P.ws->router_arrive = 0;
-      for (int i = 0; i < 16; ++i) P.ws->h_arrive[i] = 0;
       P.ws->exit_count = 0;
-      __threadfence();
+      P.ws->router_cnt = 0;
+      for (int k = 0; k < 16; ++k) P.ws->h_cnt[k] = 0;
+      P.ws->epoch = misc->tag;
     }
   }
 }
@@ -649,8 +865,7 @@ int launch_decode(const DecodePlan& plan, void* stream, bool cooperative, bool p
   }
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  err = cudaLaunchKernelEx(&cfg, kern, p);
-  return (int)err;
+  return (int)cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 int zero_workspace(void* ws, size_t bytes, void* stream) {

@@ -34,9 +34,10 @@ namespace fmoe {
 constexpr int kGroup = 64;
 constexpr int kMaxTopK = 8;
 constexpr int kMaxSlots = kMaxTopK + 1;  // K routed + 1 shared
-constexpr int kThreads = 512;            // 16 warps per block
-constexpr int kWarps = kThreads / 32;
-constexpr int kMaxNStage = 4;
+constexpr int kConsumerWarps = 16;       // warps that compute
+constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kChunkTiles = 16;          // tiles per gate/up or down task
+constexpr int kMaxTasks = 96;            // task-list capacity per block (multiple of 32)
 
 inline __host__ __device__ int tile_code_bytes(int bits) { return 16 * kGroup * bits / 8; }
 inline __host__ __device__ int tile_bytes(int bits) { return tile_code_bytes(bits) + 64; }
@@ -51,14 +52,17 @@ inline __host__ __device__ int64_t packed_gu_bytes(int H, int I, int bits) {
   return (int64_t)(I / 8) * (H / kGroup) * tile_bytes(bits);
 }
 
-// Device workspace header (counters and status), followed by logits and
-// activations.  Zero between launches: the last block of every launch resets it.
+// Device workspace header, followed by the tagged logits and activations.
+// Cross-block results are published as 64-bit words {float bits, tag} with
+// tag = epoch + 1, so a reader knows a value is from the current launch
+// without any counter, fence or atomic on the critical path.  The last block
+// to finish a launch advances the epoch (exit_count protocol).
 struct WsHeader {
-  uint32_t router_arrive;
-  uint32_t exit_count;
-  uint32_t status;
-  uint32_t pad0;
-  uint32_t h_arrive[16];
+  uint32_t epoch;           // launches completed on this workspace
+  uint32_t exit_count;      // blocks finished in the current launch
+  uint32_t status;          // kStatus* bits, cleared by fmoe_poll_status
+  uint32_t router_cnt;      // router rows published in this launch (hint for pollers)
+  uint32_t h_cnt[16];       // gate/up units published per slot in this launch (hint)
 };
 static_assert(sizeof(WsHeader) <= 256, "header");
 
@@ -67,7 +71,35 @@ constexpr uint32_t kStatusTimeoutRouter = 0x1;
 constexpr uint32_t kStatusTimeoutH = 0x2;
 constexpr uint32_t kStatusTimeoutTma = 0x4;
 
+
 enum DecodeMode : int { kModeLayer = 0, kModeExpert = 1, kModeRoute = 2 };
+
+// Task descriptors of a block's ordered work list (one 32-bit word each).
+enum TaskType : uint32_t { kTaskRouter = 0, kTaskGateUp = 1, kTaskDown = 2 };
+inline __host__ __device__ uint32_t make_task(uint32_t type, uint32_t idx, uint32_t slot, uint32_t chunk) {
+  return type | (idx << 2) | (slot << 18) | (chunk << 22);
+}
+inline __host__ __device__ uint32_t task_type(uint32_t t) { return t & 3u; }
+inline __host__ __device__ uint32_t task_idx(uint32_t t) { return (t >> 2) & 0xFFFFu; }
+inline __host__ __device__ uint32_t task_slot(uint32_t t) { return (t >> 18) & 0xFu; }
+inline __host__ __device__ uint32_t task_chunk(uint32_t t) { return (t >> 22) & 0x3FFu; }
+
+// Shared-memory bookkeeping of the fused kernel.
+struct Misc {
+  int slot_e[16];
+  float slot_w[16];
+  int abort;
+  uint32_t tag;         // epoch + 1 of this launch
+  int n_tasks;          // length of this block's task list
+  int pad[13];
+  int aflag[16];        // per-slot activation fragments: 0 none, 1 building, 2 ready
+  int rcnt[16];         // parts finished per router row of this block
+  float rpart[16][4];   // partial logits per router row and part
+  int unit_cnt[32];     // K-chunks finished per gate/up unit of this block
+  int dn_cnt[32];       // K-chunks finished per (row block, slot) down job
+  int last_task[64];    // last task issued into each ring stage (-1: none)
+  float red[16];        // RMSNorm scratch
+};
 
 // Everything the fused single-token kernel needs, computed on the host.
 struct DecodePlan {
@@ -76,34 +108,33 @@ struct DecodePlan {
   int n_slots;             // K+1 (layer), 1 (expert), 0 (route)
   int grid;                // blocks (one per SM)
   int tb, cb;              // tile bytes, code bytes per tile
-  int gu_tiles;            // H/64 tiles per gate/up row block
-  int gu_unit_bytes;       // gu_tiles * tb
-  int n_kr_gu;             // K-ranges (warps) per gate/up unit
-  int teams_gu;            // gate/up units processed concurrently (= units per stage)
+  int gu_tiles;            // H/64 tiles per gate/up row block (unit)
+  int gu_chunks;           // tasks per unit (kChunkTiles tiles each, last may be shorter)
+  int dn_tiles;            // I/64 tiles per down row block
+  int dn_chunks;           // tasks per down job
   int units_per_slot;      // I/8
   int total_units;         // n_slots * units_per_slot
-  int dn_tiles;            // I/64 tiles per down row block
-  int dn_job_bytes;        // dn_tiles * tb
-  int n_kr_dn;             // K-ranges per down job
-  int teams_dn;            // down jobs processed concurrently
+  int units_per_cta;       // max units per block
   int n_rb;                // H/16 output row blocks
   int rb_per_cta;          // max output row blocks per block
   int router_rows;         // max router rows per block
-  int router_chunks;       // 256-column chunks per router row
-  int nstage;
+  int router_parts;        // column parts per router row (one task each)
+  int router_part_cols;    // columns per part (multiple of 64; the last part may be shorter)
+  int nstage;              // ring stages (a multiple of n_issuers)
+  int n_issuers;           // producer lanes issuing copies; lane l owns stages l, l+n_issuers, ...
+  uint32_t stage_bytes;
   // shared-memory layout (byte offsets)
-  uint32_t off_ring, stage_bytes;
-  uint32_t off_down;       // [slot][rb_local] down jobs
-  uint32_t off_router;     // router rows (aliases the routed part of off_down)
+  uint32_t off_ring;
+  uint32_t off_z;          // bf16 z [H]
+  uint32_t off_lg;         // fp32 logits [E] (routing)
   uint32_t off_zfrag, off_zinfo;
-  uint32_t off_afrag, off_ainfo, afrag_bytes, ainfo_bytes;  // two buffers
-  uint32_t off_z;          // bf16 z [H] (router input; reused for logits)
-  uint32_t off_gupart;     // [2][16 warps][16] fp32
-  uint32_t off_dnpart;     // [16 warps][16] fp32
+  uint32_t off_afrag, off_ainfo, afrag_bytes, ainfo_bytes;  // per slot
+  uint32_t off_gupart;     // [units_per_cta][gu_chunks][16] fp32
+  uint32_t off_dnpart;     // [rb_per_cta][n_slots][dn_chunks][16] fp32
   uint32_t off_y;          // [rb_per_cta][n_slots][16] fp32
-  uint32_t off_rpart;      // [router_rows][16 warps] fp32
-  uint32_t off_misc;       // slot expert ids / weights
-  uint32_t off_bar;        // mbarriers
+  uint32_t off_tasks;      // [kMaxTasks] uint32, this block's task list
+  uint32_t off_misc;       // slot expert ids / weights / counters / flags
+  uint32_t off_bar;        // mbarriers: full[nstage], empty[nstage]
   uint32_t smem_bytes;
   // data
   const uint8_t* experts;  // packed experts of this layer
@@ -119,12 +150,28 @@ struct DecodePlan {
   float* w_out;            // [K] or null
   int expert_id;           // expert mode: 0..E (E = shared)
   WsHeader* ws;
-  float* ws_logits;        // [E]
-  float* ws_a;             // [kMaxSlots][I]
+  uint64_t* ws_logits;     // [E] tagged
+  uint64_t* ws_a;          // [kMaxSlots][I] tagged
+  uint64_t* ws_asum;       // [kMaxSlots][I/8] tagged per-unit sums of a
+  uint64_t* ws_amax;       // [kMaxSlots] (tag << 32) | bits of max |a| (atomic max)
+  const uint32_t* tasks;   // [grid][kMaxTasks] ordered task lists (host-built)
+  const int32_t* n_tasks;  // [grid]
   uint32_t flags;
   uint64_t timeout_ns;
   int pdl;                 // launched with programmatic stream serialisation
 };
+
+// Ring position of task i: issued by producer lane i % n_issuers into that
+// lane's (i / n_issuers) % (nstage / n_issuers)-th stage, as fill number
+// (i / n_issuers) / (nstage / n_issuers) of that stage.
+inline __host__ __device__ void task_stage(int nstage, int n_issuers, int i, int& stage, int& fill) {
+  const int L = nstage / n_issuers, j = i / n_issuers;
+  stage = (j % L) * n_issuers + i % n_issuers;
+  fill = j / L;
+}
+
+// Host-side construction of a block's ordered task list; returns its length.
+int build_task_list(const DecodePlan& P, int cta, uint32_t* out);
 
 // host launchers (return cudaError_t as int)
 int launch_repack(const uint8_t* src, uint8_t* dst, int n_experts, int H, int I, int bits, int to_packed,
