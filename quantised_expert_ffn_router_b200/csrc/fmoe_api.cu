@@ -26,8 +26,6 @@ struct fmoe_ctx {
   WsHeader* hdr = nullptr;
   uint64_t* logits = nullptr;  // tagged
   uint64_t* act = nullptr;     // tagged
-  uint64_t* asum = nullptr;    // tagged
-  uint64_t* amax = nullptr;    // tag-keyed maxima
   uint32_t* tasks = nullptr;   // device [3 modes][grid][kMaxTasks]
   int32_t* ntasks = nullptr;   // device [3 modes][grid]
   uint16_t* stack_buf[2] = {nullptr, nullptr};  // ping-pong activations, [max_tokens][H] bf16
@@ -200,8 +198,6 @@ DecodePlan bind(const fmoe_ctx* ctx, int mode, int layer) {
   P.ws = ctx->hdr;
   P.ws_logits = ctx->logits;
   P.ws_a = ctx->act;
-  P.ws_asum = ctx->asum;
-  P.ws_amax = ctx->amax;
   P.tasks = ctx->tasks + (size_t)mode * ctx->n_sm * kMaxTasks;
   P.n_tasks = ctx->ntasks + (size_t)mode * ctx->n_sm;
   P.flags = ctx->cfg.flags;
@@ -233,12 +229,12 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 namespace fmoe {
 
 // A block's ordered work list: its router row parts; the slot-0 expert's
-// gate/up K-chunks and down jobs (known before routing); then the routed
-// experts' gate/up chunks in unit order and their down jobs in slot order.
-// Routed down jobs wait for other blocks' activations, so they come last in
-// every consumer warp's queue: no gate/up chunk ever waits behind them.  The
-// slot-0 down jobs may wait, but only until the slot-0 units every block runs
-// first are done, while routed chunks cannot start anyway.
+// gate/up K-chunks (known before routing); the routed experts' gate/up chunks
+// in unit order; then every down job, slot by slot.  A down job waits for
+// other blocks' activations and holds its ring stage while it waits, so all of
+// them come after the last gate/up chunk: the producer has issued every
+// gate/up copy before any stage can be held up, and the down weights land
+// while the activations are being exchanged.
 int build_task_list(const DecodePlan& P, int cta, uint32_t* out) {
   const int G = P.grid;
   const int my_units = P.total_units > cta ? (P.total_units - cta + G - 1) / G : 0;
@@ -249,18 +245,15 @@ int build_task_list(const DecodePlan& P, int cta, uint32_t* out) {
   for (int j = 0; j < my_rrows; ++j)
     for (int q = 0; q < P.router_parts; ++q) out[n++] = make_task(kTaskRouter, j, 0, q);
   // the slot-0 expert (shared, or the single expert) needs no routing: its
-  // gate/up chunks and down jobs go first, ahead of every routed chunk
+  // gate/up chunks go first, ahead of every routed chunk
   int j = 0;
   for (; j < my_units && (cta + j * G) / P.units_per_slot == 0; ++j)
     for (int c = 0; c < P.gu_chunks; ++c) out[n++] = make_task(kTaskGateUp, j, 0, c);
-  if (P.n_slots > 0)
-    for (int r = 0; r < my_rb; ++r)
-      for (int c = 0; c < P.dn_chunks; ++c) out[n++] = make_task(kTaskDown, r, 0, c);
   for (; j < my_units; ++j) {
     const int slot = (cta + j * G) / P.units_per_slot;
     for (int c = 0; c < P.gu_chunks; ++c) out[n++] = make_task(kTaskGateUp, j, slot, c);
   }
-  for (int d = 1; d < P.n_slots; ++d)
+  for (int d = 0; d < P.n_slots; ++d)
     for (int r = 0; r < my_rb; ++r)
       for (int c = 0; c < P.dn_chunks; ++c) out[n++] = make_task(kTaskDown, r, d, c);
   return n;
@@ -336,16 +329,12 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
     if (blocks < 1) return bail(fail(ctx, FMOE_ERR_UNSUPPORTED, "fused kernel cannot be resident"));
   }
 
-  // workspace: header | logits [E] | activations [kMaxSlots][I] | 2 x [max_tokens][H] bf16
+  // workspace: header | logits [E] | activations [kMaxSlots][I] | task lists | 2 x [max_tokens][H] bf16
   size_t off = 256;
   size_t off_logits = off;
   off += ((size_t)c.n_experts * 8 + 255) / 256 * 256;
   size_t off_act = off;
   off += ((size_t)kMaxSlots * c.inter * 8 + 255) / 256 * 256;
-  size_t off_asum = off;
-  off += ((size_t)kMaxSlots * (c.inter / 8) * 8 + 255) / 256 * 256;
-  size_t off_amax = off;
-  off += 256;
   size_t off_tasks = off;
   off += ((size_t)3 * ctx->n_sm * kMaxTasks * 4 + 255) / 256 * 256;
   size_t off_ntasks = off;
@@ -364,8 +353,6 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   ctx->hdr = reinterpret_cast<WsHeader*>(base);
   ctx->logits = reinterpret_cast<uint64_t*>(base + off_logits);
   ctx->act = reinterpret_cast<uint64_t*>(base + off_act);
-  ctx->asum = reinterpret_cast<uint64_t*>(base + off_asum);
-  ctx->amax = reinterpret_cast<uint64_t*>(base + off_amax);
   ctx->tasks = reinterpret_cast<uint32_t*>(base + off_tasks);
   ctx->ntasks = reinterpret_cast<int32_t*>(base + off_ntasks);
   ctx->stack_buf[0] = reinterpret_cast<uint16_t*>(base + off_stack);

@@ -166,9 +166,6 @@ __device__ __forceinline__ ulonglong2 ld_tagged2(const uint64_t* p) {
   asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(w.x), "=l"(w.y) : "l"(p) : "memory");
   return w;
 }
-__device__ __forceinline__ void atom_max_u64(uint64_t* p, uint64_t v) {
-  asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
 __device__ __forceinline__ float tagged_value(uint64_t w) { return __uint_as_float((uint32_t)w); }
 __device__ __forceinline__ uint32_t tagged_tag(uint64_t w) { return (uint32_t)(w >> 32); }
 
@@ -196,35 +193,53 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-// fp16 B fragments of one 64-value group, built by one warp (lane holds values
-// 2*lane and 2*lane+1 of the group).  The group is scaled by 2^sh so its
-// largest magnitude lies in [2^14, 2^15); within slice s the values multiplying
-// codes stored as 4^k * q are divided by 4^k.  Fragment word for (group G, lane
-// column t, slice s, half which) sits at uint32 index ((G*4 + t)*4 + s)*2 +
-// which; info[G] = (2^-sh, sum of the group's values).
-__device__ __forceinline__ void frag_group(float v0, float v1, int G, int bits, uint32_t* frag, float2* info,
-                                           int lane) {
-  uint32_t m = max(__float_as_uint(fabsf(v0)), __float_as_uint(fabsf(v1)));
-  m = __reduce_max_sync(0xffffffffu, m);
-  float sum = v0 + v1;
+// fp16 B fragments of NG 64-value groups G0..G0+NG-1 (those below g_end), built
+// by one warp; lane l holds values 2l and 2l+1 of group k in (lo[k], hi[k]).
+// Each group is scaled by 2^sh so its largest magnitude lies in [2^14, 2^15);
+// within slice s the values multiplying codes stored as 4^k * q are divided by
+// 4^k.  Fragment word for (group G, lane column t, slice s, half which) sits at
+// uint32 index ((G*4 + t)*4 + s)*2 + which; info[G] = (2^-sh, sum of the
+// group's values, summed in xor-butterfly order).  The NG groups' reductions
+// are independent, so they overlap instead of running one after another.
+template <int NG>
+__device__ __forceinline__ void frag_batch(const float (&lo)[NG], const float (&hi)[NG], int G0, int g_end,
+                                           int bits, uint32_t* frag, float2* info, int lane) {
+  uint32_t m[NG];
+  float sum[NG];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  const int e = (int)((m >> 23) & 0xFF) - 127;  // exponent of the group maximum
-  int sh = (m == 0) ? 0 : 14 - max(e, -126);
-  sh = min(sh, 126);
-  const int k = 2 * lane, s = k / 16, kk = k % 16, which = kk / 8, t = (kk % 8) / 2;
+  for (int k = 0; k < NG; ++k) {
+    m[k] = max(__float_as_uint(fabsf(lo[k])), __float_as_uint(fabsf(hi[k])));
+    sum[k] = lo[k] + hi[k];
+  }
+#pragma unroll
+  for (int k = 0; k < NG; ++k) m[k] = __reduce_max_sync(0xffffffffu, m[k]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int k = 0; k < NG; ++k) sum[k] += __shfl_xor_sync(0xffffffffu, sum[k], o);
+  }
+  const int q = 2 * lane, s = q / 16, qq = q % 16, which = qq / 8, t = (qq % 8) / 2;
   const int fs = (bits == 4) ? (which ? 4 : 0) : ((s & 1) ? 4 : 0) + (which ? 2 : 0);
-  const float scl = exp2i(sh - fs);
-  __half2 h2 = __floats2half2_rn(v0 * scl, v1 * scl);
-  frag[((G * 4 + t) * 4 + s) * 2 + which] = *reinterpret_cast<uint32_t*>(&h2);
-  if (lane == 0) info[G] = make_float2(exp2i(-sh), sum);
+#pragma unroll
+  for (int k = 0; k < NG; ++k) {
+    if (G0 + k < g_end) {
+      const int e = (int)((m[k] >> 23) & 0xFF) - 127;  // exponent of the group maximum
+      int sh = (m[k] == 0) ? 0 : 14 - max(e, -126);
+      sh = min(sh, 126);
+      const float scl = exp2i(sh - fs);
+      __half2 h2 = __floats2half2_rn(lo[k] * scl, hi[k] * scl);
+      frag[(((G0 + k) * 4 + t) * 4 + s) * 2 + which] = *reinterpret_cast<uint32_t*>(&h2);
+      if (lane == 0) info[G0 + k] = make_float2(exp2i(-sh), sum[k]);
+    }
+  }
 }
 
 // Dot products of n consecutive tiles (groups G0..G0+n-1 of the input) with the
 // fragments in shared memory.
 template <int BITS>
-__device__ __forceinline__ void chunk_dot(const uint8_t* tiles, int n, const uint32_t* frag, const float2* info,
-                                          int G0, int lane, float& acc0, float& acc1) {
+__device__ __noinline__ float2 chunk_dot(const uint8_t* tiles, int n, const uint32_t* frag, const float2* info,
+                                          int G0, int lane) {
+  float acc0 = 0.f, acc1 = 0.f;
   constexpr int TB = 16 * kGroup * BITS / 8 + 64;
   const int t = lane & 3;
 #pragma unroll 4
@@ -235,16 +250,75 @@ __device__ __forceinline__ void chunk_dot(const uint8_t* tiles, int n, const uin
     const uint2 bf[4] = {make_uint2(x.x, x.y), make_uint2(x.z, x.w), make_uint2(y.x, y.y), make_uint2(y.z, y.w)};
     tile_dot<BITS>(tiles + tt * TB, bf, info[G], lane, acc0, acc1);
   }
+  return make_float2(acc0, acc1);
+}
+
+// Router order as one 64-bit key: larger logit first, then lower index.  The
+// logit bits map to an unsigned key that orders like the float (NaN was
+// already mapped to -inf, -0 counts as +0); the low word is ~index, so ties go to the lower
+// index.  Key 0 lies below every real entry.
+__device__ __forceinline__ uint64_t router_key(float v, int i) {
+  const uint32_t u = (v == 0.f) ? 0u : __float_as_uint(v);  // -0 ranks with +0
+  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((uint64_t)k << 32) | (uint32_t)~i;
+}
+__device__ __forceinline__ float router_key_logit(uint64_t key) {
+  const uint32_t k = (uint32_t)(key >> 32);
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Top-K of the router logits lg[0..E) (shared memory) in router-key order.
+// Round k takes the largest key below the previous pick: each lane reduces its
+// entries with a tree of independent maxima, then two warp reductions find the
+// warp maximum (high word, then low word among the lanes that hold it).
+// Nothing is written, so a dry run on any data is harmless.  Lane k < K
+// receives pick k.
+struct TopPick {
+  float logit;
+  int expert;
+};
+__device__ __noinline__ TopPick topk_select(const float* lg, int E, int K, int lane) {
+  constexpr int kPer = 16;  // entries per lane per pass
+  uint64_t prev = ~0ull;
+  TopPick mine = {-INFINITY, 0};
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    uint64_t best = 0ull;
+#pragma unroll 1
+    for (int base = 0; base < E; base += 32 * kPer) {
+      uint64_t c[kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = base + j * 32 + lane;
+        const uint64_t key = i < E ? router_key(lg[i], i) : 0ull;
+        c[j] = key < prev ? key : 0ull;
+      }
+#pragma unroll
+      for (int w = kPer / 2; w > 0; w >>= 1) {
+#pragma unroll
+        for (int j = 0; j < w; ++j) c[j] = c[j] > c[j + w] ? c[j] : c[j + w];
+      }
+      best = c[0] > best ? c[0] : best;
+    }
+    const uint32_t hmax = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32));
+    const uint32_t lmax = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32) == hmax ? (uint32_t)best : 0u);
+    prev = ((uint64_t)hmax << 32) | lmax;
+    if (lane == k && prev != 0ull) mine = {router_key_logit(prev), (int)~lmax};
+  }
+  return mine;
 }
 
 // Bounded waits; they also give up when another warp of the block aborted.
+// Spinning warps back off with a short sleep and read the global timer only
+// every few rounds, so they take few issue slots from working warps.
 __device__ __forceinline__ bool wait_mbar(uint32_t bar, uint32_t parity, uint64_t limit,
                                           const volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = gtimer();
-  for (;;) {
+  const uint64_t t0 = gtimer();
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag || gtimer() - t0 > limit) return false;
+    if ((it & 7) == 7 && (*abort_flag || gtimer() - t0 > limit)) return false;
+    if (it >= 4) __nanosleep(32);
   }
 }
 __device__ __forceinline__ bool wait_flag(const volatile int* f, int value, uint64_t limit,
@@ -326,31 +400,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       // published; each lane keeps experts lane, lane+32, ... in registers
       // (up to 512 experts; beyond that the values are staged in shared memory).
       const uint32_t tag = *reinterpret_cast<volatile uint32_t*>(&P.ws->epoch) + 1u;
-      constexpr int kRegE = 16;
-      const bool in_regs = P.E <= 32 * kRegE;
-      float vals[kRegE];
+      constexpr int kPollE = 16;  // logits per lane per load round
       float* lg = reinterpret_cast<float*>(smem + P.off_lg);
       const uint64_t t0 = gtimer();
       for (;;) {
         bool mine = true;
-        for (int base = 0; base < P.E; base += 32 * kRegE) {
-          uint64_t v[kRegE];
+        for (int base = 0; base < P.E; base += 32 * kPollE) {
+          uint64_t v[kPollE];
 #pragma unroll
-          for (int k = 0; k < kRegE; ++k) {
+          for (int k = 0; k < kPollE; ++k) {
             const int i = base + k * 32 + lane;
             v[k] = i < P.E ? ld_tagged(P.ws_logits + i) : 0ull;
           }
 #pragma unroll
-          for (int k = 0; k < kRegE; ++k) {
+          for (int k = 0; k < kPollE; ++k) {
             const int i = base + k * 32 + lane;
-            float f = -INFINITY;
             if (i < P.E) {
               mine = mine && tagged_tag(v[k]) == tag;
-              f = tagged_value(v[k]);
-              f = (f != f) ? -INFINITY : f;
-              if (!in_regs) lg[i] = f;
+              const float f = tagged_value(v[k]);
+              lg[i] = (f != f) ? -INFINITY : f;
             }
-            vals[k] = f;
           }
         }
         if (__all_sync(0xffffffffu, mine)) break;
@@ -364,58 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
       }
       __syncwarp();
-      // K rounds of warp arg-max (ties: lower index).  Each lane keeps the best
-      // of its own values; a round is two warp reductions (max of an
-      // order-preserving key, then min index among lanes holding it) and only
-      // the winning lane rescans.  Lane k keeps result k in scalars.
-      float my_top = -INFINITY;
-      int my_sel = 0;
-      float lb = -INFINITY;
-      int li = P.E;
-      auto rescan = [&]() {
-        lb = -INFINITY;
-        li = P.E;
-        if (in_regs) {
-#pragma unroll
-          for (int kk = 0; kk < kRegE; ++kk) {
-            const int i = kk * 32 + lane;
-            const bool better = i < P.E && vals[kk] == vals[kk] && (li == P.E || vals[kk] > lb);
-            lb = better ? vals[kk] : lb;
-            li = better ? i : li;
-          }
-        } else {
-          for (int i = lane; i < P.E; i += 32) {
-            const float v = lg[i];
-            if (v == v && (li == P.E || v > lb)) { lb = v; li = i; }
-          }
-        }
-      };
-      rescan();
-#pragma unroll 1
-      for (int k = 0; k < P.K; ++k) {
-        uint32_t key = 0u;  // below every real entry
-        if (li < P.E) {
-          const uint32_t u = __float_as_uint(lb);
-          key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-        }
-        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
-        const uint32_t win = __reduce_min_sync(0xffffffffu, (key == kmax && li < P.E) ? (uint32_t)li : 0xFFFFFFFFu);
-        const int bi = win < (uint32_t)P.E ? (int)win : 0;
-        const float bv = __shfl_sync(0xffffffffu, lb, bi & 31);
-        if (lane == k) { my_top = bv; my_sel = bi; }
-        if (lane == (bi & 31) && win < (uint32_t)P.E) {
-          // taken entries become NaN (loaded NaNs were turned into -inf), so
-          // the rescan skips them even among -inf ties
-          if (in_regs) {
-#pragma unroll
-            for (int kk = 0; kk < kRegE; ++kk) vals[kk] = (kk * 32 + lane == bi) ? __int_as_float(0x7fc00000) : vals[kk];
-          } else {
-            lg[bi] = __int_as_float(0x7fc00000);
-          }
-          rescan();
-        }
-        __syncwarp();
-      }
+      const TopPick pick = topk_select(lg, P.E, P.K, lane);
+      const float my_top = pick.logit;
+      const int my_sel = pick.expert;
       // renormalised weights over the K selected: p_k / sum_j p_j = e^(l_k - l_0) / sum_j e^(l_j - l_0)
       const float top0 = __shfl_sync(0xffffffffu, my_top, 0);
       const float ex = lane < P.K ? expf(my_top - top0) : 0.f;
@@ -535,14 +555,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       if (c0 < P.H) *reinterpret_cast<uint4*>(zs + c0) = hv;
       asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
       if (P.n_slots > 0) {
-        for (int Gi = warp; Gi < P.H / kGroup; Gi += kConsumerWarps) {
-          const uint32_t zz = *reinterpret_cast<const uint32_t*>(zs + Gi * kGroup + 2 * lane);
-          frag_group(bf16lo(zz), bf16hi(zz), Gi, BITS, zfrag, zinfo, lane);
+        // warp w builds groups 4w..4w+3, then 4(w+16).., so a batch is contiguous
+        const int ngz = P.H / kGroup;
+        for (int G0 = 4 * warp; G0 < ngz; G0 += 4 * kConsumerWarps) {
+          float lo[4], hi[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t zz = (G0 + k < ngz) ? *reinterpret_cast<const uint32_t*>(zs + (G0 + k) * kGroup + 2 * lane) : 0u;
+            lo[k] = bf16lo(zz);
+            hi[k] = bf16hi(zz);
+          }
+          frag_batch<4>(lo, hi, G0, ngz, BITS, zfrag, zinfo, lane);
         }
       }
       asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
     }
 
+    // The producer selects the routed experts once per launch, late; running
+    // the same selection code here on whatever the logit buffer holds (it
+    // writes nothing) brings that code into the instruction cache meanwhile.
+    if (warp == kConsumerWarps - 1 && P.mode != kModeExpert) {
+      const TopPick dummy = topk_select(reinterpret_cast<const float*>(smem + P.off_lg), P.E, P.K, lane);
+      if (dummy.expert < 0) misc->pad[0] = dummy.expert;  // never true; keeps the call
+    }
     // ---- task loop: warp w takes tasks w, w+16, ...
     for (int i = warp; i < n_tasks; i += kConsumerWarps) {
       int s, fill;
@@ -598,8 +633,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
       } else if (ty == kTaskGateUp) {
         const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
-        float acc0 = 0.f, acc1 = 0.f;
-        chunk_dot<BITS>(stage, n, zfrag, zinfo, (int)c * kChunkTiles, lane, acc0, acc1);
+        const float2 acc = chunk_dot<BITS>(stage, n, zfrag, zinfo, (int)c * kChunkTiles, lane);
+        float acc0 = acc.x, acc1 = acc.y;
         const int u = cta + (int)idx * G, rb = u % P.units_per_slot;
         bool last = true;
         if (P.gu_chunks > 1) {
@@ -630,17 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const bool writer = P.gu_chunks > 1 ? lane < 8 : (lane & 3) == 0;
           const float av = writer ? acc0 / (1.0f + expf(-acc0)) * acc1 : 0.f;
           if (writer) st_tagged(P.ws_a + (int64_t)slot * P.I + rb * 8 + row, av, tag);
-          // the unit's sum (fixed tree order) and max |a| (order-free) let
-          // readers scale and fold the bias without reducing 64 values each
-          float us = av;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) us += __shfl_xor_sync(0xffffffffu, us, o);
-          const uint32_t um = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(av)));
-          if (lane == 0) {
-            st_tagged(P.ws_asum + (int64_t)slot * P.units_per_slot + rb, us, tag);
-            atom_max_u64(P.ws_amax + slot, ((uint64_t)tag << 32) | um);
-            red_relaxed_add(&P.ws->h_cnt[slot], 1u);
-          }
+          if (lane == 0) red_relaxed_add(&P.ws->h_cnt[slot], 1u);
         }
       } else {
         // activations of this slot as fragments (built once per block)
@@ -651,83 +676,42 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         claimed = __shfl_sync(0xffffffffu, claimed, 0);
         int good = 1;
         if (claimed) {
-          // poll the slot's tagged activations (published by every block's
-          // gate/up units), 8 groups at a time, and turn them into fragments
+          // The slot's activations are tagged words published by every block's
+          // gate/up units.  Each lane fetches its pair (2*lane, 2*lane+1) of up
+          // to kFetchGroups groups in one round trip and the round is repeated
+          // until every tag is current; the published count only paces the
+          // retries.  Each group then gets its own power-of-two scale and sum,
+          // exactly as the input z does.
           const uint64_t* act = P.ws_a + (int64_t)slot * P.I;
           const int ng = P.I / kGroup;
           const uint64_t t0 = gtimer();
-          good = __all_sync(0xffffffffu,
-                            wait_count(&P.ws->h_cnt[slot], (uint32_t)P.units_per_slot, limit, abort_flag));
-          if (!good && lane == 0) {
-            if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
-            *abort_flag = 1;
-          }
-          // One scale per slot, 2^sh with the slot's largest |a| in [2^14, 2^15)
-          // (from the producers' tag-keyed atomic max), and each group's sum from
-          // its 8 units' published sums (fixed order): no reductions here.
-          float scl_base = 0.f, inv = 1.f;
-          if (good) {
-            for (;;) {
-              const uint64_t mw = ld_tagged(P.ws_amax + slot);
-              if (__all_sync(0xffffffffu, tagged_tag(mw) == tag)) {
-                const uint32_t m = (uint32_t)mw;
-                const int e = (int)((m >> 23) & 0xFF) - 127;
-                int sh = (m == 0) ? 0 : 14 - max(e, -126);
-                sh = min(sh, 126);
-                scl_base = exp2i(sh);
-                inv = exp2i(-sh);
-                break;
-              }
-              __nanosleep(64);
-              if (__any_sync(0xffffffffu, *abort_flag != 0 || gtimer() - t0 > limit)) {
-                good = 0;
-                break;
-              }
-            }
-          }
-          // this lane's pair (2*lane, 2*lane+1) of every group sits at one
-          // position of the fragment layout
-          const int kq = 2 * lane, sq = kq / 16, kkq = kq % 16, whq = kkq / 8, tq = (kkq % 8) / 2;
-          const int fsq = (BITS == 4) ? (whq ? 4 : 0) : ((sq & 1) ? 4 : 0) + (whq ? 2 : 0);
-          const float scl = scl_base * exp2i(-fsq);
-          for (int g0 = 0; g0 < ng && good; g0 += 4) {
-            ulonglong2 v[4];
-            ulonglong2 su[4];
-            const int gs = g0 + lane;  // group whose sum this lane assembles
-            for (;;) {
+          for (int g0 = 0; g0 < ng && good; g0 += kFetchGroups) {
+            ulonglong2 v[kFetchGroups];
+            for (int attempt = 0;; ++attempt) {
               bool mine = true;
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
+              for (int k = 0; k < kFetchGroups; ++k) {
                 v[k] = (g0 + k < ng) ? ld_tagged2(act + (g0 + k) * kGroup + 2 * lane) : make_ulonglong2(0ull, 0ull);
                 if (g0 + k < ng) mine = mine && tagged_tag(v[k].x) == tag && tagged_tag(v[k].y) == tag;
               }
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                su[k] = (lane < 4 && gs < ng) ? ld_tagged2(P.ws_asum + (int64_t)slot * P.units_per_slot + gs * 8 + 2 * k)
-                                              : make_ulonglong2(0ull, 0ull);
-                if (lane < 4 && gs < ng) mine = mine && tagged_tag(su[k].x) == tag && tagged_tag(su[k].y) == tag;
-              }
               if (__all_sync(0xffffffffu, mine)) break;
-              __nanosleep(64);
-              if (__any_sync(0xffffffffu, *abort_flag != 0 || gtimer() - t0 > limit)) {
+              // not all published yet: wait for the count, then fetch again
+              const bool counted =
+                  wait_count(&P.ws->h_cnt[slot], (uint32_t)P.units_per_slot, limit, abort_flag);
+              if (__any_sync(0xffffffffu, !counted || *abort_flag != 0 || gtimer() - t0 > limit)) {
                 good = 0;
                 break;
               }
+              if (attempt > 0) __nanosleep(256);
             }
             if (!good) break;
-            if (lane < 4 && gs < ng) {
-              float gsum = 0.f;
+            float lo[kFetchGroups], hi[kFetchGroups];
 #pragma unroll
-              for (int k = 0; k < 4; ++k) gsum += tagged_value(su[k].x) + tagged_value(su[k].y);
-              ai[gs] = make_float2(inv, gsum);
+            for (int k = 0; k < kFetchGroups; ++k) {
+              lo[k] = tagged_value(v[k].x);
+              hi[k] = tagged_value(v[k].y);
             }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              if (g0 + k < ng) {
-                __half2 h2 = __floats2half2_rn(tagged_value(v[k].x) * scl, tagged_value(v[k].y) * scl);
-                af[(((g0 + k) * 4 + tq) * 4 + sq) * 2 + whq] = *reinterpret_cast<uint32_t*>(&h2);
-              }
-            }
+            frag_batch<kFetchGroups>(lo, hi, g0, ng, BITS, af, ai, lane);
           }
           if (!good && lane == 0) {
             if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
@@ -751,8 +735,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         if (!good) break;
         const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
-        float acc0 = 0.f, acc1 = 0.f;
-        chunk_dot<BITS>(stage, n, af, ai, (int)c * kChunkTiles, lane, acc0, acc1);
+        const float2 acc = chunk_dot<BITS>(stage, n, af, ai, (int)c * kChunkTiles, lane);
+        const float acc0 = acc.x, acc1 = acc.y;
         float* y = ys + ((int)idx * P.n_slots + (int)slot) * 16;
         if (P.dn_chunks == 1) {
           if ((lane & 3) == 0) { y[lane >> 2] = acc0; y[8 + (lane >> 2)] = acc1; }

@@ -38,6 +38,7 @@ constexpr int kConsumerWarps = 16;       // warps that compute
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kChunkTiles = 16;          // tiles per gate/up or down task
 constexpr int kMaxTasks = 96;            // task-list capacity per block (multiple of 32)
+constexpr int kFetchGroups = 8;          // activation groups a warp fetches per round trip
 
 inline __host__ __device__ int tile_code_bytes(int bits) { return 16 * kGroup * bits / 8; }
 inline __host__ __device__ int tile_bytes(int bits) { return tile_code_bytes(bits) + 64; }
@@ -152,8 +153,6 @@ struct DecodePlan {
   WsHeader* ws;
   uint64_t* ws_logits;     // [E] tagged
   uint64_t* ws_a;          // [kMaxSlots][I] tagged
-  uint64_t* ws_asum;       // [kMaxSlots][I/8] tagged per-unit sums of a
-  uint64_t* ws_amax;       // [kMaxSlots] (tag << 32) | bits of max |a| (atomic max)
   const uint32_t* tasks;   // [grid][kMaxTasks] ordered task lists (host-built)
   const int32_t* n_tasks;  // [grid]
   uint32_t flags;
