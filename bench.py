@@ -233,14 +233,20 @@ def barrier(ws):
         dist.barrier()
 
 
-def max_over_ranks(ws, value: float) -> float:
+def max_over_ranks(ws, value: float, device: str = "cuda") -> float:
+    """The largest of every rank's value (timings are taken as the slowest rank)."""
     if ws == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(ws: int, units_per_rank: int, max_ms: float) -> float:
+    """Whole-job units/s: every rank's units over the slowest rank's time."""
+    return ws * units_per_rank / (max_ms / 1e3)
 
 
 def run_gpu(args, wl, ws, rank, local):
@@ -339,7 +345,7 @@ def run_gpu(args, wl, ws, rank, local):
     if rank != 0:
         return 0
     ms_per_step = total_ms / steps
-    tps = ws * steps / (total_ms / 1e3)
+    tps = job_throughput(ws, steps, total_ms)
     us_layer = 1e3 * ms_per_step / L
     bytes_launch = layer_bytes(wl)
     achieved = bytes_launch / (us_layer * 1e-6) / 1e9
@@ -364,7 +370,7 @@ def run_gpu(args, wl, ws, rank, local):
                      "algorithmic_bytes_per_launch": bytes_launch},
         "step_us_p10_p50_p90": [1e3 * q for q in statistics.quantiles(step_ms, n=10)[0::4]] if steps >= 10 else None,
         "warm_l2_us_per_layer": warm_us,
-        "e2e": {"value": ws * e2e_steps / (e2e_total / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(ws, e2e_steps, e2e_total), "unit": "tokens/s",
                 "h2d_bytes_per_step": wl.hidden * 2, "d2h_bytes_per_step": wl.hidden * 2},
         "gpu_launches": steps * L,
         "clocks": clocks,

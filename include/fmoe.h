@@ -3,11 +3,15 @@
  * NVIDIA B200 (sm_100a).
  *
  * One call runs one mixture-of-experts layer of the decode step that the
- * Flash-MoE pages describe (page 5 "How the SSD expert streaming pipeline
- * works": CMD2 runs the norm, the routing GEMV and the shared expert, the CPU
- * takes softmax and top-K, CMD3 runs the expert forward pass plus combine; page
- * 2 Key Takeaways: 512 experts per layer, K = 4 active; page 4 "The
- * Architecture": 4-bit experts of about 6.75 MB dequantised by an FMA kernel).
+ * Flash-MoE pages describe.  The Hysen Labs page "Flash-MoE: Running a 397B
+ * Parameter Model on a Laptop", section "How the SSD expert streaming pipeline
+ * works", splits it over a GPU command buffer (normalisation, routing GEMV,
+ * shared expert), the host (softmax and top-K) and a second command buffer
+ * (the routed experts and the combine).  The themata summary of the same title
+ * (Key Takeaways) gives 512 experts per layer with K = 4 active; "Flash-MoE:
+ * Running a 400 Billion Parameter Model on a MacBook", section "The
+ * Architecture", sizes a 4-bit expert at about 6.75 MB and dequantises it with
+ * fused multiply-adds.
  * Here every step runs on the GPU and all expert weights stay resident in HBM.
  *
  * Conventions for every entry point
@@ -95,8 +99,8 @@ typedef struct fmoe_layer_desc {
  *           c / (32/bits) of that row;
  *   scales: bf16 [R][C/64];  biases: bf16 [R][C/64];
  * weight w[r][c] = scale[r][c/64] * code[r][c] + bias[r][c/64].
- * At H = 4096, I = 1024 a blob is 7,077,888 bytes at 4 bits (the pages' "about
- * 6.75 MB" per expert) and 3,932,160 bytes at 2 bits.
+ * At H = 4096, I = 1024 a blob is 7,077,888 bytes at 4 bits (the pages size an
+ * expert at about 6.75 MB) and 3,932,160 bytes at 2 bits.
  */
 FMOE_API size_t fmoe_expert_bytes(int32_t hidden, int32_t inter, int32_t bits);
 

@@ -7,9 +7,11 @@ with it.
 
 The arithmetic lives in ``oracle.c`` (built into ``liboracle.so`` with gcc);
 this module marshals numpy arrays and composes the steps of one layer in the
-order the Flash-MoE pages give them (page 5, "How the SSD expert streaming
-pipeline works": norm and routing in CMD2, softmax and top-K on the CPU, then
-CMD3 runs the expert forward pass, the combine and the norm).
+order the Flash-MoE pages give them (the Hysen Labs page "Flash-MoE: Running a
+397B Parameter Model on a Laptop", section "How the SSD expert streaming
+pipeline works": normalisation and routing in the second command buffer,
+softmax and top-K on the host, then the third command buffer runs the experts
+and combines their outputs).
 """
 from __future__ import annotations
 
@@ -155,7 +157,7 @@ def layer_forward(h, *, router_w, router_bias, norm_w, eps, top_k, hidden, inter
 
     ``blob_of(e)`` returns the canonical blob of expert e (0..E-1 routed, E the
     shared expert); it is only asked for the K selected experts and the shared
-    one.  Steps, in the order of page 5's pipeline: norm -> router -> softmax
+    one.  Steps, in the order of that page's pipeline: norm -> router -> softmax
     and top-K -> expert forward (K routed + shared) -> combine into the residual.
     Returns a dict with z, logits, idx, w, y (routed, [K][H]), y_shared, out_f64
     and out (bf16 bits).

@@ -51,8 +51,9 @@ static int64_t matrix_bytes(int hidden, int inter, int bits, int m) {
   return R * C * bits / 8 + 2 * 2 * R * (C / GROUP);
 }
 
-/* Page 4 "The Architecture" puts one 4-bit expert at roughly 6.75 MB; three
- * matrices of 4096 x 1024 codes plus a bf16 scale and bias per 64 codes give
+/* "Flash-MoE: Running a 400 Billion Parameter Model on a MacBook",
+ * section "The Architecture", sizes one 4-bit expert at about
+ * 6.75 MB; three matrices of 4096 x 1024 codes plus a bf16 scale and bias per 64 codes give
  * exactly 7,077,888 bytes = 6.75 MiB. */
 int64_t orc_blob_bytes(int hidden, int inter, int bits) {
   return matrix_bytes(hidden, inter, bits, 0) + matrix_bytes(hidden, inter, bits, 1) +
@@ -60,9 +61,10 @@ int64_t orc_blob_bytes(int hidden, int inter, int bits) {
 }
 
 /* Dequantisation, w = q * scale + bias with one bf16 (scale, bias) per group of
- * 64 consecutive columns of a row (page 4 "The Architecture": FMA dequant in the
- * inner loop; the affine form, group size and dtypes are the readings fixed for
- * this build).  Code c of row r is field c % (32/bits) of little-endian 32-bit
+ * 64 consecutive columns of a row ("Flash-MoE: Running a 400 Billion Parameter Model on a MacBook",
+ * section "The Architecture": the inner
+ * loop dequantises with fused multiply-adds; the affine form, group size and
+ * dtypes are the readings fixed for this build).  Code c of row r is field c % (32/bits) of little-endian 32-bit
  * word c / (32/bits) of that row. */
 double orc_weight(const uint8_t* blob, int hidden, int inter, int bits, int m, int r, int c) {
   int64_t off = 0;
@@ -84,8 +86,10 @@ double orc_weight(const uint8_t* blob, int hidden, int inter, int bits, int m, i
   return orc_bf16_value(s16) * (double)q + orc_bf16_value(b16);
 }
 
-/* RMSNorm ahead of the mixture-of-experts block (page 5: CMD2 runs "norm" before
- * routing; the epsilon is the build's reading). */
+/* RMSNorm ahead of the mixture-of-experts block (the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on a Laptop",
+ * section "How the SSD expert streaming pipeline works":
+ * the second command buffer normalises before it routes; the epsilon is the
+ * build's reading). */
 void orc_rmsnorm(const uint16_t* h, const uint16_t* w, int hidden, double eps, uint16_t* z) {
   double ss = 0.0;
   for (int i = 0; i < hidden; ++i) {
@@ -99,8 +103,11 @@ void orc_rmsnorm(const uint16_t* h, const uint16_t* w, int hidden, double eps, u
   }
 }
 
-/* Router GEMV, hidden -> one logit per expert (page 5: CMD2 does "routing";
- * Key Takeaways of page 2: 512 experts per layer). */
+/* Router GEMV, hidden -> one logit per expert (the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on a Laptop",
+ * section "How the SSD expert streaming pipeline works":
+ * the second command buffer computes the routing; the themata summary "Flash-MoE: Running a 397B Parameter Model on a Laptop",
+ * Key Takeaways:
+ * 512 experts per layer). */
 void orc_router_logits(const uint16_t* wr, const float* bias, const uint16_t* z, int hidden, int n_experts,
                        float* logits) {
 #pragma omp parallel for schedule(static)
@@ -122,8 +129,11 @@ static int by_prob_desc(const void* a, const void* b) {
   return (x->e > y->e) - (x->e < y->e);
 }
 
-/* Softmax and top-K (page 5: "the CPU does softmax and topK routing"; K = 4 per
- * page 2).  Renormalising the K selected probabilities is the build's reading. */
+/* Softmax and top-K (the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on a Laptop",
+ * section "How the SSD expert streaming pipeline works":
+ * the host takes the softmax and picks the top K; the themata summary "Flash-MoE: Running a 397B Parameter Model on a Laptop",
+ * Key Takeaways: K = 4).
+ * Renormalising the K selected probabilities is the build's reading. */
 void orc_topk(const float* logits, int n_experts, int top_k, int32_t* idx, double* w, double* p) {
   double mx = -INFINITY;
   for (int e = 0; e < n_experts; ++e) mx = fmax(mx, (double)logits[e]);
@@ -148,10 +158,13 @@ void orc_topk(const float* logits, int n_experts, int top_k, int32_t* idx, doubl
   free(ent);
 }
 
-/* SwiGLU expert feed-forward with inline dequantisation (page 5: CMD3 "encodes
- * the expert forward pass"; page 4: FMA dequant kernel).  silu(t) = t/(1+e^-t)
- * applied to the gate projection, times the up projection, is the build's
- * reading of the activation. */
+/* SwiGLU expert feed-forward with inline dequantisation (the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on a Laptop",
+ * section "How the SSD expert streaming pipeline works":
+ * the third command buffer runs the experts; "Flash-MoE: Running a 400 Billion Parameter Model on a MacBook",
+ * section "The Architecture":
+ * dequantisation fused into the multiply-adds).  silu(t) = t/(1+e^-t) applied
+ * to the gate projection, times the up projection, is the build's reading of
+ * the activation. */
 void orc_expert(const uint8_t* blob, int hidden, int inter, int bits, const uint16_t* z, double* g, double* u,
                 double* a, double* y) {
   double* gg = (double*)malloc(sizeof(double) * (size_t)inter);
@@ -183,8 +196,10 @@ void orc_expert(const uint8_t* blob, int hidden, int inter, int bits, const uint
   free(aa);
 }
 
-/* Weighted combine into the residual (page 5: CMD3 "plus combine"); the shared
- * expert (page 5: "plus one shared expert") enters with weight 1. */
+/* Weighted combine into the residual (the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on a Laptop",
+ * section "How the SSD expert streaming pipeline works":
+ * the third command buffer also combines the expert outputs); the shared expert
+ * that the same section adds to the K routed ones enters with weight 1. */
 void orc_combine(const uint16_t* h, const double* w, const double* y_routed, const double* y_shared, int hidden,
                  int top_k, double* out_f64, uint16_t* out) {
   for (int j = 0; j < hidden; ++j) {

@@ -7,8 +7,10 @@
  * library; both only read the same canonical expert blobs produced by the
  * seeded generator.
  *
- * What it computes (pages: "Flash-MoE" wiki, Technical Architecture; page 5
- * "How the SSD expert streaming pipeline works"; page 4 "The Architecture"):
+ * What it computes (pages: the wiki page "Flash-MoE", Technical Architecture;
+ * the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on a Laptop",
+ * section "How the SSD expert streaming pipeline works"; "Flash-MoE: Running a
+ * 400 Billion Parameter Model on a MacBook", section "The Architecture"):
  * per token and layer, optional RMSNorm of the layer input, router GEMV over
  * E experts, softmax, top-K selection with the selected probabilities
  * renormalised, SwiGLU feed-forward of the K selected experts and of one shared

@@ -83,8 +83,12 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
   P.rb_per_cta = P.n_slots > 0 ? (P.n_rb + grid - 1) / grid : 0;
   const bool router = mode != kModeExpert;
   P.router_rows = router ? (c.n_experts + grid - 1) / grid : 0;
-  // up to 4 non-empty parts of whole 64-column groups
-  const int rgroups = c.hidden / kGroup, per_part = (rgroups + 3) / 4;
+  // A router row is one task when it fits an expert stage (one copy, one warp);
+  // otherwise it is split into up to 4 non-empty parts of whole 64-column groups.
+  const int rgroups = c.hidden / kGroup;
+  const uint32_t expert_stage = (uint32_t)std::max(std::min(kChunkTiles, c.hidden / kGroup),
+                                                   std::min(kChunkTiles, c.inter / kGroup)) * tile_bytes(c.bits);
+  const int per_part = ((uint32_t)c.hidden * 2 <= expert_stage) ? rgroups : (rgroups + 3) / 4;
   P.router_part_cols = per_part * kGroup;
   P.router_parts = (rgroups + per_part - 1) / per_part;
   const int max_tasks =
@@ -147,6 +151,7 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
   nstage = best_ns;
   P.n_issuers = best_ni;
   P.nstage = nstage;
+  P.route_first = kRouteFirst;
   P.off_ring = off;
   off = align_up((uint32_t)nstage * P.stage_bytes, 128);
   P.off_z = off + r_z;

@@ -1,8 +1,10 @@
 // fmoe_decode.cu -- fused single-token mixture-of-experts layer for sm_100a.
 //
 // One cooperative launch, one block per SM, runs the whole decode step that the
-// Flash-MoE pages split over CMD2, the CPU and CMD3 (page 5 "How the SSD expert
-// streaming pipeline works"): optional RMSNorm, router GEMV, softmax + top-K,
+// Flash-MoE pages split over two GPU command buffers and the host (the Hysen
+// Labs page "Flash-MoE: Running a 397B Parameter Model on a Laptop", section
+// "How the SSD expert streaming pipeline works"): optional RMSNorm, router GEMV,
+// softmax + top-K,
 // the K routed and the shared SwiGLU experts with inline dequantisation, and the
 // weighted combine into the residual.
 //
@@ -281,6 +283,31 @@ __device__ __noinline__ TopPick topk_select(const float* lg, int E, int K, int l
   constexpr int kPer = 16;  // entries per lane per pass
   uint64_t prev = ~0ull;
   TopPick mine = {-INFINITY, 0};
+  if (E <= 32 * kPer) {
+    // keys computed once, kept in registers
+    uint64_t key[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = j * 32 + lane;
+      key[j] = i < E ? router_key(lg[i], i) : 0ull;
+    }
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+      uint64_t c[kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) c[j] = key[j] < prev ? key[j] : 0ull;
+#pragma unroll
+      for (int w = kPer / 2; w > 0; w >>= 1) {
+#pragma unroll
+        for (int j = 0; j < w; ++j) c[j] = c[j] > c[j + w] ? c[j] : c[j + w];
+      }
+      const uint32_t hmax = __reduce_max_sync(0xffffffffu, (uint32_t)(c[0] >> 32));
+      const uint32_t lmax = __reduce_max_sync(0xffffffffu, (uint32_t)(c[0] >> 32) == hmax ? (uint32_t)c[0] : 0u);
+      prev = ((uint64_t)hmax << 32) | lmax;
+      if (lane == k && prev != 0ull) mine = {router_key_logit(prev), (int)~lmax};
+    }
+    return mine;
+  }
 #pragma unroll 1
   for (int k = 0; k < K; ++k) {
     uint64_t best = 0ull;
@@ -308,7 +335,6 @@ __device__ __noinline__ TopPick topk_select(const float* lg, int E, int K, int l
   return mine;
 }
 
-// Bounded waits; they also give up when another warp of the block aborted.
 // Spinning warps back off with a short sleep and read the global timer only
 // every few rounds, so they take few issue slots from working warps.
 __device__ __forceinline__ bool wait_mbar(uint32_t bar, uint32_t parity, uint64_t limit,
@@ -359,9 +385,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   float h_res = 0.f;  // residual input of the row this thread combines
 
   // ---------------------------------------------------------------- set-up
-  if (warp == 0) {
+  // The producer initialises the ring and, before the block barrier, already
+  // issues the copies of its first router rows (tasks 0.. of every list, known
+  // without reading it): weights do not depend on the previous launch.
+  int pre_issued = 0;
+  if (warp == kConsumerWarps) {
     for (int i = lane; i < 2 * P.nstage; i += 32) mbar_init(bar_full + 8u * i, 1);
+    misc->last_task[lane] = -1;
+    misc->last_task[lane + 32] = -1;
     asm volatile("fence.mbarrier_init.release.cluster;\n fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (has_router && P.router_parts == 1) {
+      const int my_rrows = cta < P.E ? (P.E - cta + G - 1) / G : 0;
+      pre_issued = min(my_rrows, P.n_issuers);
+      if (lane < pre_issued) {
+        int s, fill;
+        task_stage(P.nstage, P.n_issuers, lane, s, fill);  // fill 0
+        const uint32_t bytes = (uint32_t)P.H * 2;
+        mbar_expect_tx(bar_full + 8u * s, bytes);
+        tma_load(smem_u32(smem + P.off_ring + (uint32_t)s * P.stage_bytes), P.router_w + (int64_t)(cta + lane * G) * P.H,
+                 bytes, bar_full + 8u * s);
+        reinterpret_cast<volatile int*>(misc->last_task)[s] = lane;
+      }
+    }
   } else if (warp == 1) {
     if (lane < 16) {
       misc->rcnt[lane] = 0;
@@ -371,8 +417,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
     misc->unit_cnt[lane] = 0;
     misc->dn_cnt[lane] = 0;
-    misc->last_task[lane] = -1;
-    misc->last_task[lane + 32] = -1;
     if (lane == 0) misc->abort = 0;
   } else if (warp == 2) {
     // this block's ordered task list, global -> shared
@@ -494,10 +538,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     for (int r = 0; r * NI < n_tasks; ++r) {
       if (__any_sync(0xffffffffu, *abort_flag)) break;
       const int i = r * NI + lane;
-      const bool mine = lane < NI && i < n_tasks;
+      const bool mine = lane < NI && i < n_tasks && i >= pre_issued;
       const uint32_t t = mine ? tasks[i] : 0u;
-      const bool needs_route =
-          mine && P.mode == kModeLayer && !routed && task_type(t) != kTaskRouter && task_slot(t) >= 1;
+      const bool needs_route = mine && P.mode == kModeLayer && !routed && task_type(t) != kTaskRouter &&
+                               (task_slot(t) >= 1 || P.route_first);
       int ok = 1;
       if (mine && !needs_route) ok = issue(i, t);
       if (!__all_sync(0xffffffffu, ok)) break;

@@ -1,8 +1,9 @@
 // fmoe_internal.h -- packed expert layout and kernel launch plans shared by the
 // host API (fmoe_api.cu) and the kernels (fmoe_repack.cu, fmoe_decode.cu).
 //
-// Packed tile layout (build-side design; the Flash-MoE pages only say experts
-// are ~6.75 MB blobs dequantised by an FMA kernel, page 4 "The Architecture").
+// Packed tile layout (build-side design; the Flash-MoE pages only size an
+// expert at about 6.75 MB and dequantise it with fused multiply-adds: "Flash-MoE:
+// Running a 400 Billion Parameter Model on a MacBook", section "The Architecture").
 // A tile is 16 weight rows x 64 input columns, i.e. one quantisation group per
 // row, laid out for one warp's mma.sync.m16n8k16 A fragments:
 //   codes: 32 lanes x (16*64*bits/8/32) bytes, lane l = 4*g + t owns rows g and
@@ -38,6 +39,7 @@ constexpr int kConsumerWarps = 16;       // warps that compute
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kChunkTiles = 16;          // tiles per gate/up or down task
 constexpr int kMaxTasks = 96;            // task-list capacity per block (multiple of 32)
+constexpr int kRouteFirst = 1;          // see DecodePlan::route_first
 constexpr int kFetchGroups = 8;          // activation groups a warp fetches per round trip
 
 inline __host__ __device__ int tile_code_bytes(int bits) { return 16 * kGroup * bits / 8; }
@@ -123,6 +125,7 @@ struct DecodePlan {
   int router_part_cols;    // columns per part (multiple of 64; the last part may be shorter)
   int nstage;              // ring stages (a multiple of n_issuers)
   int n_issuers;           // producer lanes issuing copies; lane l owns stages l, l+n_issuers, ...
+  int route_first;         // 1: route before issuing any expert copy (keeps the logit exchange off a busy memory pipe)
   uint32_t stage_bytes;
   // shared-memory layout (byte offsets)
   uint32_t off_ring;

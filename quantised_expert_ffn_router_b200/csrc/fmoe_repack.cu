@@ -5,8 +5,8 @@
 // codes so a warp loads them with one 16-byte (4-bit) or 8-byte (2-bit) shared
 // load per lane and unpacks them straight into mma.sync fragments, with the
 // tile's scales and biases next to its codes.  This is the B200 counterpart of
-// the pages' offline expert packing (page 3 "Weight Preparation",
-// repack_experts.py); it runs once, on device, at fmoe_create.
+// the pages' offline expert packing ("Flash-MoE Inference Engine", section
+// "Weight Preparation", step 2); it runs once, on device, at fmoe_create.
 #include <cuda_runtime.h>
 
 #include "fmoe_internal.h"

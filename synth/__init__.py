@@ -104,6 +104,10 @@ def cuda():
                                                      ctypes.c_uint32, ctypes.c_int64, ctypes.c_double,
                                                      ctypes.c_double, P, P]
             L.synth_cuda_gen_normal_bf16.restype = ctypes.c_int
+            L.synth_cuda_gen_normal_rows_bf16.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
+                                                          ctypes.c_uint32, ctypes.c_int, ctypes.c_int64,
+                                                          ctypes.c_double, ctypes.c_double, P, P]
+            L.synth_cuda_gen_normal_rows_bf16.restype = ctypes.c_int
             _cuda = L
     return _cuda
 
@@ -252,3 +256,14 @@ def device_norm_weight(wl: Workload, layer: int, dst_ptr: int, stream_ptr: int =
 
 def device_token(wl: Workload, index: int, subseed: int, dst_ptr: int, stream_ptr: int = 0):
     device_normal(wl.seed, subseed, T_TOKEN, index, wl.hidden, 0.0, wl.x_std, dst_ptr, stream_ptr)
+
+
+def device_token_range(wl: Workload, first: int, count: int, subseed: int, dst_ptr: int, stream_ptr: int = 0):
+    """Tokens first..first+count-1 (bf16 rows of H) in one launch; same bytes as device_token."""
+    rc = cuda().synth_cuda_gen_normal_rows_bf16(ctypes.c_uint64(wl.seed), ctypes.c_uint32(subseed),
+                                                ctypes.c_uint32(T_TOKEN), ctypes.c_uint32(first), count,
+                                                ctypes.c_int64(wl.hidden), ctypes.c_double(0.0),
+                                                ctypes.c_double(wl.x_std), ctypes.c_void_p(dst_ptr),
+                                                ctypes.c_void_p(stream_ptr))
+    if rc != 0:
+        raise RuntimeError(f"synth_cuda_gen_normal_rows_bf16 failed: cudaError {rc}")

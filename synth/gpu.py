@@ -8,7 +8,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (Workload, device_expert_blobs, device_norm_weight, device_router_weight, device_token, zipf_bias)
+from . import (Workload, device_expert_blobs, device_norm_weight, device_router_weight, device_token,
+               device_token_range, zipf_bias)
 
 
 class DeviceLayer:
@@ -50,6 +51,10 @@ def tokens(wl: Workload, indices, subseeds=None) -> torch.Tensor:
     """bf16 [len(indices)][H] device tensor of tokens `indices` (redraw `subseeds`)."""
     stream = torch.cuda.current_stream().cuda_stream
     out = torch.empty((len(indices), wl.hidden), dtype=torch.bfloat16, device="cuda")
+    idx = [int(t) for t in indices]
+    if subseeds is None and len(idx) > 1 and idx == list(range(idx[0], idx[0] + len(idx))):
+        device_token_range(wl, idx[0], len(idx), 0, out.data_ptr(), stream)
+        return out
     for r, t in enumerate(indices):
         s = 0 if subseeds is None else int(subseeds[r])
         device_token(wl, int(t), s, out[r].data_ptr(), stream)

@@ -3,9 +3,10 @@
  *
  * This module is test and benchmark infrastructure.  It produces the synthetic
  * tensors that stand in for the trained Qwen3.5-397B-A17B weights the Flash-MoE
- * pages run on (page "Flash-MoE: Running a 397B Parameter Model on a Laptop",
- * Key Takeaways: 60 layers, 512 experts, K=4; page 5 "How the SSD expert
- * streaming pipeline works": hidden 4096, one shared expert).  It holds none of
+ * pages run on (the themata summary "Flash-MoE: Running a 397B Parameter Model
+ * on a Laptop", Key Takeaways: 60 layers, 512 experts, K=4; the Hysen Labs page
+ * of the same title, section "How the SSD expert streaming pipeline works":
+ * hidden 4096, one shared expert).  It holds none of
  * the mixture-of-experts arithmetic: it only draws random bits and turns them
  * into bf16 numbers and packed integer codes in the canonical expert-blob format.
  *

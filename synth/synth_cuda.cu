@@ -26,6 +26,16 @@ __global__ void gen_normal_kernel(uint64_t key, int64_t n, double mean, double s
     out[i] = synth_normal_elem(key, i, mean, std);
 }
 
+// Rows r = 0..rows-1 of length n: row r is stream (seed, layer, tensor, item0 + r).
+__global__ void gen_normal_rows_kernel(uint64_t seed, uint32_t layer, uint32_t tensor, uint32_t item0, int rows,
+                                       int64_t n, double mean, double std, uint16_t* __restrict__ out) {
+  const int64_t total = (int64_t)rows * n, stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int r = (int)(i / n);
+    out[i] = synth_normal_elem(synth_key(seed, layer, tensor, item0 + (uint32_t)r), i % n, mean, std);
+  }
+}
+
 int grid_for(int64_t n) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -56,6 +66,17 @@ int synth_cuda_gen_normal_bf16(uint64_t seed, uint32_t layer, uint32_t tensor, u
   if (n <= 0) return 0;
   uint64_t key = synth_key(seed, layer, tensor, item);
   gen_normal_kernel<<<grid_for(n), 256, 0, (cudaStream_t)stream>>>(key, n, mean, std, (uint16_t*)dst);
+  return (int)cudaGetLastError();
+}
+
+/* Fills dst (device) with `rows` consecutive rows of n normal bf16 values; row r
+ * is the stream (seed, layer, tensor, item0 + r), identical to the single-row call. */
+int synth_cuda_gen_normal_rows_bf16(uint64_t seed, uint32_t layer, uint32_t tensor, uint32_t item0, int rows,
+                                    int64_t n, double mean, double std, void* dst, void* stream) {
+  if (n <= 0 || rows <= 0) return 0;
+  gen_normal_rows_kernel<<<grid_for((int64_t)rows * n), 256, 0, (cudaStream_t)stream>>>(seed, layer, tensor, item0,
+                                                                                     rows, n, mean, std,
+                                                                                     (uint16_t*)dst);
   return (int)cudaGetLastError();
 }
 

@@ -43,6 +43,15 @@ def _tokens(wl, n, layer=0, start=0):
     return idx, sub, tokens(wl, idx, sub)
 
 
+def test_device_tokens_match_host_generator(torch):
+    # a contiguous range is drawn by one launch; it must give the host bytes
+    from synth.gpu import tokens
+    for wl in (TINY, LAYER):
+        got = tokens(wl, range(5, 12)).view(torch.int16).cpu().numpy().view(np.uint16)
+        for r, t in enumerate(range(5, 12)):
+            assert np.array_equal(got[r], synth.token(wl, t)), (wl.name, t)
+
+
 @pytest.mark.parametrize("wl", SMALL + [STACK], ids=lambda w: w.name)
 def test_packed_layout_round_trip(torch, wl):
     with Model(wl) as m:
