@@ -128,6 +128,24 @@ FMOE_API fmoe_status fmoe_route(fmoe_ctx* ctx, int32_t layer, const void* x_dev,
                        float* w_dev, void* stream);
 
 /*
+ * The router step of fmoe_route (same inputs, outputs and selection rule)
+ * computed without any device allocation: its only scratch, the fp32 logits
+ * [T][E], is a fixed 128 KB device array inside the library.  The pages have
+ * no counterpart; it exists for callers that cannot allocate device memory per
+ * call -- a loop whose device memory is held entirely by its own pool
+ * allocator, or one that cannot take cudaFree's device-wide synchronisation.
+ * Limits: T * E <= 32768 and T <= 4096; larger calls return UNSUPPORTED
+ * before any GPU work.  The first call on a device looks up the array's
+ * address (cudaGetSymbolAddress); make it before any stream capture.  Calls
+ * that overlap in time share the array and race: order them on one stream.
+ * Logits accumulate in a different order than fmoe_route's, so weights may
+ * differ in the last bits; the indices agree except at near-ties.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA.
+ */
+FMOE_API fmoe_status fmoe_route_static(fmoe_ctx* ctx, int32_t layer, const void* x_dev, int32_t T,
+                                       int32_t* idx_dev, float* w_dev, void* stream);
+
+/*
  * One expert's SwiGLU feed-forward on the layer's (normed) input:
  * y = W_down (silu(W_gate z) * (W_up z)), z as in fmoe_route.
  *   expert  : 0..E-1 for a routed expert, -1 for the shared expert.

@@ -18,7 +18,7 @@ __all__ = [
     "FMOE_OK", "FMOE_ERR_INVALID_ARG", "FMOE_ERR_UNSUPPORTED", "FMOE_ERR_ALIGNMENT", "FMOE_ERR_CUDA",
     "FMOE_ERR_OOM", "FMOE_ERR_TIMEOUT", "FMOE_FLAG_FORCE_PER_TOKEN", "FMOE_FLAG_FORCE_GROUPED",
     "FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE", "Config", "LayerDesc", "FmoeError", "lib", "fmoe_expert_bytes",
-    "fmoe_create", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward", "fmoe_stack_forward",
+    "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward", "fmoe_layer_forward", "fmoe_stack_forward",
     "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error", "EXPORTED_SYMBOLS",
 ]
 
@@ -28,8 +28,8 @@ FMOE_FLAG_FORCE_PER_TOKEN = 0x1
 FMOE_FLAG_FORCE_GROUPED = 0x2
 FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE = 0x100
 
-EXPORTED_SYMBOLS = ["fmoe_expert_bytes", "fmoe_create", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
-                    "fmoe_stack_forward", "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy",
+EXPORTED_SYMBOLS = ["fmoe_expert_bytes", "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward",
+                    "fmoe_layer_forward", "fmoe_stack_forward", "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy",
                     "fmoe_last_error"]
 
 
@@ -71,6 +71,7 @@ def lib():
             L.fmoe_expert_bytes.restype = ctypes.c_size_t
             L.fmoe_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerDesc), P, ctypes.POINTER(P)]
             L.fmoe_route.argtypes = [P, i32, P, i32, P, P, P]
+            L.fmoe_route_static.argtypes = [P, i32, P, i32, P, P, P]
             L.fmoe_expert_forward.argtypes = [P, i32, i32, P, i32, P, P]
             L.fmoe_layer_forward.argtypes = [P, i32, P, i32, P, P, P, P]
             L.fmoe_stack_forward.argtypes = [P, i32, i32, P, i32, P, P]
@@ -117,6 +118,11 @@ def fmoe_create(cfg: Config, layers, stream: int = 0, *, check: bool = True):
 
 def fmoe_route(ctx, layer, x_dev, T, idx_dev, w_dev, stream=0, *, check=True) -> int:
     st = lib().fmoe_route(_vp(ctx), layer, _vp(x_dev), T, _vp(idx_dev), _vp(w_dev), _vp(stream))
+    return _check(ctx, st) if check else st
+
+
+def fmoe_route_static(ctx, layer, x_dev, T, idx_dev, w_dev, stream=0, *, check=True) -> int:
+    st = lib().fmoe_route_static(_vp(ctx), layer, _vp(x_dev), T, _vp(idx_dev), _vp(w_dev), _vp(stream))
     return _check(ctx, st) if check else st
 
 

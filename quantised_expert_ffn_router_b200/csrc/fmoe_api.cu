@@ -445,6 +445,31 @@ fmoe_status fmoe_route(fmoe_ctx* ctx, int32_t layer, const void* x_dev, int32_t 
   return FMOE_OK;
 }
 
+fmoe_status fmoe_route_static(fmoe_ctx* ctx, int32_t layer, const void* x_dev, int32_t T, int32_t* idx_dev,
+                              float* w_dev, void* stream) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  fmoe_status s = check_ctx_layer(ctx, layer, T);
+  if (s != FMOE_OK) return s;
+  if (T == 0) return FMOE_OK;
+  if (!x_dev || !idx_dev || !w_dev) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL tensor");
+  if (misaligned(x_dev) || misaligned(idx_dev) || misaligned(w_dev))
+    return fail(ctx, FMOE_ERR_ALIGNMENT, "tensor not 16-byte aligned");
+  const fmoe_config& c = ctx->cfg;
+  if ((int64_t)T * c.n_experts > kStaticRouteLogits || T > kStaticRouteMaxTokens)
+    return fail(ctx, FMOE_ERR_UNSUPPORTED, "T=%d x E=%d exceeds the fixed scratch (%d logits, %d tokens)", T,
+                c.n_experts, kStaticRouteLogits, kStaticRouteMaxTokens);
+  const fmoe_layer_desc& L = ctx->layers[layer];
+  const int rc = launch_route_static(static_cast<const uint16_t*>(L.router_w_dev), L.router_bias_dev,
+                                     static_cast<const uint16_t*>(L.norm_w_dev), c.rms_eps,
+                                     static_cast<const uint16_t*>(x_dev), T, c.hidden, c.n_experts, c.top_k, idx_dev,
+                                     w_dev, stream);
+  if (rc != 0) {
+    cudaGetLastError();
+    return cuda_fail(ctx, (cudaError_t)rc, "static route launch");
+  }
+  return FMOE_OK;
+}
+
 fmoe_status fmoe_expert_forward(fmoe_ctx* ctx, int32_t layer, int32_t expert, const void* x_dev, int32_t T,
                                 float* y_dev, void* stream) {
   if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");

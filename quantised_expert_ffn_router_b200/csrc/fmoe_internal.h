@@ -39,6 +39,9 @@ constexpr int kConsumerWarps = 16;       // warps that compute
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kChunkTiles = 16;          // tiles per gate/up or down task
 constexpr int kMaxTasks = 96;            // task-list capacity per block (multiple of 32)
+constexpr int kStaticRouteLogits = 32768; // fp32 logits in the fixed scratch of fmoe_route_static (128 KB)
+constexpr int kStaticRouteMaxTokens = 4096;  // tokens per fmoe_route_static call
+constexpr int kMaxDevices = 64;          // devices fmoe_route_static caches a scratch address for
 constexpr int kRouteFirst = 1;          // see DecodePlan::route_first
 constexpr int kFetchGroups = 8;          // activation groups a warp fetches per round trip
 
@@ -179,6 +182,10 @@ int build_task_list(const DecodePlan& P, int cta, uint32_t* out);
 int launch_repack(const uint8_t* src, uint8_t* dst, int n_experts, int H, int I, int bits, int to_packed,
                   void* stream);
 int launch_decode(const DecodePlan& plan, void* stream, bool cooperative, bool pdl);
+// Router step with its scratch in a fixed device array (fmoe_static.cu); returns
+// a cudaError_t value.
+int launch_route_static(const uint16_t* wr, const float* bias, const uint16_t* norm_w, float eps,
+                        const uint16_t* x, int T, int H, int E, int K, int32_t* idx_out, float* w_out, void* stream);
 int decode_max_smem_optin(int device);
 int decode_occupancy(int bits, int smem_bytes, int* blocks_per_sm);
 int zero_workspace(void* ws, size_t bytes, void* stream);
