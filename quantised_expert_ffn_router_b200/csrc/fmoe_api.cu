@@ -125,14 +125,26 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
   const uint32_t r_y = region((uint32_t)(std::max(P.rb_per_cta, 1) * std::max(P.n_slots, 1) * 16 * 4));
   const uint32_t r_tasks = region((uint32_t)kMaxTasks * 4);
   const uint32_t r_misc = region((uint32_t)sizeof(Misc));
-  // ring: as many stages as fit (<= 64, <= tasks), each stage_bytes
-  int nstage = 0;
-  for (int ns = std::min(64, std::max(max_tasks, 1)); ns >= 1; --ns) {
-    uint32_t total = align_up((uint32_t)ns * P.stage_bytes, 128) + fixed + align_up((uint32_t)(2 * ns * 8), 128);
-    if ((int)total <= max_smem) {
-      nstage = ns;
-      break;
+  // Down jobs get a stage each after the ring when that leaves the ring at
+  // least kMinRingStages stages (else they share the ring, streamed last).  A
+  // ring stage turns over in about one loaded HBM round trip plus one task's
+  // processing (~1.5 + ~1.7 us), so keeping HBM busy takes ~20 stages of
+  // 9 KB per SM; a shallower ring loses more than early down weights gain.
+  // The ring takes as many stages as still fit (<= 64 in all, <= its tasks).
+  auto fit_ring = [&](int n_down) {
+    const int ring_tasks = std::max(max_tasks - n_down, 1);
+    for (int ns = std::min(64 - n_down, ring_tasks); ns >= 1; --ns) {
+      const int all = ns + n_down;
+      uint32_t total = align_up((uint32_t)all * P.stage_bytes, 128) + fixed + align_up((uint32_t)(2 * all * 8), 128);
+      if ((int)total <= max_smem) return ns;
     }
+    return 0;
+  };
+  P.n_down_max = P.n_slots > 0 ? P.rb_per_cta * P.n_slots * P.dn_chunks : 0;
+  int nstage = P.n_down_max > 0 && P.n_down_max <= 32 ? fit_ring(P.n_down_max) : 0;
+  if (nstage < std::min(kMinRingStages, std::max(max_tasks - P.n_down_max, 1))) {
+    P.n_down_max = 0;
+    nstage = fit_ring(0);
   }
   if (nstage < 1) return false;
   // several issuing lanes (one copy instruction in flight per lane); keep the
@@ -153,7 +165,7 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
   P.nstage = nstage;
   P.route_first = kRouteFirst;
   P.off_ring = off;
-  off = align_up((uint32_t)nstage * P.stage_bytes, 128);
+  off = align_up((uint32_t)(nstage + P.n_down_max) * P.stage_bytes, 128);
   P.off_z = off + r_z;
   P.off_lg = off + r_lg;
   P.off_zfrag = off + r_zfrag;
@@ -167,7 +179,7 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
   P.off_misc = off + r_misc;
   off += fixed;
   P.off_bar = off;
-  off = align_up(off + (uint32_t)(2 * nstage * 8), 128);
+  off = align_up(off + (uint32_t)(2 * (nstage + P.n_down_max) * 8), 128);
   P.smem_bytes = off;
   return (int)P.smem_bytes <= max_smem;
 }

@@ -369,7 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   volatile int* abort_flag = &misc->abort;
   uint32_t* tasks = reinterpret_cast<uint32_t*>(smem + P.off_tasks);
   const uint32_t bar_full = smem_u32(smem + P.off_bar);
-  const uint32_t bar_empty = bar_full + 8u * P.nstage;
+  const int n_stages_all = P.nstage + P.n_down_max;
+  const uint32_t bar_empty = bar_full + 8u * n_stages_all;
   uint16_t* zs = reinterpret_cast<uint16_t*>(smem + P.off_z);
   uint32_t* zfrag = reinterpret_cast<uint32_t*>(smem + P.off_zfrag);
   float2* zinfo = reinterpret_cast<float2*>(smem + P.off_zinfo);
@@ -382,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int first_rb = G - 1 - cta;
   const int my_rb = (P.n_slots > 0 && first_rb < P.n_rb) ? (P.n_rb - first_rb + G - 1) / G : 0;
   const bool has_router = P.mode != kModeExpert;
+  const int n_down = P.n_down_max > 0 ? my_rb * P.n_slots * P.dn_chunks : 0;
   float h_res = 0.f;  // residual input of the row this thread combines
 
   // ---------------------------------------------------------------- set-up
@@ -390,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   // without reading it): weights do not depend on the previous launch.
   int pre_issued = 0;
   if (warp == kConsumerWarps) {
-    for (int i = lane; i < 2 * P.nstage; i += 32) mbar_init(bar_full + 8u * i, 1);
+    for (int i = lane; i < 2 * n_stages_all; i += 32) mbar_init(bar_full + 8u * i, 1);
     misc->last_task[lane] = -1;
     misc->last_task[lane + 32] = -1;
     asm volatile("fence.mbarrier_init.release.cluster;\n fence.proxy.async.shared::cta;" ::: "memory");
@@ -441,8 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       if (P.pdl && !waited_grid) asm volatile("griddepcontrol.wait;" ::: "memory");
       waited_grid = true;
       // Poll the tagged logits until every router row of this launch is
-      // published; each lane keeps experts lane, lane+32, ... in registers
-      // (up to 512 experts; beyond that the values are staged in shared memory).
+      // published; each round a lane reads experts lane, lane+32, ... (16 loads
+      // issued back to back) and stages them in shared memory for top-K.
       const uint32_t tag = *reinterpret_cast<volatile uint32_t*>(&P.ws->epoch) + 1u;
       constexpr int kPollE = 16;  // logits per lane per load round
       float* lg = reinterpret_cast<float*>(smem + P.off_lg);
@@ -454,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #pragma unroll
           for (int k = 0; k < kPollE; ++k) {
             const int i = base + k * 32 + lane;
-            v[k] = i < P.E ? ld_tagged(P.ws_logits + i) : 0ull;
+            v[k] = ld_tagged(P.ws_logits + min(i, P.E - 1));  // past the end: ignored below
           }
 #pragma unroll
           for (int k = 0; k < kPollE; ++k) {
@@ -503,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const int NI = P.n_issuers;
     auto issue = [&](int i, uint32_t t) -> int {
       int s, fill;
-      task_stage(P.nstage, NI, i, s, fill);
+      task_stage_of(P.nstage, NI, n_tasks, n_down, i, s, fill);
       if (fill > 0 && !wait_mbar(bar_empty + 8u * s, (uint32_t)((fill - 1) & 1), limit, abort_flag)) {
         if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutTma);
         *abort_flag = 1;
@@ -535,10 +537,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       reinterpret_cast<volatile int*>(misc->last_task)[s] = i;
       return 1;
     };
-    for (int r = 0; r * NI < n_tasks; ++r) {
+    // Down jobs with stages of their own (the block's last n_down tasks) are all
+    // issued as soon as their experts are known, ahead of the gate/up stream:
+    // their weights land early and nothing streams any more when the
+    // activations are exchanged.
+    const int ring_end = n_tasks - n_down;
+    bool downs_issued = n_down == 0;
+    auto issue_downs = [&]() -> bool {
+      for (int r = 0; ring_end + r * NI < n_tasks; ++r) {
+        const int i = ring_end + r * NI + lane;
+        const int ok = (lane < NI && i < n_tasks) ? issue(i, tasks[i]) : 1;
+        if (!__all_sync(0xffffffffu, ok)) return false;
+      }
+      downs_issued = true;
+      return true;
+    };
+    bool failed = P.mode == kModeExpert && !downs_issued && !issue_downs();
+    for (int r = 0; r * NI < ring_end && !failed; ++r) {
       if (__any_sync(0xffffffffu, *abort_flag)) break;
       const int i = r * NI + lane;
-      const bool mine = lane < NI && i < n_tasks && i >= pre_issued;
+      const bool mine = lane < NI && i < ring_end && i >= pre_issued;
       const uint32_t t = mine ? tasks[i] : 0u;
       const bool needs_route = mine && P.mode == kModeLayer && !routed && task_type(t) != kTaskRouter &&
                                (task_slot(t) >= 1 || P.route_first);
@@ -548,9 +566,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       if (__any_sync(0xffffffffu, needs_route)) {
         if (!do_routing()) break;
         routed = true;
+        if (!downs_issued && !issue_downs()) break;
         if (needs_route) ok = issue(i, t);
         if (!__all_sync(0xffffffffu, ok)) break;
       }
+    }
+    // a block whose own list needed no routing still owes its down jobs
+    if (!downs_issued && !__any_sync(0xffffffffu, *abort_flag)) {
+      if (P.mode == kModeLayer && !routed) routed = do_routing();
+      if (routed || P.mode != kModeLayer) issue_downs();
     }
     // routing still owed for the output indices
     if (!__any_sync(0xffffffffu, *abort_flag) && !routed && has_router && cta == 0 && (P.idx_out || P.w_out))
@@ -625,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // ---- task loop: warp w takes tasks w, w+16, ...
     for (int i = warp; i < n_tasks; i += kConsumerWarps) {
       int s, fill;
-      task_stage(P.nstage, P.n_issuers, i, s, fill);
+      task_stage_of(P.nstage, P.n_issuers, n_tasks, n_down, i, s, fill);
       // A stage's fills are consumed by different warps, so first make sure
       // task i is the stage's current fill (all earlier fills consumed); only
       // then is the parity wait unambiguous.  Every lane observes the phase,
@@ -732,12 +756,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           for (int g0 = 0; g0 < ng && good; g0 += kFetchGroups) {
             ulonglong2 v[kFetchGroups];
             for (int attempt = 0;; ++attempt) {
+              // every load is issued before any result is examined: the loads
+              // are volatile, so a check between two of them would wait for
+              // the first one's round trip before issuing the second
+#pragma unroll
+              for (int k = 0; k < kFetchGroups; ++k)  // past the end: re-read the last group, ignored below
+                v[k] = ld_tagged2(act + min(g0 + k, ng - 1) * kGroup + 2 * lane);
               bool mine = true;
 #pragma unroll
-              for (int k = 0; k < kFetchGroups; ++k) {
-                v[k] = (g0 + k < ng) ? ld_tagged2(act + (g0 + k) * kGroup + 2 * lane) : make_ulonglong2(0ull, 0ull);
+              for (int k = 0; k < kFetchGroups; ++k)
                 if (g0 + k < ng) mine = mine && tagged_tag(v[k].x) == tag && tagged_tag(v[k].y) == tag;
-              }
               if (__all_sync(0xffffffffu, mine)) break;
               // not all published yet: wait for the count, then fetch again
               const bool counted =
@@ -829,11 +857,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   if (tid == kConsumerWarps * 32) {
     // After an abort the latest copy into every stage must land before the
     // block exits (without one, every issued copy was consumed already).
-    for (int s = 0; s < P.nstage && aborted; ++s) {
+    for (int s = 0; s < n_stages_all && aborted; ++s) {
       const int i = misc->last_task[s];
       if (i < 0) continue;
       int s2, fill;
-      task_stage(P.nstage, P.n_issuers, i, s2, fill);
+      task_stage_of(P.nstage, P.n_issuers, n_tasks, n_down, i, s2, fill);
       const uint64_t t0 = gtimer();
       while (!mbar_try_wait(bar_full + 8u * s, (uint32_t)(fill & 1)))
         if (gtimer() - t0 > limit) {

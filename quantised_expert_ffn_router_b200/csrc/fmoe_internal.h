@@ -42,6 +42,7 @@ constexpr int kMaxTasks = 96;            // task-list capacity per block (multip
 constexpr int kStaticRouteLogits = 32768; // fp32 logits in the fixed scratch of fmoe_route_static (128 KB)
 constexpr int kStaticRouteMaxTokens = 4096;  // tokens per fmoe_route_static call
 constexpr int kMaxDevices = 64;          // devices fmoe_route_static caches a scratch address for
+constexpr int kMinRingStages = 20;       // ring stages kept when down jobs get stages of their own
 constexpr int kRouteFirst = 1;          // see DecodePlan::route_first
 constexpr int kFetchGroups = 8;          // activation groups a warp fetches per round trip
 
@@ -126,7 +127,8 @@ struct DecodePlan {
   int router_rows;         // max router rows per block
   int router_parts;        // column parts per router row (one task each)
   int router_part_cols;    // columns per part (multiple of 64; the last part may be shorter)
-  int nstage;              // ring stages (a multiple of n_issuers)
+  int nstage;              // ring stages for router and gate/up tasks (a multiple of n_issuers)
+  int n_down_max;          // stages after the ring, one per down job (filled once per launch)
   int n_issuers;           // producer lanes issuing copies; lane l owns stages l, l+n_issuers, ...
   int route_first;         // 1: route before issuing any expert copy (keeps the logit exchange off a busy memory pipe)
   uint32_t stage_bytes;
@@ -173,6 +175,20 @@ inline __host__ __device__ void task_stage(int nstage, int n_issuers, int i, int
   const int L = nstage / n_issuers, j = i / n_issuers;
   stage = (j % L) * n_issuers + i % n_issuers;
   fill = j / L;
+}
+
+// Stage and fill of task i of a block whose last n_down tasks are its down
+// jobs: those sit in dedicated stages after the ring (one fill each), the other
+// tasks cycle through the ring.
+inline __host__ __device__ void task_stage_of(int nstage, int n_issuers, int n_tasks, int n_down, int i, int& stage,
+                                              int& fill) {
+  const int ring_end = n_tasks - n_down;
+  if (i >= ring_end) {
+    stage = nstage + (i - ring_end);
+    fill = 0;
+  } else {
+    task_stage(nstage, n_issuers, i, stage, fill);
+  }
 }
 
 // Host-side construction of a block's ordered task list; returns its length.
