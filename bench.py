@@ -204,9 +204,12 @@ def metric_name(wl):
 
 
 def config_dict(wl, flushed, cpu=False):
+    batched = wl.name == "batched"
     return {"workload": wl.name,
             "shape": f"H{wl.hidden} E{wl.n_experts} top{wl.top_k}+1shared I{wl.inter} {wl.bits}-bit g64",
-            "layers": wl.n_layers, "tokens": wl.tokens, "batch": 1, "norm": wl.norm,
+            "layers": wl.n_layers, "tokens": wl.tokens * (wl.steps if batched else 1),
+            "batch": wl.tokens if batched else 1, "norm": wl.norm,
+            **({"router_bias": f"Zipf(s={wl.zipf}) over a seeded expert ranking"} if wl.zipf else {}),
             "l2": "n/a (CPU oracle)" if cpu else ("flushed (256 MB write) before every timed step" if flushed else
                                                   "per-step weight traffic far above L2 (no flush)"),
             "parallelism": "replicas"}
@@ -260,23 +263,28 @@ def run_gpu(args, wl, ws, rank, local):
     sp = stream.cuda_stream
     weights = DeviceWeights(wl)
     descs = [fm.LayerDesc(**d) for d in weights.descs()]
-    cfg = fm.Config(wl.hidden, wl.n_experts, wl.top_k, wl.inter, wl.bits, 64, wl.n_layers, 1, wl.rms_eps, 0, 0)
+    batched = wl.name == "batched"
+    B = wl.tokens if batched else 1          # tokens per step
+    cfg = fm.Config(wl.hidden, wl.n_experts, wl.top_k, wl.inter, wl.bits, 64, wl.n_layers, B, wl.rms_eps, 0, 0)
     _, ctx = fm.fmoe_create(cfg, descs, sp)
-    n_tok = wl.tokens
-    X = tokens(wl, range(n_tok))
+    n_batches = wl.steps if batched else wl.tokens   # distinct inputs cycled through
+    X = tokens(wl, range(n_batches * B)).view(n_batches, B, wl.hidden)
     OUT = torch.empty_like(X)
+    IDX = torch.zeros((n_batches, B, wl.top_k), dtype=torch.int32, device="cuda")
     L = wl.n_layers
     stacked = L > 1
 
     def step(i, x_ptr=None, out_ptr=None):
-        x_ptr = X[i % n_tok].data_ptr() if x_ptr is None else x_ptr
-        out_ptr = OUT[i % n_tok].data_ptr() if out_ptr is None else out_ptr
+        x_ptr = X[i % n_batches].data_ptr() if x_ptr is None else x_ptr
+        out_ptr = OUT[i % n_batches].data_ptr() if out_ptr is None else out_ptr
         if stacked:
-            fm.fmoe_stack_forward(ctx, 0, L, x_ptr, 1, out_ptr, sp)
+            fm.fmoe_stack_forward(ctx, 0, L, x_ptr, B, out_ptr, sp)
         else:
-            fm.fmoe_layer_forward(ctx, 0, x_ptr, 1, out_ptr, None, None, sp)
+            fm.fmoe_layer_forward(ctx, 0, x_ptr, B, out_ptr, IDX[i % n_batches].data_ptr() if batched else None,
+                                  None, sp)
 
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if not stacked else None
+    # a batched step streams ~0.5 GB of expert weights, far above L2: no flush
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if not (stacked or batched) else None
 
     def maybe_flush(i):
         if flush is not None:
@@ -313,7 +321,7 @@ def run_gpu(args, wl, ws, rank, local):
 
     # warm (no flush) reference number for the single layer
     warm_us = None
-    if not stacked:
+    if not (stacked or batched):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for i in range(steps):
@@ -324,18 +332,18 @@ def run_gpu(args, wl, ws, rank, local):
 
     # end to end through the public API with host buffers (pinned), copies timed
     e2e_steps = min(steps, args.e2e_steps)
-    x_host = X[:n_tok].cpu().pin_memory()
+    x_host = X[:min(n_batches, e2e_steps)].cpu().pin_memory()
     out_host = torch.empty_like(x_host).pin_memory()
-    xd = torch.empty((1, wl.hidden), dtype=torch.bfloat16, device="cuda")
+    xd = torch.empty((B, wl.hidden), dtype=torch.bfloat16, device="cuda")
     od = torch.empty_like(xd)
     e2e_ms = []
     for i in range(e2e_steps):
         maybe_flush(i)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        xd.copy_(x_host[i % n_tok:i % n_tok + 1], non_blocking=True)
+        xd.copy_(x_host[i % len(x_host)], non_blocking=True)
         step(i, xd.data_ptr(), od.data_ptr())
-        out_host[i % n_tok:i % n_tok + 1].copy_(od, non_blocking=True)
+        out_host[i % len(x_host)].copy_(od, non_blocking=True)
         b.record(stream)
         stream.synchronize()
         e2e_ms.append(a.elapsed_time(b))
@@ -345,9 +353,19 @@ def run_gpu(args, wl, ws, rank, local):
     if rank != 0:
         return 0
     ms_per_step = total_ms / steps
-    tps = job_throughput(ws, steps, total_ms)
+    tps = job_throughput(ws, steps * B, total_ms)
     us_layer = 1e3 * ms_per_step / L
     bytes_launch = layer_bytes(wl)
+    tensor = None
+    if batched:
+        # per step: router + every distinct selected expert + the shared one, tokens in and out
+        idx_h = IDX.cpu().numpy()
+        uniq = [len(set(idx_h[i % n_batches].ravel().tolist())) for i in range(steps)]
+        bytes_launch = (wl.n_experts * wl.hidden * 2 + (statistics.mean(uniq) + 1) * wl.blob_bytes
+                        + 2 * B * wl.hidden * 2)
+        flops = 2 * B * (wl.top_k + 1) * 3 * wl.hidden * wl.inter + 2 * B * wl.hidden * wl.n_experts
+        tensor = {"flops_per_step": flops, "achieved_tflops": flops / (ms_per_step * 1e-3) / 1e12,
+                  "unique_experts_per_step": statistics.mean(uniq)}
     achieved = bytes_launch / (us_layer * 1e-6) / 1e9
     peak, peak_kind = hbm_peak()
     traffic = None
@@ -370,11 +388,13 @@ def run_gpu(args, wl, ws, rank, local):
                      "algorithmic_bytes_per_launch": bytes_launch},
         "step_us_p10_p50_p90": [1e3 * q for q in statistics.quantiles(step_ms, n=10)[0::4]] if steps >= 10 else None,
         "warm_l2_us_per_layer": warm_us,
-        "e2e": {"value": job_throughput(ws, e2e_steps, e2e_total), "unit": "tokens/s",
-                "h2d_bytes_per_step": wl.hidden * 2, "d2h_bytes_per_step": wl.hidden * 2},
-        "gpu_launches": steps * L,
+        "e2e": {"value": job_throughput(ws, e2e_steps * B, e2e_total), "unit": "tokens/s",
+                "h2d_bytes_per_step": B * wl.hidden * 2, "d2h_bytes_per_step": B * wl.hidden * 2},
+        "gpu_launches": steps * (9 if batched else L),
         "clocks": clocks,
     }
+    if tensor is not None:
+        line["batched"] = tensor
     if ws == 1 and not args.no_cpu_baseline:
         tps_cpu, done, threads, dt = oracle_tokens_per_s(wl, 400, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tps_cpu, "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -390,14 +410,14 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer", "stack4", "stack2", "tiny"], default="layer")
+    ap.add_argument("--workload", choices=["layer", "stack4", "stack2", "tiny", "batched"], default="layer")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     wl = synth.WORKLOADS[args.workload]
     if args.steps is None:
-        args.steps = {"layer": 3000, "stack4": 256, "stack2": 256, "tiny": 1000}[args.workload]
+        args.steps = {"layer": 3000, "stack4": 256, "stack2": 256, "tiny": 1000, "batched": 100}[args.workload]
     args.warmup = max(args.warmup, 3)
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -29,6 +29,8 @@ struct fmoe_ctx {
   uint32_t* tasks = nullptr;   // device [3 modes][grid][kMaxTasks]
   int32_t* ntasks = nullptr;   // device [3 modes][grid]
   uint16_t* stack_buf[2] = {nullptr, nullptr};  // ping-pong activations, [max_tokens][H] bf16
+  void* bws_mem = nullptr;  // batched-path workspace (max_tokens > 1)
+  BatchWs bws{};
   DecodePlan plan[3];  // per mode: layer, expert, route (pointers filled per call)
   std::string err;
 };
@@ -309,7 +311,7 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   if (c.max_tokens < 0) return fail(nullptr, FMOE_ERR_INVALID_ARG, "max_tokens=%d", c.max_tokens);
   if (!(c.rms_eps >= 0.f)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "rms_eps must be >= 0");
   if (c.top_k > kMaxTopK) return fail(nullptr, FMOE_ERR_UNSUPPORTED, "top_k=%d above %d", c.top_k, kMaxTopK);
-  if (c.hidden > 4096 || c.inter > 4096)
+  if (c.hidden > kMaxHidden || c.inter > 4096)
     return fail(nullptr, FMOE_ERR_UNSUPPORTED, "hidden=%d / inter=%d above 4096", c.hidden, c.inter);
   if (c.n_experts > 65536) return fail(nullptr, FMOE_ERR_UNSUPPORTED, "n_experts=%d above 65536", c.n_experts);
   for (int l = 0; l < c.n_layers; ++l) {
@@ -327,6 +329,7 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   auto bail = [&](fmoe_status st) {
     g_create_err = ctx->err;
     if (ctx->ws) cudaFree(ctx->ws);
+    if (ctx->bws_mem) cudaFree(ctx->bws_mem);
     delete ctx;
     return st;
   };
@@ -374,6 +377,18 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   ctx->ntasks = reinterpret_cast<int32_t*>(base + off_ntasks);
   ctx->stack_buf[0] = reinterpret_cast<uint16_t*>(base + off_stack);
   ctx->stack_buf[1] = reinterpret_cast<uint16_t*>(base + off_stack + stack_bytes);
+  // batched path: sized for max_tokens, only when more than one token is allowed
+  if (c.max_tokens > 1 || (c.flags & FMOE_FLAG_FORCE_GROUPED)) {
+    const size_t bb = batch_ws_bytes(c.hidden, c.n_experts, c.top_k, c.inter, std::max(c.max_tokens, 1));
+    e = cudaMalloc(&ctx->bws_mem, bb);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      ctx->bws_mem = nullptr;
+      return bail(fail(ctx, FMOE_ERR_OOM, "batched workspace allocation of %zu bytes failed", bb));
+    }
+    batch_ws_carve(static_cast<uint8_t*>(ctx->bws_mem), c.hidden, c.n_experts, c.top_k, c.inter,
+                   std::max(c.max_tokens, 1), ctx->bws);
+  }
   cudaStream_t st = (cudaStream_t)stream;
   e = cudaMemsetAsync(ctx->ws, 0, ctx->ws_bytes, st);
   if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "workspace clear"));
@@ -432,7 +447,46 @@ fmoe_status fmoe_destroy(fmoe_ctx* ctx) {
     }
   }
   if (ctx->ws) cudaFree(ctx->ws);
+  if (ctx->bws_mem) cudaFree(ctx->bws_mem);
   delete ctx;
+  return FMOE_OK;
+}
+
+// The batched path takes T >= kGroupedMinTokens tokens (any T with
+// FORCE_GROUPED) unless FORCE_PER_TOKEN asks for one batch-1 launch per token.
+static bool use_batched(const fmoe_ctx* ctx, int32_t T) {
+  if (ctx->bws_mem == nullptr) return false;
+  if (ctx->cfg.flags & FMOE_FLAG_FORCE_GROUPED) return true;
+  if (ctx->cfg.flags & FMOE_FLAG_FORCE_PER_TOKEN) return false;
+  return T >= kGroupedMinTokens;
+}
+
+static BatchArgs batch_args(const fmoe_ctx* ctx, int32_t layer, int32_t T) {
+  const fmoe_config& c = ctx->cfg;
+  const fmoe_layer_desc& L = ctx->layers[layer];
+  BatchArgs a{};
+  a.H = c.hidden;
+  a.E = c.n_experts;
+  a.K = c.top_k;
+  a.I = c.inter;
+  a.bits = c.bits;
+  a.T = T;
+  a.experts = static_cast<const uint8_t*>(L.experts_dev);
+  a.blob_bytes = expert_bytes(c.hidden, c.inter, c.bits);
+  a.router_w = static_cast<const uint16_t*>(L.router_w_dev);
+  a.router_bias = L.router_bias_dev;
+  a.norm_w = static_cast<const uint16_t*>(L.norm_w_dev);
+  a.eps = c.rms_eps;
+  a.single_expert = -1;
+  return a;
+}
+
+static fmoe_status run_batched(fmoe_ctx* ctx, const BatchArgs& a, void* stream) {
+  const int rc = launch_batched(a, ctx->bws, ctx->n_sm, stream);
+  if (rc != 0) {
+    cudaGetLastError();
+    return cuda_fail(ctx, (cudaError_t)rc, "batched launch");
+  }
   return FMOE_OK;
 }
 
@@ -492,6 +546,13 @@ fmoe_status fmoe_expert_forward(fmoe_ctx* ctx, int32_t layer, int32_t expert, co
   if (T == 0) return FMOE_OK;
   if (!x_dev || !y_dev) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL tensor");
   if (misaligned(x_dev) || misaligned(y_dev)) return fail(ctx, FMOE_ERR_ALIGNMENT, "tensor not 16-byte aligned");
+  if (use_batched(ctx, T)) {
+    BatchArgs a = batch_args(ctx, layer, T);
+    a.h_in = static_cast<const uint16_t*>(x_dev);
+    a.single_expert = expert < 0 ? ctx->cfg.n_experts : expert;
+    a.y_out = y_dev;
+    return run_batched(ctx, a, stream);
+  }
   const int H = ctx->cfg.hidden;
   for (int t = 0; t < T; ++t) {
     DecodePlan P = bind(ctx, kModeExpert, layer);
@@ -506,6 +567,14 @@ fmoe_status fmoe_expert_forward(fmoe_ctx* ctx, int32_t layer, int32_t expert, co
 
 static fmoe_status layer_tokens(fmoe_ctx* ctx, int32_t layer, const uint16_t* h_in, int32_t T, uint16_t* h_out,
                                 int32_t* idx, float* w, void* stream) {
+  if (use_batched(ctx, T)) {
+    BatchArgs a = batch_args(ctx, layer, T);
+    a.h_in = h_in;
+    a.h_out = h_out;
+    a.idx_out = idx;
+    a.w_out = w;
+    return run_batched(ctx, a, stream);
+  }
   const int H = ctx->cfg.hidden, K = ctx->cfg.top_k;
   for (int t = 0; t < T; ++t) {
     DecodePlan P = bind(ctx, kModeLayer, layer);

@@ -83,8 +83,9 @@ __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
 }
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  // not volatile: the result is the only effect, so independent tiles' chains
+  // may be interleaved by the compiler
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -589,41 +590,59 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       h_res = bf16f(P.h_in[(first_rb + (tid / 16) * G) * 16 + tid % 16]);
     // ---- input: z = RMSNorm(h_in) or h_in (bf16, shared memory) and its fragments
     {
-      const int c0 = tid * 8;
-      uint4 hv = make_uint4(0u, 0u, 0u, 0u);
-      if (c0 < P.H) hv = *reinterpret_cast<const uint4*>(P.h_in + c0);
+      // thread tid holds columns 8*(tid + j*threads) .. +7, j < kPrepChunks
+      constexpr int kCT = kConsumerWarps * 32;
+      constexpr int kPrepChunks = (kMaxHidden + 8 * kCT - 1) / (8 * kCT);
+      uint4 hv[kPrepChunks];
+#pragma unroll
+      for (int j = 0; j < kPrepChunks; ++j) {
+        const int c0 = (tid + j * kCT) * 8;
+        hv[j] = c0 < P.H ? *reinterpret_cast<const uint4*>(P.h_in + c0) : make_uint4(0u, 0u, 0u, 0u);
+      }
       if (P.norm_w != nullptr) {
-        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
         float ss = 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          ss = fmaf(bf16lo(hw[k]), bf16lo(hw[k]), ss);
-          ss = fmaf(bf16hi(hw[k]), bf16hi(hw[k]), ss);
+        for (int j = 0; j < kPrepChunks; ++j) {
+          const uint32_t hw[4] = {hv[j].x, hv[j].y, hv[j].z, hv[j].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            ss = fmaf(bf16lo(hw[k]), bf16lo(hw[k]), ss);
+            ss = fmaf(bf16hi(hw[k]), bf16hi(hw[k]), ss);
+          }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         if (lane == 0) misc->red[warp] = ss;
-        asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
+        asm volatile("bar.sync 1, %0;" ::"r"(kCT) : "memory");
         float tot = 0.f;
         for (int w = 0; w < kConsumerWarps; ++w) tot += misc->red[w];
         const float r = 1.0f / sqrtf(tot / (float)P.H + P.eps);
-        if (c0 < P.H) {
-          const uint4 wv = *reinterpret_cast<const uint4*>(P.norm_w + c0);
-          const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-          uint32_t zz[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t lo = f2bf16(bf16lo(hw[k]) * r * bf16lo(ww[k]));
-            const uint32_t hi = f2bf16(bf16hi(hw[k]) * r * bf16hi(ww[k]));
-            zz[k] = lo | (hi << 16);
+        for (int j = 0; j < kPrepChunks; ++j) {
+          const int c0 = (tid + j * kCT) * 8;
+          if (c0 < P.H) {
+            const uint4 wv = *reinterpret_cast<const uint4*>(P.norm_w + c0);
+            const uint32_t hw[4] = {hv[j].x, hv[j].y, hv[j].z, hv[j].w};
+            const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+            uint32_t zz[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t lo = f2bf16(bf16lo(hw[k]) * r * bf16lo(ww[k]));
+              const uint32_t hi = f2bf16(bf16hi(hw[k]) * r * bf16hi(ww[k]));
+              zz[k] = lo | (hi << 16);
+            }
+            hv[j] = make_uint4(zz[0], zz[1], zz[2], zz[3]);
           }
-          hv = make_uint4(zz[0], zz[1], zz[2], zz[3]);
         }
       }
-      if (c0 < P.H) *reinterpret_cast<uint4*>(zs + c0) = hv;
-      asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
+#pragma unroll
+      for (int j = 0; j < kPrepChunks; ++j) {
+        const int c0 = (tid + j * kCT) * 8;
+        if (c0 < P.H) *reinterpret_cast<uint4*>(zs + c0) = hv[j];
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(kCT) : "memory");
       if (P.n_slots > 0) {
-        // warp w builds groups 4w..4w+3, then 4(w+16).., so a batch is contiguous
+        // warp w builds groups 4w..4w+3, then 4(w+W).., so a batch is contiguous
         const int ngz = P.H / kGroup;
         for (int G0 = 4 * warp; G0 < ngz; G0 += 4 * kConsumerWarps) {
           float lo[4], hi[4];

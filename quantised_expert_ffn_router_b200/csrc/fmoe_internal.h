@@ -35,7 +35,8 @@ namespace fmoe {
 constexpr int kGroup = 64;
 constexpr int kMaxTopK = 8;
 constexpr int kMaxSlots = kMaxTopK + 1;  // K routed + 1 shared
-constexpr int kConsumerWarps = 16;       // warps that compute
+constexpr int kConsumerWarps = 15;       // warps that compute (16 warps in all: 4 per SM sub-partition, 128 registers each)
+constexpr int kMaxHidden = 4096;         // largest hidden size a context accepts
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kChunkTiles = 16;          // tiles per gate/up or down task
 constexpr int kMaxTasks = 96;            // task-list capacity per block (multiple of 32)
@@ -190,6 +191,61 @@ inline __host__ __device__ void task_stage_of(int nstage, int n_issuers, int n_t
     task_stage(nstage, n_issuers, i, stage, fill);
   }
 }
+
+// ---------------------------------------------------------------- batched path
+// T tokens at once (fmoe_batched.cu): RMSNorm, router GEMM, top-K, a stable
+// per-expert permutation of the T*(K+1) (token, slot) pairs into segments, a
+// grouped gate/up GEMM (128 rows x 64 tokens per work item, codes exact on the
+// tensor pipe, per-group scale/bias epilogue, silu(g)*u in the epilogue), a
+// grouped down GEMM, and a fixed-order combine.  Positions 0..T*K-1 hold the
+// routed pairs grouped by expert; positions T*K.. hold the shared expert.
+constexpr int kGemmRows = 128;       // rows per work item (8 warps x 16)
+constexpr int kGemmTokens = 64;      // tokens (positions) per work item
+constexpr int kGroupedMinTokens = 8; // fmoe_layer_forward uses the batched path from this T on
+
+struct BatchWs {              // device buffers, sized for max_tokens at create
+  uint16_t* z;                // bf16 [T][H]   (normalised input)
+  uint8_t* zf;                // [T][H/64] records: 64 scaled fp16 values, (2^-scale, group sum), pad
+  float* logits;              // [T][E]
+  float* logit_part;          // [4][T][E] partial router logits (K split)
+  int32_t* idx;               // [T][K]
+  float* w;                   // [T][K]
+  int32_t* seg;               // [4][E+1]: expert, start, count, items-prefix per segment; [4*(E+1)] = n_seg
+  int32_t* cursor;            // [E+1] scatter cursors
+  int32_t* pos_tok;           // [T*(K+1)] token of each position
+  int32_t* pos_of;            // [T][K+1] position of (token, slot); slot K = shared
+  uint32_t* items_gu;         // work items (seg, row block, token block)
+  uint32_t* items_dn;
+  int32_t* n_items;           // [2]
+  float* a;                   // [T*(K+1)][I] activations
+  uint8_t* af;                // [T*(K+1)][I/64] records, as zf
+  float* y;                   // [T*(K+1)][H] expert outputs
+  int max_items_gu, max_items_dn;
+};
+
+struct BatchArgs {
+  int H, E, K, I, bits, T;
+  const uint8_t* experts;     // packed experts of the layer (E routed + shared)
+  int64_t blob_bytes;
+  const uint16_t* router_w;
+  const float* router_bias;
+  const uint16_t* norm_w;
+  float eps;
+  const uint16_t* h_in;       // [T][H]
+  uint16_t* h_out;            // [T][H]
+  int32_t* idx_out;           // [T][K] or null
+  float* w_out;               // [T][K] or null
+  int single_expert;          // >= 0: expert mode on this expert (0..E, E = shared), output y_out
+  float* y_out;               // [T][H] fp32 (expert mode)
+};
+
+// Bytes of the batched workspace for T tokens; carves it out of `base`.
+size_t batch_ws_bytes(int H, int E, int K, int I, int T);
+void batch_ws_carve(uint8_t* base, int H, int E, int K, int I, int T, BatchWs& ws);
+int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream);
+
+// Top-K and renormalised weights of T rows of fp32 logits (one warp per row).
+int launch_topk_rows(const float* logits, int T, int E, int K, int32_t* idx_out, float* w_out, void* stream);
 
 // Host-side construction of a block's ordered task list; returns its length.
 int build_task_list(const DecodePlan& P, int cta, uint32_t* out);

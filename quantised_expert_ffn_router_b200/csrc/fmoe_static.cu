@@ -152,6 +152,12 @@ float* g_symbol_addr[kMaxDevices] = {};
 
 }  // namespace
 
+int launch_topk_rows(const float* logits, int T, int E, int K, int32_t* idx_out, float* w_out, void* stream) {
+  static_topk_kernel<<<(T + kWarps - 1) / kWarps, kWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(logits, T, E, K,
+                                                                                                  idx_out, w_out);
+  return (int)cudaGetLastError();
+}
+
 int launch_route_static(const uint16_t* wr, const float* bias, const uint16_t* norm_w, float eps,
                         const uint16_t* x, int T, int H, int E, int K, int32_t* idx_out, float* w_out, void* stream) {
   int dev = 0;
