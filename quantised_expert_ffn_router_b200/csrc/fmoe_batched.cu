@@ -30,7 +30,6 @@ namespace {
 
 __device__ __forceinline__ float bflo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bfhi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-__device__ __forceinline__ float bf(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
 __device__ __forceinline__ uint16_t to_bf16(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
 __device__ __forceinline__ float pow2(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -57,13 +56,9 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// 16-byte (or 8-byte) async copy global -> shared; src_bytes 0 fills zeros.
+// 16-byte async copy global -> shared; src_bytes 0 fills zeros.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async8(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -245,24 +240,76 @@ struct PermuteArgs {
   int max_items_gu, max_items_dn;
 };
 
-// One block.  Counts per expert, exclusive scan, scatter of the T*K routed
-// pairs (positions within an expert follow atomics, so their order varies,
-// but every position is computed independently: the results do not depend on
-// it), the shared expert's segment after them, and the GEMM work items of every
-// non-empty segment in expert order.
+// Block-wide exclusive scan of three counters per thread (blockDim 1024);
+// returns the prefixes and writes the totals to tot[0..2].
+__device__ __forceinline__ int3 block_scan3(int3 v, int32_t* scratch, int32_t* tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int3 inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, inc.x, o), y = __shfl_up_sync(0xffffffffu, inc.y, o),
+              z = __shfl_up_sync(0xffffffffu, inc.z, o);
+    if (lane >= o) {
+      inc.x += x;
+      inc.y += y;
+      inc.z += z;
+    }
+  }
+  if (lane == 31) {
+    scratch[3 * warp] = inc.x;
+    scratch[3 * warp + 1] = inc.y;
+    scratch[3 * warp + 2] = inc.z;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int3 w = lane < nw ? make_int3(scratch[3 * lane], scratch[3 * lane + 1], scratch[3 * lane + 2]) : make_int3(0, 0, 0);
+    int3 wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, wi.x, o), y = __shfl_up_sync(0xffffffffu, wi.y, o),
+                z = __shfl_up_sync(0xffffffffu, wi.z, o);
+      if (lane >= o) {
+        wi.x += x;
+        wi.y += y;
+        wi.z += z;
+      }
+    }
+    if (lane < nw) {
+      scratch[3 * lane] = wi.x - w.x;
+      scratch[3 * lane + 1] = wi.y - w.y;
+      scratch[3 * lane + 2] = wi.z - w.z;
+    }
+    if (lane == nw - 1) {
+      tot[0] = wi.x;
+      tot[1] = wi.y;
+      tot[2] = wi.z;
+    }
+  }
+  __syncthreads();
+  return make_int3(scratch[3 * warp] + inc.x - v.x, scratch[3 * warp + 1] + inc.y - v.y,
+                   scratch[3 * warp + 2] + inc.z - v.z);
+}
+
+// One block of 1024 threads (E + 1 <= 1024).  Counts per expert (lanes that
+// hold the same expert add once), one scan for segment starts, segment numbers
+// and work-item offsets, a scatter of the T*K routed pairs (positions within an
+// expert follow the atomics, so their order varies, but every position is
+// computed independently: the results do not depend on it), the shared
+// expert's segment after them, and the GEMM work items of every non-empty
+// segment in expert order.
 __global__ void __launch_bounds__(1024) bt_permute_kernel(PermuteArgs p) {
   extern __shared__ int32_t sh[];
   const int S = p.E + 1;  // segment candidates: experts 0..E-1, then the shared one
   int32_t* cnt = sh;
-  int32_t* start = sh + S;
-  int32_t* seg_of = sh + 2 * S;  // segment index of each candidate (-1: empty)
-  int32_t* cur = sh + 3 * S;     // scatter cursors
-  int32_t* tot = sh + 4 * S;     // [2] item totals
-  const int tid = threadIdx.x;
+  int32_t* cur = sh + S;          // scatter cursors
+  int32_t* scratch = sh + 2 * S;  // [3 * 32] scan scratch
+  int32_t* tot = scratch + 96;    // [3] totals
+  const int tid = threadIdx.x, lane = tid & 31;
   int32_t* seg_e = p.seg;
   int32_t* seg_start = p.seg + S;
   int32_t* seg_cnt = p.seg + 2 * S;
   int32_t* seg_item = p.seg + 3 * S;  // first gate/up item of each segment
+  const int rbg = (p.rows_gu + kGemmRows - 1) / kGemmRows, rbd = (p.rows_dn + kGemmRows - 1) / kGemmRows;
   if (p.single_expert >= 0) {
     if (tid == 0) {
       seg_e[0] = p.single_expert;
@@ -271,80 +318,80 @@ __global__ void __launch_bounds__(1024) bt_permute_kernel(PermuteArgs p) {
       p.seg[4 * S] = 1;
     }
     for (int t = tid; t < p.T; t += blockDim.x) p.pos_tok[t] = t;
-    __syncthreads();
     const int ntb = (p.T + kGemmTokens - 1) / kGemmTokens;
-    const int rbg = (p.rows_gu + kGemmRows - 1) / kGemmRows, rbd = (p.rows_dn + kGemmRows - 1) / kGemmRows;
-    for (int i = tid; i < rbg * ntb; i += blockDim.x) p.items_gu[i] = (0u << 16) | ((uint32_t)(i / ntb) << 8) | (i % ntb);
-    for (int i = tid; i < rbd * ntb; i += blockDim.x) p.items_dn[i] = (0u << 16) | ((uint32_t)(i / ntb) << 8) | (i % ntb);
+    for (int i = tid; i < rbg * ntb; i += blockDim.x) p.items_gu[i] = ((uint32_t)(i / ntb) << 8) | (i % ntb);
+    for (int i = tid; i < rbd * ntb; i += blockDim.x) p.items_dn[i] = ((uint32_t)(i / ntb) << 8) | (i % ntb);
     if (tid == 0) {
       p.n_items[0] = rbg * ntb;
       p.n_items[1] = rbd * ntb;
     }
     return;
   }
+  const int n = p.T * p.K;
   for (int e = tid; e < S; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
-  for (int i = tid; i < p.T * p.K; i += blockDim.x) atomicAdd(&cnt[p.idx[i]], 1);
-  __syncthreads();
-  if (tid == 0) {
-    cnt[p.E] = p.T;
-    int acc = 0, ns = 0, ig = 0, id = 0;
-    const int rbg = (p.rows_gu + kGemmRows - 1) / kGemmRows, rbd = (p.rows_dn + kGemmRows - 1) / kGemmRows;
-    for (int e = 0; e < S; ++e) {
-      start[e] = acc;
-      acc += cnt[e];
-      if (cnt[e] > 0) {
-        const int ntb = (cnt[e] + kGemmTokens - 1) / kGemmTokens;
-        seg_of[e] = ns;
-        seg_e[ns] = e;
-        seg_start[ns] = start[e];
-        seg_cnt[ns] = cnt[e];
-        seg_item[ns] = ig;
-        ig += rbg * ntb;
-        id += rbd * ntb;
-        ++ns;
-      } else {
-        seg_of[e] = -1;
-      }
-    }
-    p.seg[4 * S] = ns;
-    tot[0] = min(ig, p.max_items_gu);
-    tot[1] = min(id, p.max_items_dn);
-    p.n_items[0] = tot[0];
-    p.n_items[1] = tot[1];
+  for (int base = tid - lane; base < n; base += blockDim.x) {
+    const int i = base + lane;
+    const int e = i < n ? p.idx[i] : -1;
+    const uint32_t same = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(same) - 1) atomicAdd(&cnt[e], __popc(same));
   }
   __syncthreads();
-  for (int e = tid; e < S; e += blockDim.x) cur[e] = start[e];
+  if (tid == 0) cnt[p.E] = p.T;
   __syncthreads();
-  for (int i = tid; i < p.T * p.K; i += blockDim.x) {
-    const int e = p.idx[i];
-    const int pos = atomicAdd(&cur[e], 1);
-    p.pos_tok[pos] = i / p.K;
-    p.pos_of[(i / p.K) * (p.K + 1) + i % p.K] = pos;
+  // per candidate: positions, a segment if non-empty, its token blocks
+  const int c = tid < S ? cnt[tid] : 0;
+  const int ntb = (c + kGemmTokens - 1) / kGemmTokens;
+  const int3 pre = block_scan3(make_int3(c, c > 0 ? 1 : 0, ntb), scratch, tot);
+  const int n_seg = tot[1], n_tb = tot[2];
+  if (tid < S) {
+    cur[tid] = pre.x;
+    if (c > 0) {
+      seg_e[pre.y] = tid;
+      seg_start[pre.y] = pre.x;
+      seg_cnt[pre.y] = c;
+      seg_item[pre.y] = rbg * pre.z;
+    }
+  }
+  if (tid == 0) {
+    p.seg[4 * S] = n_seg;
+    p.n_items[0] = min(rbg * n_tb, p.max_items_gu);
+    p.n_items[1] = min(rbd * n_tb, p.max_items_dn);
+  }
+  __syncthreads();
+  for (int base = tid - lane; base < n; base += blockDim.x) {
+    const int i = base + lane;
+    const int e = i < n ? p.idx[i] : -1;
+    const uint32_t same = __match_any_sync(0xffffffffu, e);
+    const int leader = __ffs(same) - 1;
+    int first = 0;
+    if (e >= 0 && lane == leader) first = atomicAdd(&cur[e], __popc(same));
+    first = __shfl_sync(0xffffffffu, first, leader);
+    if (e >= 0) {
+      const int pos = first + __popc(same & ((1u << lane) - 1u));
+      p.pos_tok[pos] = i / p.K;
+      p.pos_of[(i / p.K) * (p.K + 1) + i % p.K] = pos;
+    }
   }
   for (int t = tid; t < p.T; t += blockDim.x) {
-    const int pos = start[p.E] + t;
+    const int pos = p.T * p.K + t;
     p.pos_tok[pos] = t;
     p.pos_of[t * (p.K + 1) + p.K] = pos;
   }
-  // work items: segment-major, then row block, then token block (token blocks
-  // of one row block run side by side and share the weight tiles in L2)
-  const int rbg = (p.rows_gu + kGemmRows - 1) / kGemmRows, rbd = (p.rows_dn + kGemmRows - 1) / kGemmRows;
-  for (int e = tid; e < S; e += blockDim.x) {
-    const int s = seg_of[e];
-    if (s < 0) continue;
-    const int ntb = (cnt[e] + kGemmTokens - 1) / kGemmTokens;
-    const int ig0 = seg_item[s];
-    const int id0 = ig0 / rbg * rbd;  // same number of token blocks before this segment
+  // work items of this thread's segment: segment-major, then row block, then
+  // token block (token blocks of one row block run side by side and share the
+  // weight tiles in L2)
+  if (tid < S && c > 0) {
+    const int s = pre.y, ig0 = rbg * pre.z, id0 = rbd * pre.z;
     for (int rb = 0; rb < rbg; ++rb)
       for (int tb = 0; tb < ntb; ++tb) {
         const int i = ig0 + rb * ntb + tb;
-        if (i < tot[0]) p.items_gu[i] = ((uint32_t)s << 16) | ((uint32_t)rb << 8) | (uint32_t)tb;
+        if (i < p.max_items_gu) p.items_gu[i] = ((uint32_t)s << 16) | ((uint32_t)rb << 8) | (uint32_t)tb;
       }
     for (int rb = 0; rb < rbd; ++rb)
       for (int tb = 0; tb < ntb; ++tb) {
         const int i = id0 + rb * ntb + tb;
-        if (i < tot[1]) p.items_dn[i] = ((uint32_t)s << 16) | ((uint32_t)rb << 8) | (uint32_t)tb;
+        if (i < p.max_items_dn) p.items_dn[i] = ((uint32_t)s << 16) | ((uint32_t)rb << 8) | (uint32_t)tb;
       }
   }
 }
@@ -551,17 +598,28 @@ __global__ void __launch_bounds__(256) bt_gemm_kernel(GemmArgs p) {
 }
 
 // ------------------------------------------------------------------ combine
-// out[t] = bf16(h[t] + y[shared] + sum_k w[t][k] * y[routed k]), fixed order.
+// out[t] = bf16(h[t] + y[shared] + sum_k w[t][k] * y[routed k]), fixed order;
+// four consecutive outputs per thread.
 __global__ void bt_combine_kernel(const uint16_t* __restrict__ h, const float* __restrict__ y,
                                   const int32_t* __restrict__ pos_of, const float* __restrict__ w, int T, int H, int K,
                                   uint16_t* __restrict__ out) {
-  const int64_t n = (int64_t)T * H;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const int tk = (int)(i / H), c = (int)(i % H);
+  const int64_t n4 = (int64_t)T * H / 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const int tk = (int)(4 * i / H), c = (int)(4 * i % H);
     const int32_t* po = pos_of + (size_t)tk * (K + 1);
-    float acc = bf(h[i]) + y[(size_t)po[K] * H + c];
-    for (int k = 0; k < K; ++k) acc = fmaf(w[(size_t)tk * K + k], y[(size_t)po[k] * H + c], acc);
-    out[i] = to_bf16(acc);
+    const uint2 hv = *reinterpret_cast<const uint2*>(h + 4 * i);
+    const float4 ys = *reinterpret_cast<const float4*>(y + (size_t)po[K] * H + c);
+    float a0 = bflo(hv.x) + ys.x, a1 = bfhi(hv.x) + ys.y, a2 = bflo(hv.y) + ys.z, a3 = bfhi(hv.y) + ys.w;
+    for (int k = 0; k < K; ++k) {
+      const float wk = w[(size_t)tk * K + k];
+      const float4 yk = *reinterpret_cast<const float4*>(y + (size_t)po[k] * H + c);
+      a0 = fmaf(wk, yk.x, a0);
+      a1 = fmaf(wk, yk.y, a1);
+      a2 = fmaf(wk, yk.z, a2);
+      a3 = fmaf(wk, yk.w, a3);
+    }
+    *reinterpret_cast<uint2*>(out + 4 * i) = make_uint2((uint32_t)to_bf16(a0) | ((uint32_t)to_bf16(a1) << 16),
+                                                        (uint32_t)to_bf16(a2) | ((uint32_t)to_bf16(a3) << 16));
   }
 }
 
@@ -693,13 +751,13 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   pa.n_items = ws.n_items;
   pa.max_items_gu = ws.max_items_gu;
   pa.max_items_dn = ws.max_items_dn;
-  bt_permute_kernel<<<1, 1024, (size_t)(4 * (a.E + 1) + 2) * 4, st>>>(pa);
+  bt_permute_kernel<<<1, 1024, (size_t)(2 * (a.E + 1) + 96 + 3) * 4, st>>>(pa);
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
   const int rc = a.bits == 4 ? launch_gemms<4>(a, ws, n_sm, st, positions) : launch_gemms<2>(a, ws, n_sm, st, positions);
   if (rc != 0) return rc;
   if (layer) {
-    bt_combine_kernel<<<grid_of((int64_t)a.T * a.H, 256, 8 * n_sm), 256, 0, st>>>(a.h_in, ws.y, ws.pos_of, ws.w, a.T,
+    bt_combine_kernel<<<grid_of((int64_t)a.T * a.H / 4, 256, 8 * n_sm), 256, 0, st>>>(a.h_in, ws.y, ws.pos_of, ws.w, a.T,
                                                                                   a.H, a.K, a.h_out);
     e = cudaGetLastError();
     if (e != cudaSuccess) return (int)e;

@@ -155,8 +155,7 @@ __device__ __forceinline__ void tile_dot(const uint8_t* tile, const uint2 (&bf)[
 // were measured to linger for several microseconds under load.
 __device__ __forceinline__ void st_tagged(uint64_t* p, float v, uint32_t tag) {
   const uint64_t w = (uint64_t)__float_as_uint(v) | ((uint64_t)tag << 32);
-  uint64_t old;
-  asm volatile("atom.relaxed.gpu.global.exch.b64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(w) : "memory");
+  asm volatile("{ .reg .b64 old; atom.relaxed.gpu.global.exch.b64 old, [%0], %1; }" ::"l"(p), "l"(w) : "memory");
 }
 __device__ __forceinline__ uint64_t ld_tagged(const uint64_t* p) {
   uint64_t w;

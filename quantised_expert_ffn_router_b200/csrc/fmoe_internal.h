@@ -202,6 +202,7 @@ inline __host__ __device__ void task_stage_of(int nstage, int n_issuers, int n_t
 constexpr int kGemmRows = 128;       // rows per work item (8 warps x 16)
 constexpr int kGemmTokens = 64;      // tokens (positions) per work item
 constexpr int kGroupedMinTokens = 8; // fmoe_layer_forward uses the batched path from this T on
+constexpr int kBatchMaxExperts = 1023;  // batched permute: one thread per expert plus the shared one
 
 struct BatchWs {              // device buffers, sized for max_tokens at create
   uint16_t* z;                // bf16 [T][H]   (normalised input)
