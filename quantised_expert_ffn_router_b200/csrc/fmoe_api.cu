@@ -31,6 +31,7 @@ struct fmoe_ctx {
   uint16_t* stack_buf[2] = {nullptr, nullptr};  // ping-pong activations, [max_tokens][H] bf16
   void* bws_mem = nullptr;  // batched-path workspace (max_tokens > 1)
   BatchWs bws{};
+  std::vector<TmaDesc> tc_maps;  // per layer: tensor maps of the packed gate/up and down matrices
   DecodePlan plan[3];  // per mode: layer, expert, route (pointers filled per call)
   std::string err;
 };
@@ -388,8 +389,22 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
       ctx->bws_mem = nullptr;
       return bail(fail(ctx, FMOE_ERR_OOM, "batched workspace allocation of %zu bytes failed", bb));
     }
-    batch_ws_carve(static_cast<uint8_t*>(ctx->bws_mem), c.hidden, c.n_experts, c.top_k, c.inter,
-                   std::max(c.max_tokens, 1), ctx->bws);
+    const int rc = batch_ws_carve(static_cast<uint8_t*>(ctx->bws_mem), c.hidden, c.n_experts, c.top_k, c.inter,
+                                  std::max(c.max_tokens, 1), ctx->bws);
+    if (rc != 0) return bail(cuda_fail(ctx, (cudaError_t)rc, "batched tensor maps"));
+    // GEMM inputs past a step's positions are read into unused columns: keep them finite
+    e = cudaMemsetAsync(ctx->bws_mem, 0, bb, (cudaStream_t)stream);
+    if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "batched workspace clear"));
+    ctx->tc_maps.resize((size_t)2 * c.n_layers);
+    const int64_t blob = expert_bytes(c.hidden, c.inter, c.bits);
+    for (int l = 0; l < c.n_layers; ++l) {
+      const uint8_t* ex = static_cast<const uint8_t*>(ctx->layers[l].experts_dev);
+      int r2 = tc_encode_weight_map(ex, blob, c.n_experts + 1, 2 * c.inter, c.hidden, c.bits, &ctx->tc_maps[2 * l]);
+      if (r2 == 0)
+        r2 = tc_encode_weight_map(ex + packed_gu_bytes(c.hidden, c.inter, c.bits), blob, c.n_experts + 1, c.hidden,
+                                  c.inter, c.bits, &ctx->tc_maps[2 * l + 1]);
+      if (r2 != 0) return bail(cuda_fail(ctx, (cudaError_t)r2, "expert tensor maps"));
+    }
   }
   cudaStream_t st = (cudaStream_t)stream;
   e = cudaMemsetAsync(ctx->ws, 0, ctx->ws_bytes, st);
@@ -480,6 +495,11 @@ static BatchArgs batch_args(const fmoe_ctx* ctx, int32_t layer, int32_t T) {
   a.norm_w = static_cast<const uint16_t*>(L.norm_w_dev);
   a.eps = c.rms_eps;
   a.single_expert = -1;
+  if (!ctx->tc_maps.empty()) {
+    a.wmap_gu = &ctx->tc_maps[2 * (size_t)layer];
+    a.wmap_dn = &ctx->tc_maps[2 * (size_t)layer + 1];
+  }
+  a.status = &ctx->hdr->status;
   return a;
 }
 

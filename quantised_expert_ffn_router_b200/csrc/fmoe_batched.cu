@@ -6,18 +6,18 @@
 // every expert once per token; here each selected expert is read once per 64
 // of its tokens.  The steps, all on the caller's stream:
 //   norm     z = RMSNorm(h) (or h), bf16
-//   frag     per (token, 64-group): fp16 values scaled by a power of two so the
-//            group's largest magnitude lies in [2^14, 2^15), plus the group sum
 //   router   logits = W_r z (+ bias), bf16 tensor-core GEMM, fp32 accumulate
 //   top-K    per token (launch_topk_rows)
 //   permute  (token, slot) pairs grouped by expert into segments; the shared
 //            expert's segment holds every token; a list of GEMM work items
-//   gate/up  grouped GEMM: a work item is 128 rows (8 units of 8 gate + 8 up
-//            rows) x 64 positions of one expert; exact integer codes x fp16
-//            values on mma.sync, per-group s*sum(q*x) + b*sum(x) epilogue,
+//   prep     per position: its token's z as fp16, scaled by a power of two so
+//            the row's largest magnitude lies in [2^14, 2^15), columns in the
+//            order the tensor-core A operand uses
+//   gate/up  grouped tcgen05 GEMM (fmoe_grouped_tc.cu): a work item is 128 rows
+//            (8 units of 8 gate + 8 up rows) x up to 64 positions of one expert;
 //            a = silu(g)*u written per position
-//   frag     of a, per (position, 64-group)
-//   down     grouped GEMM, 128 output rows x 64 positions per work item
+//   prep     of a, per position
+//   down     grouped tcgen05 GEMM, 128 output rows x up to 64 positions
 //   combine  out = h + y_shared + sum_k w_k y_k, fp32, one bf16 rounding
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -34,22 +34,6 @@ __device__ __forceinline__ uint16_t to_bf16(float f) { return __bfloat16_as_usho
 __device__ __forceinline__ float pow2(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t c) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(c));
-  return d;
-}
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                        uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                          uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
@@ -64,9 +48,6 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-constexpr uint32_t kMagic = 0x64006400u;  // fp16 pair (1024, 1024)
-constexpr int kBRowBytes = 144;          // fragment record: 128 B of fp16 values, 8 B info, 8 B pad
 
 // ------------------------------------------------------------------ norm
 // One warp per token: z = bf16(h * r * w), r = 1/sqrt(mean(h^2) + eps); a
@@ -105,47 +86,67 @@ __global__ void bt_norm_kernel(const uint16_t* __restrict__ h, const uint16_t* _
   }
 }
 
-// ------------------------------------------------------------------ fragments
-// One warp per (row, 64-group); lane l holds elements 2l, 2l+1.  The group is
-// scaled by 2^sh so its largest magnitude lies in [2^14, 2^15) (any finite
-// input fits fp16); element k of the group is further divided by 4^fs(k) where
-// the packed layout stores its codes as code * 4^fs (the same positions the
-// batch-1 kernel's fragments use).  Output: one 144-byte record per (row,
-// group): 64 fp16 values, then (2^-sh, sum of the group) as two floats, then
-// 8 bytes of padding -- exactly the shared-memory row the GEMM reads, so the
-// copies of a row bring its values and its scale together.
-template <typename Src>
-__global__ void bt_frag_kernel(const Src* __restrict__ src, int rows, int cols, int bits, uint8_t* __restrict__ dst) {
-  const int lane = threadIdx.x & 31;
-  const int ng = cols / kGroup;
-  const int q = 2 * lane, s = q / 16, which = (q % 16) / 8;
-  const int fs = (bits == 4) ? (which ? 4 : 0) : ((s & 1) ? 4 : 0) + (which ? 2 : 0);
-  for (int item = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); item < rows * ng;
-       item += gridDim.x * (blockDim.x / 32)) {
-    const int r = item / ng, G = item % ng;
-    const size_t off = (size_t)r * cols + (size_t)G * kGroup + q;
-    float v0, v1;
-    if constexpr (sizeof(Src) == 2) {
-      const uint32_t p = *reinterpret_cast<const uint32_t*>(src + off);
-      v0 = bflo(p);
-      v1 = bfhi(p);
-    } else {
-      const float2 p = *reinterpret_cast<const float2*>(src + off);
-      v0 = p.x;
-      v1 = p.y;
-    }
-    uint32_t m = max(__float_as_uint(fabsf(v0)), __float_as_uint(fabsf(v1)));
-    m = __reduce_max_sync(0xffffffffu, m);
-    float sum = v0 + v1;
+// ------------------------------------------------------------------ prep
+// Element p of every 16 columns of a GEMM input row holds source column pi(p):
+// the order in which the tensor-core A operand holds the weights (the 16x256b
+// tensor-memory store of an mma.sync-ordered fragment; fmoe_grouped_tc.cu).
+__host__ __device__ constexpr int k_perm(int p) { return 2 * (p >> 2) + (p & 1) + 8 * ((p >> 1) & 1); }
+
+__device__ __forceinline__ void load16(const uint16_t* src, float (&v)[16]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(src), b = *reinterpret_cast<const uint4*>(src + 8);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  for (int k = 0; k < 8; ++k) {
+    v[2 * k] = bflo(w[k]);
+    v[2 * k + 1] = bfhi(w[k]);
+  }
+}
+__device__ __forceinline__ void load16(const float* src, float (&v)[16]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float4 f = reinterpret_cast<const float4*>(src)[k];
+    v[4 * k] = f.x;
+    v[4 * k + 1] = f.y;
+    v[4 * k + 2] = f.z;
+    v[4 * k + 3] = f.w;
+  }
+}
+
+// One warp per position p: dst[p] = fp16(src[row(p)] * 2^sh) in k_perm order,
+// with sh putting the row's largest magnitude in [2^14, 2^15) (any finite row
+// fits fp16; bf16 inputs convert exactly unless they are 2^28 times smaller
+// than the row's largest), and scale[p] = 2^-sh.  row(p) = rowmap[p], or p.
+template <typename Src>
+__global__ void bt_prep_kernel(const Src* __restrict__ src, const int32_t* __restrict__ rowmap, int P, int K,
+                               uint16_t* __restrict__ dst, float* __restrict__ scale) {
+  const int lane = threadIdx.x & 31, nb = K / 16;
+  for (int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x / 32)) {
+    const Src* row = src + (size_t)(rowmap ? rowmap[p] : p) * K;
+    uint32_t m = 0;
+    for (int b = lane; b < nb; b += 32) {
+      float v[16];
+      load16(row + 16 * b, v);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) m = max(m, __float_as_uint(fabsf(v[k])));
+    }
+    m = __reduce_max_sync(0xffffffffu, m);
     const int e = (int)((m >> 23) & 0xFF) - 127;
-    int sh = (m == 0) ? 0 : 14 - max(e, -126);
-    sh = min(sh, 126);
-    const float scl = pow2(sh - fs);
-    uint8_t* row = dst + ((size_t)r * ng + G) * kBRowBytes;
-    *reinterpret_cast<__half2*>(row + 4 * lane) = __floats2half2_rn(v0 * scl, v1 * scl);
-    if (lane == 0) *reinterpret_cast<float2*>(row + kGroup * 2) = make_float2(pow2(-sh), sum);  // after the values
+    const int sh = m == 0 ? 0 : min(14 - max(e, -126), 126);
+    const float mul = pow2(sh);
+    if (lane == 0) scale[p] = pow2(-sh);
+    uint16_t* drow = dst + (size_t)p * K;
+    for (int b = lane; b < nb; b += 32) {
+      float v[16];
+      load16(row + 16 * b, v);
+      uint32_t o[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const __half2 h = __floats2half2_rn(v[k_perm(2 * k)] * mul, v[k_perm(2 * k + 1)] * mul);
+        o[k] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      reinterpret_cast<uint4*>(drow + 16 * b)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      reinterpret_cast<uint4*>(drow + 16 * b)[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
   }
 }
 
@@ -396,207 +397,6 @@ __global__ void __launch_bounds__(1024) bt_permute_kernel(PermuteArgs p) {
   }
 }
 
-// ------------------------------------------------------------------ grouped GEMM
-struct GemmArgs {
-  const uint8_t* experts;
-  int64_t blob_bytes;
-  int64_t region;        // byte offset of the matrix inside a blob (0: gate/up, else down)
-  int rows;              // matrix rows (2I gate/up, H down)
-  int k_groups;          // 64-column groups along K (H/64 gate/up, I/64 down)
-  int ldo;               // elements per output row (I for a, H for y)
-  const int32_t* seg;    // segment table
-  int n_seg_stride;      // E+1
-  const uint32_t* items;
-  const int32_t* n_items;
-  const int32_t* pos_tok;  // B row of a position (gate/up: its token; null: the position itself)
-  const uint8_t* bsrc;     // fragment records [rows][k_groups][144 B]
-  float* out;              // gate/up: a [pos][I]; down: y [pos][H]
-};
-
-constexpr int kStages = 6;      // 6 x 13.5 KB per block; two blocks per SM keep ~140 KB of copies in flight
-constexpr int kBRowWords = kBRowBytes / 4;  // 36: the record's 4 extra words keep fragment reads conflict-free
-template <int BITS>
-struct GemmSmem {
-  static constexpr int TB = 16 * kGroup * BITS / 8 + 64;
-  static constexpr int A_BYTES = 8 * TB;
-  static constexpr int B_BYTES = kGemmTokens * kBRowBytes;
-  static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int TOTAL = kStages * STAGE;
-};
-
-// 4-bit: the four A fragment registers of one 16-column slice from lane word w.
-__device__ __forceinline__ void a_frag4(uint32_t w, uint32_t (&a)[4]) {
-  const uint32_t w8 = w >> 8;
-  a[0] = hsub2(lop_and_or(w, 0x000F000Fu, kMagic), kMagic);
-  a[1] = hsub2(lop_and_or(w8, 0x000F000Fu, kMagic), kMagic);
-  a[2] = hsub2(lop_and_or(w, 0x00F000F0u, kMagic), kMagic);
-  a[3] = hsub2(lop_and_or(w8, 0x00F000F0u, kMagic), kMagic);
-}
-// 2-bit: fragments of the even and odd slices stored in lane word w.
-__device__ __forceinline__ void a_frag2(uint32_t w, uint32_t (&ae)[4], uint32_t (&ao)[4]) {
-  const uint32_t w8 = w >> 8;
-  ae[0] = hsub2(lop_and_or(w, 0x00030003u, kMagic), kMagic);
-  ae[1] = hsub2(lop_and_or(w8, 0x00030003u, kMagic), kMagic);
-  ae[2] = hsub2(lop_and_or(w, 0x000C000Cu, kMagic), kMagic);
-  ae[3] = hsub2(lop_and_or(w8, 0x000C000Cu, kMagic), kMagic);
-  ao[0] = hsub2(lop_and_or(w, 0x00300030u, kMagic), kMagic);
-  ao[1] = hsub2(lop_and_or(w8, 0x00300030u, kMagic), kMagic);
-  ao[2] = hsub2(lop_and_or(w, 0x00C000C0u, kMagic), kMagic);
-  ao[3] = hsub2(lop_and_or(w8, 0x00C000C0u, kMagic), kMagic);
-}
-
-// One 128-row x 64-position work item per iteration.  Warp w owns rows
-// 16*(8*rb + w) .. +15 (one packed row block); per 64-column group it takes 4
-// k-slices x (positions/8) token blocks of mma.sync and folds the group's scale
-// and bias: acc += s * C * inv_scale(position, group) + b * sum(position, group).
-// All threads stream each group's 8 weight tiles and B records into a ring of
-// stages with 16-byte cp.async copies (records are gathered rows, too small
-// for bulk copies to pay); a stage is refilled after the block barrier that
-// follows its last use.
-template <int BITS, bool GATE_UP>
-__global__ void __launch_bounds__(256) bt_gemm_kernel(GemmArgs p) {
-  using L = GemmSmem<BITS>;
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int S = p.n_seg_stride;
-  const int n_items = *p.n_items;
-  const int n_rb16 = p.rows / 16;  // packed row blocks of the matrix
-  constexpr int kAChunks = L::A_BYTES / 16, kBChunks = kGemmTokens * kBRowBytes / 16;
-  constexpr int kAPer = (kAChunks + 255) / 256, kBPer = (kBChunks + 255) / 256;
-  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-    const uint32_t item = p.items[it];
-    const int s = (int)(item >> 16), rb = (int)((item >> 8) & 0xFF), tb = (int)(item & 0xFF);
-    const int e = p.seg[s], pos0 = p.seg[S + s] + tb * kGemmTokens;
-    const int ntok = min(kGemmTokens, p.seg[2 * S + s] - tb * kGemmTokens);
-    const uint8_t* mat = p.experts + (int64_t)e * p.blob_bytes + p.region;
-    const int my_rb = rb * 8 + warp;  // this warp's packed row block
-    const bool active = my_rb < n_rb16;
-    const int nb = (ntok + 7) / 8;    // 8-position blocks holding tokens (the rest are skipped)
-    // This thread's 16-byte copies of every group: sources at group 0 (a
-    // group adds TB to a weight source and 144 to a record source) and fixed
-    // shared-memory offsets.  Weight tiles of rows past the matrix and records
-    // of positions past the segment are not copied (their columns are unused).
-    const uint8_t* asrc[kAPer];
-    uint32_t adst[kAPer];
-    bool aok[kAPer];
-#pragma unroll
-    for (int k = 0; k < kAPer; ++k) {
-      const int c = tid + 256 * k, w = c / (L::TB / 16), off = (c % (L::TB / 16)) * 16;
-      aok[k] = c < kAChunks && rb * 8 + w < n_rb16;
-      asrc[k] = mat + (int64_t)(aok[k] ? rb * 8 + w : 0) * p.k_groups * L::TB + off;
-      adst[k] = (uint32_t)(w * L::TB + off);
-    }
-    const uint8_t* bsrc[kBPer];
-    uint32_t bdst[kBPer];
-    bool bok[kBPer];
-#pragma unroll
-    for (int k = 0; k < kBPer; ++k) {
-      const int c = tid + 256 * k, j = c / (kBRowBytes / 16), part = c % (kBRowBytes / 16);
-      bok[k] = c < kBChunks && j < ntok;
-      const int row = bok[k] ? (p.pos_tok ? p.pos_tok[pos0 + j] : pos0 + j) : 0;
-      bsrc[k] = p.bsrc + (size_t)row * p.k_groups * kBRowBytes + part * 16;
-      bdst[k] = (uint32_t)(L::A_BYTES + j * kBRowBytes + part * 16);
-    }
-    auto load = [&](int gi, int st) {
-      uint8_t* base = smem + st * L::STAGE;
-#pragma unroll
-      for (int k = 0; k < kAPer; ++k)
-        if (aok[k]) cp_async16(base + adst[k], asrc[k] + (int64_t)gi * L::TB, 16u);
-#pragma unroll
-      for (int k = 0; k < kBPer; ++k)
-        if (bok[k]) cp_async16(base + bdst[k], bsrc[k] + (size_t)gi * kBRowBytes, 16u);
-    };
-    float acc[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-    __syncthreads();  // the previous item's stages are no longer read
-#pragma unroll
-    for (int st = 0; st < kStages - 1; ++st) {
-      if (st < p.k_groups) load(st, st);
-      cp_async_commit();
-    }
-    for (int gi = 0; gi < p.k_groups; ++gi) {
-      cp_async_wait<kStages - 2>();
-      __syncthreads();  // stage gi visible to all; the stage of gi - 1 is free again
-      if (gi + kStages - 1 < p.k_groups) load(gi + kStages - 1, (gi + kStages - 1) % kStages);
-      cp_async_commit();
-      const int st = gi % kStages;
-      if (active) {
-        const uint8_t* sa = smem + st * L::STAGE;
-        const uint32_t* sb = reinterpret_cast<const uint32_t*>(sa + L::A_BYTES);
-        const uint8_t* tile = sa + warp * L::TB;
-        float c[8][4];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.f;
-        if (BITS == 4) {
-          const uint4 qv = *reinterpret_cast<const uint4*>(tile + lane * 16);
-          const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-          for (int sl = 0; sl < 4; ++sl) {
-            uint32_t a[4];
-            a_frag4(qw[sl], a);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (j >= nb) break;
-              const uint32_t* br = sb + (8 * j + g) * kBRowWords + 8 * sl + t;
-              mma_f16(c[j], a[0], a[1], a[2], a[3], br[0], br[4]);
-            }
-          }
-        } else {
-          const uint2 qv = *reinterpret_cast<const uint2*>(tile + lane * 8);
-          const uint32_t qw[2] = {qv.x, qv.y};
-#pragma unroll
-          for (int wj = 0; wj < 2; ++wj) {
-            uint32_t ae[4], ao[4];
-            a_frag2(qw[wj], ae, ao);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (j >= nb) break;
-              const uint32_t* be = sb + (8 * j + g) * kBRowWords + 8 * (2 * wj) + t;
-              const uint32_t* bo = sb + (8 * j + g) * kBRowWords + 8 * (2 * wj + 1) + t;
-              mma_f16(c[j], ae[0], ae[1], ae[2], ae[3], be[0], be[4]);
-              mma_f16(c[j], ao[0], ao[1], ao[2], ao[3], bo[0], bo[4]);
-            }
-          }
-        }
-        const uint2 sbv = *reinterpret_cast<const uint2*>(tile + 16 * kGroup * BITS / 8 + g * 8);
-        const float s0 = bflo(sbv.x), b0 = bfhi(sbv.x), s8 = bflo(sbv.y), b8 = bfhi(sbv.y);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j >= nb) break;
-          // the record's info: (2^-scale, sum) right after the 64 values
-          const float2 i0 = *reinterpret_cast<const float2*>(sb + (8 * j + 2 * t) * kBRowWords + 32);
-          const float2 i1 = *reinterpret_cast<const float2*>(sb + (8 * j + 2 * t + 1) * kBRowWords + 32);
-          acc[j][0] = fmaf(s0 * i0.x, c[j][0], fmaf(b0, i0.y, acc[j][0]));
-          acc[j][1] = fmaf(s0 * i1.x, c[j][1], fmaf(b0, i1.y, acc[j][1]));
-          acc[j][2] = fmaf(s8 * i0.x, c[j][2], fmaf(b8, i0.y, acc[j][2]));
-          acc[j][3] = fmaf(s8 * i1.x, c[j][3], fmaf(b8, i1.y, acc[j][3]));
-        }
-      }
-    }
-    cp_async_wait<0>();
-    if (!active) continue;
-    // lane holds rows g, g+8 of its row block for positions 8j + 2t, 8j + 2t + 1
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int jt = 8 * j + 2 * t + h;
-        if (jt >= ntok) continue;
-        float* orow = p.out + (size_t)(pos0 + jt) * p.ldo;
-        if (GATE_UP) {
-          // row g is gate row 8*my_rb + g, row g + 8 its up row
-          const float gv = acc[j][h], uv = acc[j][2 + h];
-          orow[my_rb * 8 + g] = gv / (1.0f + expf(-gv)) * uv;
-        } else {
-          orow[my_rb * 16 + g] = acc[j][h];
-          orow[my_rb * 16 + g + 8] = acc[j][2 + h];
-        }
-      }
-    }
-  }
-}
-
 // ------------------------------------------------------------------ combine
 // out[t] = bf16(h[t] + y[shared] + sum_k w[t][k] * y[routed k]), fixed order;
 // four consecutive outputs per thread.
@@ -628,46 +428,6 @@ int grid_of(int64_t work, int per_block, int cap) {
   return (int)(b < 1 ? 1 : (b > cap ? cap : b));
 }
 
-template <int BITS>
-int launch_gemms(const BatchArgs& a, const BatchWs& ws, int n_sm, cudaStream_t st, int positions) {
-  using L = GemmSmem<BITS>;
-  cudaFuncSetAttribute(bt_gemm_kernel<BITS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
-  cudaFuncSetAttribute(bt_gemm_kernel<BITS, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
-  GemmArgs g{};
-  g.experts = a.experts;
-  g.blob_bytes = a.blob_bytes;
-  g.seg = ws.seg;
-  g.n_seg_stride = a.E + 1;
-  // gate/up: B = z fragments of each position's token
-  g.region = 0;
-  g.rows = 2 * a.I;
-  g.k_groups = a.H / kGroup;
-  g.ldo = a.I;
-  g.items = ws.items_gu;
-  g.n_items = ws.n_items;
-  g.pos_tok = ws.pos_tok;
-  g.bsrc = ws.zf;
-  g.out = ws.a;
-  bt_gemm_kernel<BITS, true><<<2 * n_sm, 256, L::TOTAL, st>>>(g);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return (int)e;
-  // fragments of a, per position
-  bt_frag_kernel<float><<<grid_of((int64_t)positions * (a.I / kGroup), 8, 8 * n_sm), 256, 0, st>>>(
-      ws.a, positions, a.I, BITS, ws.af);
-  // down: B = a fragments of the position itself
-  g.region = packed_gu_bytes(a.H, a.I, BITS);
-  g.rows = a.H;
-  g.k_groups = a.I / kGroup;
-  g.ldo = a.H;
-  g.items = ws.items_dn;
-  g.n_items = ws.n_items + 1;
-  g.pos_tok = nullptr;
-  g.bsrc = ws.af;
-  g.out = a.single_expert >= 0 ? a.y_out : ws.y;
-  bt_gemm_kernel<BITS, false><<<2 * n_sm, 256, L::TOTAL, st>>>(g);
-  return (int)cudaGetLastError();
-}
-
 }  // namespace
 
 namespace {
@@ -686,7 +446,8 @@ size_t carve(uintptr_t base, int H, int E, int K, int I, int T, BatchWs& ws) {
   ws.max_items_gu = rbg * max_tb;
   ws.max_items_dn = rbd * max_tb;
   ws.z = reinterpret_cast<uint16_t*>(take((size_t)T * H * 2));
-  ws.zf = reinterpret_cast<uint8_t*>(take((size_t)T * (H / kGroup) * kBRowBytes));
+  ws.zp = reinterpret_cast<uint16_t*>(take(P * H * 2));
+  ws.zsc = reinterpret_cast<float*>(take(P * 4));
   ws.logits = reinterpret_cast<float*>(take((size_t)T * E * 4));
   ws.logit_part = reinterpret_cast<float*>(take((size_t)kRtSplit * T * E * 4));
   ws.idx = reinterpret_cast<int32_t*>(take((size_t)T * K * 4));
@@ -699,7 +460,8 @@ size_t carve(uintptr_t base, int H, int E, int K, int I, int T, BatchWs& ws) {
   ws.items_dn = reinterpret_cast<uint32_t*>(take((size_t)ws.max_items_dn * 4));
   ws.n_items = reinterpret_cast<int32_t*>(take(2 * 4));
   ws.a = reinterpret_cast<float*>(take(P * I * 4));
-  ws.af = reinterpret_cast<uint8_t*>(take(P * (I / kGroup) * kBRowBytes));
+  ws.ap = reinterpret_cast<uint16_t*>(take(P * I * 2));
+  ws.asc = reinterpret_cast<float*>(take(P * 4));
   ws.y = reinterpret_cast<float*>(take(P * H * 4));
   return off;
 }
@@ -710,8 +472,11 @@ size_t batch_ws_bytes(int H, int E, int K, int I, int T) {
   return carve(0, H, E, K, I, T, ws);
 }
 
-void batch_ws_carve(uint8_t* base, int H, int E, int K, int I, int T, BatchWs& ws) {
+int batch_ws_carve(uint8_t* base, int H, int E, int K, int I, int T, BatchWs& ws) {
   carve(reinterpret_cast<uintptr_t>(base), H, E, K, I, T, ws);
+  const int P = T * (K + 1);
+  const int rc = tc_encode_token_map(ws.zp, H, P, &ws.zmap);
+  return rc != 0 ? rc : tc_encode_token_map(ws.ap, I, P, &ws.amap);
 }
 
 int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream) {
@@ -719,8 +484,6 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   const bool layer = a.single_expert < 0;
   const int positions = layer ? a.T * (a.K + 1) : a.T;
   bt_norm_kernel<<<grid_of(a.T, 8, 4 * n_sm), 256, 0, st>>>(a.h_in, a.norm_w, a.eps, a.T, a.H, ws.z);
-  bt_frag_kernel<uint16_t><<<grid_of((int64_t)a.T * (a.H / kGroup), 8, 8 * n_sm), 256, 0, st>>>(
-      ws.z, a.T, a.H, a.bits, ws.zf);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
   if (layer) {
@@ -754,7 +517,32 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   bt_permute_kernel<<<1, 1024, (size_t)(2 * (a.E + 1) + 96 + 3) * 4, st>>>(pa);
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
-  const int rc = a.bits == 4 ? launch_gemms<4>(a, ws, n_sm, st, positions) : launch_gemms<2>(a, ws, n_sm, st, positions);
+  // gate/up: B = each position's token input
+  bt_prep_kernel<uint16_t><<<grid_of(positions, 8, 8 * n_sm), 256, 0, st>>>(ws.z, ws.pos_tok, positions, a.H, ws.zp,
+                                                                           ws.zsc);
+  TcArgs g{};
+  g.seg = ws.seg;
+  g.S = a.E + 1;
+  g.items = ws.items_gu;
+  g.n_items = ws.n_items;
+  g.k_chunks = (a.H + 127) / 128;
+  g.rows = 2 * a.I;
+  g.ldo = a.I;
+  g.bscale = ws.zsc;
+  g.out = ws.a;
+  g.status = a.status;
+  int rc = launch_tc_gemm(a.bits, true, *a.wmap_gu, ws.zmap, g, n_sm, stream);
+  if (rc != 0) return rc;
+  // down: B = the position's activation
+  bt_prep_kernel<float><<<grid_of(positions, 8, 8 * n_sm), 256, 0, st>>>(ws.a, nullptr, positions, a.I, ws.ap, ws.asc);
+  g.items = ws.items_dn;
+  g.n_items = ws.n_items + 1;
+  g.k_chunks = (a.I + 127) / 128;
+  g.rows = a.H;
+  g.ldo = a.H;
+  g.bscale = ws.asc;
+  g.out = layer ? ws.y : a.y_out;
+  rc = launch_tc_gemm(a.bits, false, *a.wmap_dn, ws.amap, g, n_sm, stream);
   if (rc != 0) return rc;
   if (layer) {
     bt_combine_kernel<<<grid_of((int64_t)a.T * a.H / 4, 256, 8 * n_sm), 256, 0, st>>>(a.h_in, ws.y, ws.pos_of, ws.w, a.T,

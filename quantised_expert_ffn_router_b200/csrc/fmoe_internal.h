@@ -78,6 +78,7 @@ static_assert(sizeof(WsHeader) <= 256, "header");
 constexpr uint32_t kStatusTimeoutRouter = 0x1;
 constexpr uint32_t kStatusTimeoutH = 0x2;
 constexpr uint32_t kStatusTimeoutTma = 0x4;
+constexpr uint32_t kStatusTimeoutTc = 0x8;   // a bounded wait of the grouped tensor-core GEMM ran out
 
 
 enum DecodeMode : int { kModeLayer = 0, kModeExpert = 1, kModeRoute = 2 };
@@ -204,9 +205,15 @@ constexpr int kGemmTokens = 64;      // tokens (positions) per work item
 constexpr int kGroupedMinTokens = 8; // fmoe_layer_forward uses the batched path from this T on
 constexpr int kBatchMaxExperts = 1023;  // batched permute: one thread per expert plus the shared one
 
+// Opaque copy of a TMA tensor map (CUtensorMap: 128 bytes, 64-byte aligned).
+struct TmaDesc {
+  alignas(64) unsigned char bytes[128];
+};
+
 struct BatchWs {              // device buffers, sized for max_tokens at create
   uint16_t* z;                // bf16 [T][H]   (normalised input)
-  uint8_t* zf;                // [T][H/64] records: 64 scaled fp16 values, (2^-scale, group sum), pad
+  uint16_t* zp;               // fp16 [T*(K+1)][H] GEMM input of each position (scaled, k-permuted)
+  float* zsc;                 // [T*(K+1)] 2^sh that undoes the scaling of zp
   float* logits;              // [T][E]
   float* logit_part;          // [4][T][E] partial router logits (K split)
   int32_t* idx;               // [T][K]
@@ -219,9 +226,11 @@ struct BatchWs {              // device buffers, sized for max_tokens at create
   uint32_t* items_dn;
   int32_t* n_items;           // [2]
   float* a;                   // [T*(K+1)][I] activations
-  uint8_t* af;                // [T*(K+1)][I/64] records, as zf
+  uint16_t* ap;               // fp16 [T*(K+1)][I] down-GEMM input (scaled, k-permuted)
+  float* asc;                 // [T*(K+1)]
   float* y;                   // [T*(K+1)][H] expert outputs
   int max_items_gu, max_items_dn;
+  TmaDesc zmap, amap;         // 16 x 64 boxes of zp / ap, 128-byte swizzle
 };
 
 struct BatchArgs {
@@ -238,11 +247,38 @@ struct BatchArgs {
   float* w_out;               // [T][K] or null
   int single_expert;          // >= 0: expert mode on this expert (0..E, E = shared), output y_out
   float* y_out;               // [T][H] fp32 (expert mode)
+  const TmaDesc* wmap_gu;     // tensor maps of the layer's packed gate/up and down matrices
+  const TmaDesc* wmap_dn;
+  uint32_t* status;           // device status word (kStatus* bits)
 };
 
-// Bytes of the batched workspace for T tokens; carves it out of `base`.
+// Bytes of the batched workspace for T tokens; carves it out of `base` and
+// encodes its tensor maps (returns a cudaError_t value).
 size_t batch_ws_bytes(int H, int E, int K, int I, int T);
-void batch_ws_carve(uint8_t* base, int H, int E, int K, int I, int T, BatchWs& ws);
+int batch_ws_carve(uint8_t* base, int H, int E, int K, int I, int T, BatchWs& ws);
+
+// Grouped tensor-core GEMM (fmoe_grouped_tc.cu).
+struct TcArgs {
+  const int32_t* seg;         // segment table ([4][S] + n_seg)
+  int S;                      // E + 1
+  const uint32_t* items;      // work items (seg << 16 | row block << 8 | token block)
+  const int32_t* n_items;
+  int k_chunks;               // ceil(K / 128)
+  int rows;                   // matrix rows (2I gate/up, H down)
+  int ldo;                    // output row length (I: a, H: y)
+  const float* bscale;        // per position: 2^sh undoing the input scaling
+  float* out;                 // gate/up: a [pos][I]; down: y [pos][H]
+  uint32_t* status;
+};
+// Tensor map over the packed matrix at `matrix0` of each of n_blobs experts
+// (blob_bytes apart): uint64 elements, 3-D (band bytes/8, rows/16, n_blobs),
+// box = 2 tiles x 8 bands.
+int tc_encode_weight_map(const uint8_t* matrix0, int64_t blob_bytes, int n_blobs, int rows, int cols, int bits,
+                         TmaDesc* out);
+// Tensor map over an fp16 [rows][cols] matrix, 64 x 16 boxes, 128-byte swizzle.
+int tc_encode_token_map(const uint16_t* base, int cols, int rows, TmaDesc* out);
+int launch_tc_gemm(int bits, bool gate_up, const TmaDesc& wmap, const TmaDesc& xmap, const TcArgs& a, int n_sm,
+                   void* stream);
 int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream);
 
 // Top-K and renormalised weights of T rows of fp32 logits (one warp per row).
