@@ -475,8 +475,8 @@ size_t batch_ws_bytes(int H, int E, int K, int I, int T) {
 int batch_ws_carve(uint8_t* base, int H, int E, int K, int I, int T, BatchWs& ws) {
   carve(reinterpret_cast<uintptr_t>(base), H, E, K, I, T, ws);
   const int P = T * (K + 1);
-  const int rc = tc_encode_token_map(ws.zp, H, P, &ws.zmap);
-  return rc != 0 ? rc : tc_encode_token_map(ws.ap, I, P, &ws.amap);
+  const int rc = tc_encode_token_maps(ws.zp, H, P, ws.zmap);
+  return rc != 0 ? rc : tc_encode_token_maps(ws.ap, I, P, ws.amap);
 }
 
 int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream) {

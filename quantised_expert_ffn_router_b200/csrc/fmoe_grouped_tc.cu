@@ -9,23 +9,28 @@
 // Architecture") and X an fp16 copy of the positions' inputs, each row scaled
 // by a power of two (bt_prep_kernel, fmoe_batched.cu).
 //
-// One persistent block per SM, 14 warps:
+// One persistent block per SM, 15 warps:
 //   warp 0      TMA producer.  Per 128-column chunk (one ring stage): one 3-D
-//               copy of the item's 8 bands x 2 packed tiles and 2*ceil(n/16)
-//               copies of 16-row x 64-column fp16 boxes of X (128-byte swizzle).
-//   warp 1      allocates tensor memory; one lane issues tcgen05.mma (A from
-//               tensor memory, B from shared memory, fp32 accumulator in tensor
-//               memory, M=128, N=ceil(n/16)*16, 8 x K=16 per chunk) and commits
-//               to the ring / buffer barriers.
+//               copy of the item's 8 bands x 2 packed tiles and one 3-D copy of
+//               the n' = ceil(n/16)*16 rows x 2 x 64 columns of X (128-byte
+//               swizzle; one of four tensor maps by n').  A TMA instruction
+//               costs the issuing lane ~0.1 us, so a chunk takes two.
+//   warps 1, 14 MMA issuers (warp 1 also allocates tensor memory): one lane
+//               each, even / odd chunks, each into its own accumulator (A from
+//               tensor memory, B from shared memory, fp32 in tensor memory,
+//               M=128, N=ceil(n/16)*16, 8 x K=16 per chunk), committing to the
+//               ring / buffer barriers.  A thread issues one tcgen05.mma per
+//               ~55 cycles however small N is, so two issuers halve the time
+//               the tensor core needs per chunk.
 //   warps 2-9   two groups of four that take alternate chunks: a warp turns two
 //               bands (32 rows) x 2 tiles into fp16 weights and stores them into
 //               the A buffer with tcgen05.st.16x256b, whose thread layout is the
 //               mma.sync fragment layout the packed tile is stored in (lane
 //               4g+t: rows g and g+8, columns 2t, 2t+1 | 2t+8, 2t+9).
-//   warps 10-13 epilogue: read the accumulator (two buffers, so it overlaps
-//               the next item's main loop), scale each column back by its
-//               position's power of two, and write a = silu(g)*u (gate/up) or
-//               y (down) in fp32.
+//   warps 10-13 epilogue: add the two accumulators (double-buffered, so it
+//               overlaps the next item's main loop), scale each column back by
+//               its position's power of two, and write a = silu(g)*u (gate/up)
+//               or y (down) in fp32.
 //
 // K order.  The 16x256b store puts a lane's fragment columns {2t, 2t+1, 2t+8,
 // 2t+9} of a 16-column slice at tensor-memory positions 4t..4t+3, so within
@@ -54,14 +59,15 @@
 namespace fmoe {
 namespace {
 
-constexpr int kTcWarps = 14;
+constexpr int kTcWarps = 15;
 constexpr int kTcThreads = kTcWarps * 32;
 constexpr int kTcChunk = 128;                     // K columns per ring stage (2 tiles)
-constexpr int kTcBHalf = kGemmTokens * 128;       // one 64-column half of X: 64 rows x 128 B
-constexpr int kTcBBytes = 2 * kTcBHalf;           // 16 KB
+constexpr int kTcBBytes = 2 * kGemmTokens * 128;  // X in a stage: 2 halves x up to 64 rows x 128 B (16 KB)
 constexpr int kTcABufs = 4;                       // A buffers in tensor memory (64 columns each)
-constexpr int kTcDCols = kGemmTokens;             // accumulator columns per buffer
-constexpr int kTcACol0 = 2 * kTcDCols;            // first A column (after two accumulators)
+constexpr int kTcXMaps = kGemmTokens / 16;          // input tensor maps, one per box height
+constexpr int kTcIssuers = 2;                     // MMA-issuing threads, one accumulator each
+constexpr int kTcDCols = kTcIssuers * kGemmTokens;  // accumulator columns per buffer (both issuers)
+constexpr int kTcACol0 = 2 * kTcDCols;            // first A column (after two buffers)
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint64_t kTcWaitNs = 500ull * 1000 * 1000;  // bounded waits: 0.5 s
 
@@ -117,13 +123,6 @@ __device__ __forceinline__ void tma_3d(uint32_t dst, const void* map, int x, int
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
           dst),
       "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tma_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          dst),
-      "l"(map), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -261,9 +260,13 @@ __device__ __forceinline__ ItemInfo item_info(const TcArgs& p, int it) {
   return f;
 }
 
+struct XMaps {
+  CUtensorMap m[kTcXMaps];  // box heights 16, 32, 48, 64
+};
+
 template <int BITS, bool GATE_UP>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    bt_tc_gemm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, TcArgs p) {
+    bt_tc_gemm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ XMaps xmaps, TcArgs p) {
   using L = TcL<BITS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
@@ -291,10 +294,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(aempty(b), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(dfull(b), 1);
+      mbar_init(dfull(b), kTcIssuers);
       mbar_init(dempty(b), 4);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, kTcIssuers);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -333,23 +336,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t st = sbase + (uint32_t)s * L::STAGE;
           mbar_expect_tx(full(s), bytes);
           tma_3d(st + kTcBBytes, &wmap, kc * 2 * L::TB / 8, f.rb * 8, f.e, full(s));
-          for (int j = 0; j < f.npad / 16; ++j) {
-            tma_2d(st + 2048u * j, &xmap, kc * kTcChunk, f.pos0 + 16 * j, full(s));
-            tma_2d(st + kTcBHalf + 2048u * j, &xmap, kc * kTcChunk + 64, f.pos0 + 16 * j, full(s));
-          }
+          // X rows pos0 .. pos0 + n' - 1, 64-column blocks 2kc and 2kc + 1: [half][n'][128 B]
+          tma_3d(st, &xmaps.m[f.npad / 16 - 1], 0, f.pos0, 2 * kc, full(s));
         }
       }
       // copies still in flight land before the block exits
       const uint32_t c0 = c > (uint32_t)L::NS ? c - L::NS : 0u;
       for (uint32_t k = c0; k < c; ++k) mbar_wait(full((int)(k % L::NS)), (k / L::NS) & 1u, nullptr);
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == 14) {
+    // ---------------------------------------------------------------- MMA issuers
+    // Everything between two MMAs is a constant offset: per chunk one
+    // descriptor add and eight unrolled MMAs.  The ring's full barrier was
+    // waited on by the dequantisers whose A-buffer barrier this lane waits on.
     if (lane == 0) {
+      const int j = warp == 1 ? 0 : 1;
+      const uint64_t bdesc0 = sw128_desc(sbase);
       uint32_t c = 0, ii = 0;
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++ii) {
-        const ItemInfo f = item_info(p, it);
+      int it = blockIdx.x;
+      ItemInfo f = it < n_items ? item_info(p, it) : ItemInfo{};
+      for (; ok && it < n_items; it += gridDim.x, ++ii) {
+        const int nit = it + (int)gridDim.x;
+        const ItemInfo nf = nit < n_items ? item_info(p, nit) : f;  // loads in flight during this item
         const int d = (int)(ii & 1u);
         if (!mbar_wait(dempty(d), ((ii >> 1) & 1u) ^ 1u, abort_flag)) {
           fail();
@@ -357,27 +366,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_fence_after();
         const uint32_t idesc = f16_idesc(f.npad);
-        const uint32_t dcol = tmem + (uint32_t)(d * kTcDCols);
+        const uint32_t dcol = tmem + (uint32_t)(d * kTcDCols + j * kGemmTokens);
         for (int kc = 0; kc < p.k_chunks; ++kc, ++c) {
+          if ((kc & 1) != j) continue;
           const int s = (int)(c % L::NS), ab = (int)(c % kTcABufs);
-          if (!mbar_wait(full(s), (c / L::NS) & 1u, abort_flag) ||
-              !mbar_wait(afull(ab), (c / kTcABufs) & 1u, abort_flag)) {
+          if (!mbar_wait(afull(ab), (c / kTcABufs) & 1u, abort_flag)) {
             fail();
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t st = sbase + (uint32_t)s * L::STAGE;
-          const uint32_t acol = tmem + (uint32_t)(kTcACol0 + ab * 64);
+          const uint64_t bd = bdesc0 + (uint64_t)((uint32_t)s * (uint32_t)(L::STAGE >> 4));
+          const uint32_t ad = tmem + (uint32_t)(kTcACol0 + ab * 64);
+          // K step ks: A columns +8, B +32 bytes inside a 64-column half, +n' rows of
+          // 128 bytes across halves
+          tc_mma(dcol, ad, bd, idesc, kc > 1 ? 1u : 0u);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t bdesc = sw128_desc(st + (uint32_t)((ks >> 2) * kTcBHalf + (ks & 3) * 32));
-            tc_mma(dcol, acol + 8u * ks, bdesc, idesc, (kc | ks) != 0 ? 1u : 0u);
-          }
+          for (int ks = 1; ks < 4; ++ks) tc_mma(dcol, ad + 8u * ks, bd + (uint64_t)(ks * 2), idesc, 1u);
+          const uint64_t bd1 = bd + (uint64_t)(f.npad * 8);
+#pragma unroll
+          for (int ks = 4; ks < 8; ++ks) tc_mma(dcol, ad + 8u * ks, bd1 + (uint64_t)((ks - 4) * 2), idesc, 1u);
           tc_commit(empty(s));
           tc_commit(aempty(ab));
         }
         if (ok) tc_commit(dfull(d));
+        f = nf;
       }
       // all issued tensor-core work completes before tensor memory is freed
       tc_commit(drain);
@@ -432,20 +445,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tc_fence_after();
       const uint32_t dcol = tmem + (uint32_t)(d * kTcDCols);
+      const bool two = p.k_chunks > 1;  // the second issuer's accumulator holds chunks 1, 3, ...
+      auto sum2 = [&](uint32_t (&a)[32], const uint32_t (&b)[32]) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) a[k] = __float_as_uint(__uint_as_float(a[k]) + __uint_as_float(b[k]));
+      };
       if constexpr (GATE_UP) {
         // lane 4g+t: gate row j (tensor-memory lane 16*band + g) and its up row
         // (lane 16*band + 8 + g) for positions 8i + 2t, 8i + 2t + 1
-        uint32_t r0[32], r1[32];
-        tmem_ld16x256x8(dcol + ((uint32_t)(32 * q) << 16), r0);
-        tmem_ld16x256x8(dcol + ((uint32_t)(32 * q + 16) << 16), r1);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dempty(d));
         const int g = lane >> 2, t = lane & 3;
-#pragma unroll
+#pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-          const uint32_t* r = h ? r1 : r0;
+          uint32_t r[32], r1[32];
+          const uint32_t ta = dcol + ((uint32_t)(32 * q + 16 * h) << 16);
+          tmem_ld16x256x8(ta, r);
+          if (two) tmem_ld16x256x8(ta + (uint32_t)kGemmTokens, r1);
+          tmem_wait_ld();
+          if (two) sum2(r, r1);
           const int j = f.rb * 64 + (2 * q + h) * 8 + g;
           if (j >= p.ldo) continue;
 #pragma unroll
@@ -461,24 +477,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       } else {
-        // lane l of warp q: output row 128*rb + 32*q + l, 64 positions
-        uint32_t r0[32], r1[32];
-        tmem_ld32x32x32(dcol + ((uint32_t)(32 * q) << 16), r0);
-        tmem_ld32x32x32(dcol + ((uint32_t)(32 * q) << 16) + 32u, r1);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dempty(d));
+        // lane l of warp q: output row 128*rb + 32*q + l, 32 positions per pass
         const int row = f.rb * 128 + 32 * q + lane;
-        if (row < p.rows) {
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[32], r1[32];
+          const uint32_t ta = dcol + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * h);
+          tmem_ld32x32x32(ta, r);
+          if (two) tmem_ld32x32x32(ta + (uint32_t)kGemmTokens, r1);
+          tmem_wait_ld();
+          if (two) sum2(r, r1);
+          if (row < p.rows) {
 #pragma unroll
-          for (int n = 0; n < 64; ++n) {
-            if (n >= f.ntok) break;
-            const float v = __uint_as_float(n < 32 ? r0[n] : r1[n - 32]);
-            p.out[(size_t)(f.pos0 + n) * p.ldo + row] = v * p.bscale[f.pos0 + n];
+            for (int n = 0; n < 32; ++n) {
+              if (32 * h + n >= f.ntok) break;
+              p.out[(size_t)(f.pos0 + 32 * h + n) * p.ldo + row] = __uint_as_float(r[n]) * p.bscale[f.pos0 + 32 * h + n];
+            }
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dempty(d));
     }
   }
   tc_fence_before();
@@ -503,15 +523,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 template <int BITS, bool GATE_UP>
-int launch_one(const TmaDesc& w, const TmaDesc& x, const TcArgs& a, int n_sm, cudaStream_t st) {
+int launch_one(const TmaDesc& w, const TmaDesc* x, const TcArgs& a, int n_sm, cudaStream_t st) {
   using L = TcL<BITS>;
   cudaError_t e = cudaFuncSetAttribute(bt_tc_gemm_kernel<BITS, GATE_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        L::SMEM);
   if (e != cudaSuccess) return (int)e;
-  CUtensorMap wm, xm;
+  CUtensorMap wm;
+  XMaps xm;
   static_assert(sizeof(TmaDesc) == sizeof(CUtensorMap), "tensor map size");
   memcpy(&wm, w.bytes, sizeof wm);
-  memcpy(&xm, x.bytes, sizeof xm);
+  for (int k = 0; k < kTcXMaps; ++k) memcpy(&xm.m[k], x[k].bytes, sizeof(CUtensorMap));
   bt_tc_gemm_kernel<BITS, GATE_UP><<<n_sm, kTcThreads, L::SMEM, st>>>(wm, xm, a);
   return (int)cudaGetLastError();
 }
@@ -537,27 +558,31 @@ int tc_encode_weight_map(const uint8_t* matrix0, int64_t blob_bytes, int n_blobs
   return 0;
 }
 
-int tc_encode_token_map(const uint16_t* base, int cols, int rows, TmaDesc* out) {
+int tc_encode_token_maps(const uint16_t* base, int cols, int rows, TmaDesc* out) {
   auto fn = encode_fn();
   if (fn == nullptr) return (int)cudaErrorNotSupported;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64u, 16u};
-  const cuuint32_t estr[2] = {1u, 1u};
-  CUtensorMap m;
-  const CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return (int)cudaErrorInvalidValue;
-  memcpy(out->bytes, &m, sizeof m);
+  // (64 columns, rows, 64-column blocks) view of the row-major [rows][cols] matrix
+  const cuuint64_t dims[3] = {64u, (cuuint64_t)rows, (cuuint64_t)(cols / 64)};
+  const cuuint64_t strides[2] = {(cuuint64_t)cols * 2, 128u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  for (int k = 0; k < kTcXMaps; ++k) {
+    const cuuint32_t box[3] = {64u, (cuuint32_t)(16 * (k + 1)), 2u};
+    CUtensorMap m;
+    const CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return (int)cudaErrorInvalidValue;
+    memcpy(out[k].bytes, &m, sizeof m);
+  }
   return 0;
 }
 
-int launch_tc_gemm(int bits, bool gate_up, const TmaDesc& wmap, const TmaDesc& xmap, const TcArgs& a, int n_sm,
+int launch_tc_gemm(int bits, bool gate_up, const TmaDesc& wmap, const TmaDesc* xmaps, const TcArgs& a, int n_sm,
                    void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (bits == 4) return gate_up ? launch_one<4, true>(wmap, xmap, a, n_sm, st) : launch_one<4, false>(wmap, xmap, a, n_sm, st);
-  return gate_up ? launch_one<2, true>(wmap, xmap, a, n_sm, st) : launch_one<2, false>(wmap, xmap, a, n_sm, st);
+  if (bits == 4)
+    return gate_up ? launch_one<4, true>(wmap, xmaps, a, n_sm, st) : launch_one<4, false>(wmap, xmaps, a, n_sm, st);
+  return gate_up ? launch_one<2, true>(wmap, xmaps, a, n_sm, st) : launch_one<2, false>(wmap, xmaps, a, n_sm, st);
 }
 
 }  // namespace fmoe

@@ -230,7 +230,7 @@ struct BatchWs {              // device buffers, sized for max_tokens at create
   float* asc;                 // [T*(K+1)]
   float* y;                   // [T*(K+1)][H] expert outputs
   int max_items_gu, max_items_dn;
-  TmaDesc zmap, amap;         // 16 x 64 boxes of zp / ap, 128-byte swizzle
+  TmaDesc zmap[4], amap[4];   // zp / ap boxes of 16, 32, 48, 64 rows x 2 x 64 columns, 128-byte swizzle
 };
 
 struct BatchArgs {
@@ -275,9 +275,10 @@ struct TcArgs {
 // box = 2 tiles x 8 bands.
 int tc_encode_weight_map(const uint8_t* matrix0, int64_t blob_bytes, int n_blobs, int rows, int cols, int bits,
                          TmaDesc* out);
-// Tensor map over an fp16 [rows][cols] matrix, 64 x 16 boxes, 128-byte swizzle.
-int tc_encode_token_map(const uint16_t* base, int cols, int rows, TmaDesc* out);
-int launch_tc_gemm(int bits, bool gate_up, const TmaDesc& wmap, const TmaDesc& xmap, const TcArgs& a, int n_sm,
+// Four tensor maps over an fp16 [rows][cols] matrix seen as (64 columns, rows,
+// cols/64 blocks): boxes of 16, 32, 48, 64 rows x 2 blocks, 128-byte swizzle.
+int tc_encode_token_maps(const uint16_t* base, int cols, int rows, TmaDesc* out);
+int launch_tc_gemm(int bits, bool gate_up, const TmaDesc& wmap, const TmaDesc* xmaps, const TcArgs& a, int n_sm,
                    void* stream);
 int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream);
 
