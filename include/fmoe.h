@@ -57,9 +57,9 @@ typedef enum fmoe_status {
 /* fmoe_config.flags */
 #define FMOE_FLAG_FORCE_PER_TOKEN 0x1u /* T > 1: run the batch-1 kernel once per token  */
 #define FMOE_FLAG_FORCE_GROUPED 0x2u   /* T >= 1: always use the grouped batched path   */
-/* The grouped batched path needs n_experts <= 1023: with more experts a context
- * runs every token count through the batch-1 kernel, and FORCE_GROUPED makes
- * fmoe_create fail with FMOE_ERR_UNSUPPORTED. */
+/* The grouped batched path needs n_experts <= 1023 and max_tokens <= 16320:
+ * beyond either a context runs every token count through the batch-1 kernel,
+ * and FORCE_GROUPED makes fmoe_create fail with FMOE_ERR_UNSUPPORTED. */
 /* Fault injection for tests: the router step never publishes its completion,
  * so every block's bounded wait for it runs out and the call reports
  * FMOE_ERR_TIMEOUT through fmoe_poll_status (no GPU fault, no hang). */

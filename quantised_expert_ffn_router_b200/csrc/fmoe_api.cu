@@ -379,9 +379,11 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   ctx->stack_buf[0] = reinterpret_cast<uint16_t*>(base + off_stack);
   ctx->stack_buf[1] = reinterpret_cast<uint16_t*>(base + off_stack + stack_bytes);
   // batched path: sized for max_tokens, only when more than one token is allowed
-  if ((c.flags & FMOE_FLAG_FORCE_GROUPED) && c.n_experts > kBatchMaxExperts)
-    return bail(fail(ctx, FMOE_ERR_UNSUPPORTED, "grouped path: n_experts=%d above %d", c.n_experts, kBatchMaxExperts));
-  if ((c.max_tokens > 1 || (c.flags & FMOE_FLAG_FORCE_GROUPED)) && c.n_experts <= kBatchMaxExperts) {
+  const bool grouped_ok = c.n_experts <= kBatchMaxExperts && c.max_tokens <= kBatchMaxTokens;
+  if ((c.flags & FMOE_FLAG_FORCE_GROUPED) && !grouped_ok)
+    return bail(fail(ctx, FMOE_ERR_UNSUPPORTED, "grouped path: n_experts=%d (max %d), max_tokens=%d (max %d)",
+                     c.n_experts, kBatchMaxExperts, c.max_tokens, kBatchMaxTokens));
+  if ((c.max_tokens > 1 || (c.flags & FMOE_FLAG_FORCE_GROUPED)) && grouped_ok) {
     const size_t bb = batch_ws_bytes(c.hidden, c.n_experts, c.top_k, c.inter, std::max(c.max_tokens, 1));
     e = cudaMalloc(&ctx->bws_mem, bb);
     if (e != cudaSuccess) {

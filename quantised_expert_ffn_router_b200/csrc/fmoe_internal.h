@@ -194,16 +194,18 @@ inline __host__ __device__ void task_stage_of(int nstage, int n_issuers, int n_t
 }
 
 // ---------------------------------------------------------------- batched path
-// T tokens at once (fmoe_batched.cu): RMSNorm, router GEMM, top-K, a stable
+// T tokens at once (fmoe_batched.cu): RMSNorm, router GEMM, top-K, a
 // per-expert permutation of the T*(K+1) (token, slot) pairs into segments, a
-// grouped gate/up GEMM (128 rows x 64 tokens per work item, codes exact on the
-// tensor pipe, per-group scale/bias epilogue, silu(g)*u in the epilogue), a
-// grouped down GEMM, and a fixed-order combine.  Positions 0..T*K-1 hold the
-// routed pairs grouped by expert; positions T*K.. hold the shared expert.
-constexpr int kGemmRows = 128;       // rows per work item (8 warps x 16)
+// grouped gate/up GEMM on tcgen05 (fmoe_grouped_tc.cu: 128 rows x up to 64
+// positions per work item, weights dequantised to fp16 in tensor memory,
+// silu(g)*u in the epilogue), a grouped down GEMM, and a fixed-order combine.
+// Positions 0..T*K-1 hold the routed pairs grouped by expert; positions T*K..
+// hold the shared expert.
+constexpr int kGemmRows = 128;       // rows per work item (8 packed bands of 16)
 constexpr int kGemmTokens = 64;      // tokens (positions) per work item
 constexpr int kGroupedMinTokens = 8; // fmoe_layer_forward uses the batched path from this T on
 constexpr int kBatchMaxExperts = 1023;  // batched permute: one thread per expert plus the shared one
+constexpr int kBatchMaxTokens = 255 * kGemmTokens;  // token blocks per segment fit 8 bits of a work item
 
 // Opaque copy of a TMA tensor map (CUtensorMap: 128 bytes, 64-byte aligned).
 struct TmaDesc {
