@@ -306,17 +306,30 @@ def run_gpu(args, wl, ws, rank, local):
 
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    # batched: the library records these around its two grouped GEMM launches
+    # (recorded once here so that the handles exist)
+    gemm_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)] if batched else None
+    if batched:
+        for evs in gemm_ev:
+            for e in evs:
+                e.record(stream)
+        torch.cuda.synchronize()
     sampler = ClockSampler(torch.cuda.current_device())
     barrier(ws)
     torch.cuda.synchronize()
     sampler.start()
     for i in range(steps):
         maybe_flush(i)
+        if batched:
+            fm.fmoe_set_gemm_events(ctx, [e.cuda_event for e in gemm_ev[i]])
         ev0[i].record(stream)
         step(i)
         ev1[i].record(stream)
     torch.cuda.synchronize()
     barrier(ws)
+    if batched:
+        fm.fmoe_set_gemm_events(ctx, None)
+        gemm_ms = [statistics.mean(e[2 * k].elapsed_time(e[2 * k + 1]) for e in gemm_ev) for k in range(2)]
     clocks = sampler.summary()
     step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
     total_ms = max_over_ranks(ws, sum(step_ms))
@@ -369,8 +382,24 @@ def run_gpu(args, wl, ws, rank, local):
         bytes_launch = (wl.n_experts * wl.hidden * 2 + (statistics.mean(uniq) + 1) * wl.blob_bytes
                         + 2 * B * wl.hidden * 2)
         flops = 2 * B * (wl.top_k + 1) * 3 * wl.hidden * wl.inter + 2 * B * wl.hidden * wl.n_experts
+        # the grouped GEMMs, timed on the launching stream: weights of every
+        # selected expert once, inputs read and outputs written once
+        P = B * (wl.top_k + 1)
+        tb = 16 * 64 * wl.bits // 8 + 64
+        gu_w = (wl.inter // 8) * (wl.hidden // 64) * tb
+        dn_w = (wl.hidden // 16) * (wl.inter // 64) * tb
+        ne = statistics.mean(uniq) + 1
+        gu_bytes = ne * gu_w + P * wl.hidden * 2 + P * wl.inter * 4
+        dn_bytes = ne * dn_w + P * wl.inter * 2 + P * wl.hidden * 4
+        gu_flops = 2 * P * 2 * wl.inter * wl.hidden
         tensor = {"flops_per_step": flops, "achieved_tflops": flops / (ms_per_step * 1e-3) / 1e12,
-                  "unique_experts_per_step": statistics.mean(uniq)}
+                  "unique_experts_per_step": statistics.mean(uniq),
+                  "gate_up_gemm": {"kernel": f"bt_tc_gemm_kernel<{wl.bits}, true>", "us": 1e3 * gemm_ms[0],
+                                   "algorithmic_bytes": gu_bytes, "gbs": gu_bytes / (gemm_ms[0] * 1e-3) / 1e9,
+                                   "tflops": gu_flops / (gemm_ms[0] * 1e-3) / 1e12},
+                  "down_gemm": {"kernel": f"bt_tc_gemm_kernel<{wl.bits}, false>", "us": 1e3 * gemm_ms[1],
+                                "algorithmic_bytes": dn_bytes, "gbs": dn_bytes / (gemm_ms[1] * 1e-3) / 1e9,
+                                "tflops": gu_flops / 2 / (gemm_ms[1] * 1e-3) / 1e12}}
     achieved = bytes_launch / (us_layer * 1e-6) / 1e9
     peak, peak_kind = hbm_peak()
     traffic = None
@@ -389,9 +418,13 @@ def run_gpu(args, wl, ws, rank, local):
         "data": "synthetic (seeded, shaped like the pages' model; random weights)",
         "config": config_dict(wl, flushed=not stacked),
         "us_per_layer": us_layer, "hbm_gbs": achieved, "hbm_frac": achieved / peak,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "peak_source": peak_kind, "kernel": f"decode_kernel<{wl.bits}>",
-                     "algorithmic_bytes_per_launch": bytes_launch},
+        "roofline": ({"bound": "hbm", "achieved": tensor["gate_up_gemm"]["gbs"], "peak": peak, "unit": "GB/s",
+                      "frac": tensor["gate_up_gemm"]["gbs"] / peak, "traffic": traffic, "peak_source": peak_kind,
+                      "kernel": tensor["gate_up_gemm"]["kernel"],
+                      "algorithmic_bytes_per_launch": tensor["gate_up_gemm"]["algorithmic_bytes"]} if batched else
+                     {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                      "traffic": traffic, "peak_source": peak_kind, "kernel": f"decode_kernel<{wl.bits}>",
+                      "algorithmic_bytes_per_launch": bytes_launch}),
         "step_us_p10_p50_p90": [1e3 * q for q in statistics.quantiles(step_ms, n=10)[0::4]] if steps >= 10 else None,
         "warm_l2_us_per_layer": warm_us,
         "e2e": {"value": job_throughput(ws, e2e_steps * B, e2e_total), "unit": "tokens/s",

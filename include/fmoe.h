@@ -197,6 +197,19 @@ FMOE_API fmoe_status fmoe_unpack_expert(fmoe_ctx* ctx, int32_t layer, int32_t ex
  */
 FMOE_API fmoe_status fmoe_poll_status(fmoe_ctx* ctx, void* stream, uint32_t* device_status);
 
+/*
+ * Timing hook for the grouped (batched) path, for benchmarks; no counterpart on
+ * the pages.  While set, every call that takes the grouped path records
+ * events[0] / events[1] on its stream immediately before / after the grouped
+ * gate/up GEMM launch, and events[2] / events[3] around the grouped down GEMM
+ * launch, so cudaEventElapsedTime gives each GEMM's device time.  `events`
+ * points to 4 cudaEvent_t handles (passed as void*) owned by the caller and
+ * created on the context's device; the library copies the handles and never
+ * creates, synchronises or destroys them.  NULL clears the hook.  Returns
+ * FMOE_ERR_INVALID_ARG for an invalid context or a NULL handle in the array.
+ */
+FMOE_API fmoe_status fmoe_set_gemm_events(fmoe_ctx* ctx, void* const* events);
+
 /* Releases the workspace; the context pointer is invalid afterwards (later
  * calls with it return FMOE_ERR_INVALID_ARG).  Does not free caller memory. */
 FMOE_API fmoe_status fmoe_destroy(fmoe_ctx* ctx);

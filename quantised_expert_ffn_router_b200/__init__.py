@@ -29,8 +29,8 @@ FMOE_FLAG_FORCE_GROUPED = 0x2
 FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE = 0x100
 
 EXPORTED_SYMBOLS = ["fmoe_expert_bytes", "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward",
-                    "fmoe_layer_forward", "fmoe_stack_forward", "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy",
-                    "fmoe_last_error"]
+                    "fmoe_layer_forward", "fmoe_stack_forward", "fmoe_unpack_expert", "fmoe_set_gemm_events",
+                    "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error"]
 
 
 class Config(ctypes.Structure):
@@ -77,6 +77,7 @@ def lib():
             L.fmoe_stack_forward.argtypes = [P, i32, i32, P, i32, P, P]
             L.fmoe_unpack_expert.argtypes = [P, i32, i32, P, P]
             L.fmoe_poll_status.argtypes = [P, P, ctypes.POINTER(u32)]
+            L.fmoe_set_gemm_events.argtypes = [P, P]
             L.fmoe_destroy.argtypes = [P]
             L.fmoe_last_error.argtypes = [P]
             L.fmoe_last_error.restype = ctypes.c_char_p
@@ -146,6 +147,15 @@ def fmoe_stack_forward(ctx, layer_begin, layer_end, h_in_dev, T, h_out_dev, stre
 def fmoe_unpack_expert(ctx, layer, expert, dst_dev, stream=0, *, check=True) -> int:
     st = lib().fmoe_unpack_expert(_vp(ctx), layer, expert, _vp(dst_dev), _vp(stream))
     return _check(ctx, st) if check else st
+
+
+def fmoe_set_gemm_events(ctx, handles=None) -> int:
+    """Records the grouped GEMMs of later batched calls between 4 caller-owned
+    cudaEvent_t handles (ints); None clears the hook."""
+    if handles is None:
+        return lib().fmoe_set_gemm_events(_vp(ctx), None)
+    arr = (ctypes.c_void_p * 4)(*[int(h) for h in handles])
+    return lib().fmoe_set_gemm_events(_vp(ctx), arr)
 
 
 def fmoe_poll_status(ctx, stream=0):

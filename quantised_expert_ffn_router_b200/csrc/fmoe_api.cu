@@ -32,6 +32,7 @@ struct fmoe_ctx {
   void* bws_mem = nullptr;  // batched-path workspace (max_tokens > 1)
   BatchWs bws{};
   std::vector<TmaDesc> tc_maps;  // per layer: tensor maps of the packed gate/up and down matrices
+  void* gemm_events[4] = {nullptr, nullptr, nullptr, nullptr};  // caller's timing events (fmoe_set_gemm_events)
   DecodePlan plan[3];  // per mode: layer, expert, route (pointers filled per call)
   std::string err;
 };
@@ -502,6 +503,7 @@ static BatchArgs batch_args(const fmoe_ctx* ctx, int32_t layer, int32_t T) {
     a.wmap_dn = &ctx->tc_maps[2 * (size_t)layer + 1];
   }
   a.status = &ctx->hdr->status;
+  for (int k = 0; k < 4; ++k) a.gemm_events[k] = ctx->gemm_events[k];
   return a;
 }
 
@@ -662,6 +664,18 @@ fmoe_status fmoe_unpack_expert(fmoe_ctx* ctx, int32_t layer, int32_t expert, voi
   int rc = launch_repack(src, static_cast<uint8_t*>(dst_dev), 1, ctx->cfg.hidden, ctx->cfg.inter, ctx->cfg.bits, 0,
                          stream);
   if (rc != 0) return cuda_fail(ctx, (cudaError_t)rc, "unpack");
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_set_gemm_events(fmoe_ctx* ctx, void* const* events) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  if (events == nullptr) {
+    for (int k = 0; k < 4; ++k) ctx->gemm_events[k] = nullptr;
+    return FMOE_OK;
+  }
+  for (int k = 0; k < 4; ++k)
+    if (events[k] == nullptr) return fail(ctx, FMOE_ERR_INVALID_ARG, "event %d is NULL", k);
+  for (int k = 0; k < 4; ++k) ctx->gemm_events[k] = events[k];
   return FMOE_OK;
 }
 

@@ -531,8 +531,13 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   g.bscale = ws.zsc;
   g.out = ws.a;
   g.status = a.status;
+  auto mark = [&](int k) {
+    if (a.gemm_events[k]) cudaEventRecord(static_cast<cudaEvent_t>(a.gemm_events[k]), st);
+  };
+  mark(0);
   int rc = launch_tc_gemm(a.bits, true, *a.wmap_gu, ws.zmap, g, n_sm, stream);
   if (rc != 0) return rc;
+  mark(1);
   // down: B = the position's activation
   bt_prep_kernel<float><<<grid_of(positions, 8, 8 * n_sm), 256, 0, st>>>(ws.a, nullptr, positions, a.I, ws.ap, ws.asc);
   g.items = ws.items_dn;
@@ -542,8 +547,10 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   g.ldo = a.H;
   g.bscale = ws.asc;
   g.out = layer ? ws.y : a.y_out;
+  mark(2);
   rc = launch_tc_gemm(a.bits, false, *a.wmap_dn, ws.amap, g, n_sm, stream);
   if (rc != 0) return rc;
+  mark(3);
   if (layer) {
     bt_combine_kernel<<<grid_of((int64_t)a.T * a.H / 4, 256, 8 * n_sm), 256, 0, st>>>(a.h_in, ws.y, ws.pos_of, ws.w, a.T,
                                                                                   a.H, a.K, a.h_out);

@@ -252,6 +252,7 @@ struct BatchArgs {
   const TmaDesc* wmap_gu;     // tensor maps of the layer's packed gate/up and down matrices
   const TmaDesc* wmap_dn;
   uint32_t* status;           // device status word (kStatus* bits)
+  void* gemm_events[4];       // cudaEvent_t recorded around the two grouped GEMMs, or null
 };
 
 // Bytes of the batched workspace for T tokens; carves it out of `base` and
