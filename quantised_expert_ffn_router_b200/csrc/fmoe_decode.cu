@@ -411,9 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
     }
   } else if (warp == 1) {
+    misc->aflag[lane] = 0;
     if (lane < 16) {
       misc->rcnt[lane] = 0;
-      misc->aflag[lane] = 0;
       misc->slot_e[lane] = (lane == 0) ? (P.mode == kModeExpert ? P.expert_id : P.E) : 0;
       misc->slot_w[lane] = (lane == 0) ? 1.f : 0.f;
     }
@@ -754,24 +754,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           if (lane == 0) red_relaxed_add(&P.ws->h_cnt[slot], 1u);
         }
       } else {
-        // activations of this slot as fragments (built once per block)
+        // activations of this slot as fragments, built once per block in two
+        // halves of the slot's groups: the block's two down jobs of a slot
+        // usually run on two warps, which then fetch and build a half each.
         uint32_t* af = reinterpret_cast<uint32_t*>(smem + P.off_afrag + slot * P.afrag_bytes);
         float2* ai = reinterpret_cast<float2*>(smem + P.off_ainfo + slot * P.ainfo_bytes);
-        int claimed = 0;
-        if (lane == 0 && misc->aflag[slot] == 0 && atomicCAS(&misc->aflag[slot], 0, 1) == 0) claimed = 1;
-        claimed = __shfl_sync(0xffffffffu, claimed, 0);
+        const uint64_t* act = P.ws_a + (int64_t)slot * P.I;
+        const int ng = P.I / kGroup, half_g = (ng + 1) / 2;
         int good = 1;
-        if (claimed) {
+        for (int h = 0; h < 2 && good; ++h) {
+          const int gb = h * half_g, ge = min(ng, gb + half_g);
+          int* flag = &misc->aflag[2 * (int)slot + h];
+          int claimed = 0;
+          if (lane == 0 && *reinterpret_cast<volatile int*>(flag) == 0 && atomicCAS(flag, 0, 1) == 0) claimed = 1;
+          claimed = __shfl_sync(0xffffffffu, claimed, 0);
+          if (!claimed) continue;
           // The slot's activations are tagged words published by every block's
           // gate/up units.  Each lane fetches its pair (2*lane, 2*lane+1) of up
           // to kFetchGroups groups in one round trip and the round is repeated
           // until every tag is current; the published count only paces the
           // retries.  Each group then gets its own power-of-two scale and sum,
           // exactly as the input z does.
-          const uint64_t* act = P.ws_a + (int64_t)slot * P.I;
-          const int ng = P.I / kGroup;
           const uint64_t t0 = gtimer();
-          for (int g0 = 0; g0 < ng && good; g0 += kFetchGroups) {
+          for (int g0 = gb; g0 < ge && good; g0 += kFetchGroups) {
             ulonglong2 v[kFetchGroups];
             for (int attempt = 0;; ++attempt) {
               // every load is issued before any result is examined: the loads
@@ -779,11 +784,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
               // the first one's round trip before issuing the second
 #pragma unroll
               for (int k = 0; k < kFetchGroups; ++k)  // past the end: re-read the last group, ignored below
-                v[k] = ld_tagged2(act + min(g0 + k, ng - 1) * kGroup + 2 * lane);
+                v[k] = ld_tagged2(act + min(g0 + k, ge - 1) * kGroup + 2 * lane);
               bool mine = true;
 #pragma unroll
               for (int k = 0; k < kFetchGroups; ++k)
-                if (g0 + k < ng) mine = mine && tagged_tag(v[k].x) == tag && tagged_tag(v[k].y) == tag;
+                if (g0 + k < ge) mine = mine && tagged_tag(v[k].x) == tag && tagged_tag(v[k].y) == tag;
               if (__all_sync(0xffffffffu, mine)) break;
               // not all published yet: wait for the count, then fetch again
               const bool counted =
@@ -801,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
               lo[k] = tagged_value(v[k].x);
               hi[k] = tagged_value(v[k].y);
             }
-            frag_batch<kFetchGroups>(lo, hi, g0, ng, BITS, af, ai, lane);
+            frag_batch<kFetchGroups>(lo, hi, g0, ge, BITS, af, ai, lane);
           }
           if (!good && lane == 0) {
             if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
@@ -811,18 +816,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             __syncwarp();
             if (lane == 0) {
               __threadfence_block();
-              *reinterpret_cast<volatile int*>(&misc->aflag[slot]) = 2;
+              *reinterpret_cast<volatile int*>(flag) = 2;
             }
           }
-        } else {
-          if (lane == 0 && !wait_flag(&misc->aflag[slot], 2, limit, abort_flag)) {
+        }
+        // both halves ready (built here or by another warp)
+        for (int h = 0; h < 2 && good; ++h) {
+          if (h * half_g >= ng) continue;
+          if (lane == 0 && !wait_flag(&misc->aflag[2 * (int)slot + h], 2, limit, abort_flag)) {
             if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
             *abort_flag = 1;
             good = 0;
           }
           good = __shfl_sync(0xffffffffu, good, 0);
-          __threadfence_block();
         }
+        __threadfence_block();
         if (!good) break;
         const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
         const float2 acc = chunk_dot<BITS>(stage, n, af, ai, (int)c * kChunkTiles, lane);

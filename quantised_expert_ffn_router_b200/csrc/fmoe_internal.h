@@ -101,7 +101,7 @@ struct Misc {
   uint32_t tag;         // epoch + 1 of this launch
   int n_tasks;          // length of this block's task list
   int pad[13];
-  int aflag[16];        // per-slot activation fragments: 0 none, 1 building, 2 ready
+  int aflag[32];        // per (slot, half) activation fragments: 0 none, 1 building, 2 ready
   int rcnt[16];         // parts finished per router row of this block
   float rpart[16][4];   // partial logits per router row and part
   int unit_cnt[32];     // K-chunks finished per gate/up unit of this block
