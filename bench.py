@@ -39,7 +39,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_PATH = os.path.join(ROOT, "profiles", "decode_traffic.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "kernel_traffic.json")
 CSRC = os.path.join(ROOT, "quantised_expert_ffn_router_b200", "csrc")
 FALLBACK_HBM_GBS = 6650.0
 
