@@ -145,3 +145,36 @@ def test_grouped_path_is_deterministic(torch):
         m.fm.fmoe_layer_forward(m.ctx, 0, x.data_ptr(), T, a.data_ptr(), None, None, m.stream)
         m.fm.fmoe_layer_forward(m.ctx, 0, x.data_ptr(), T, b.data_ptr(), None, None, m.stream)
         assert torch.equal(a, b)
+
+
+@pytest.mark.slow
+def test_full_batched_step_sampled_tokens(torch):
+    """The batched workload at full size: 256 tokens per step through the
+    grouped path (H 4096, 512 experts with a Zipf(1.1) router skew, top-4 +
+    shared, I 1024, 4-bit).  Routing is checked for every token, the layer
+    output for a sample of 8 tokens."""
+    wl = synth.WORKLOADS["batched"]
+    T = wl.tokens
+    x = _tokens(wl, T)
+    with Model(wl) as m:
+        out = torch.empty_like(x)
+        idx = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+        m.fm.fmoe_layer_forward(m.ctx, 0, x.data_ptr(), T, out.data_ptr(), idx.data_ptr(), w.data_ptr(), m.stream)
+        torch.cuda.synchronize()
+        st, word = m.fm.fmoe_poll_status(m.ctx, m.stream)
+        assert st == 0, hex(word)
+        got, gi, gw = bf16_tensor_bits(out), idx.cpu().numpy(), w.cpu().numpy()
+        del m
+    torch.cuda.empty_cache()
+    ol = OracleLayer(wl, 0)
+    xb = bf16_tensor_bits(x)
+    for t in range(T):
+        logits = oracle.router_logits(ol.router, ol.bias, xb[t])
+        ri, rw, _ = oracle.topk(logits, wl.top_k)
+        assert list(gi[t]) == list(ri), t
+        assert np.max(np.abs(gw[t] - rw)) <= W_TOL, t
+    for t in np.random.default_rng(1).choice(T, size=8, replace=False):
+        r = ol.forward(xb[t])
+        err = rel_l2(oracle.bf16_to_f64(got[t]), oracle.bf16_to_f64(r["out"]))
+        assert err <= REL_L2_TOL, (int(t), err)

@@ -196,6 +196,56 @@ def test_full_layer_sampled_tokens(torch):
     assert worst <= REL_L2_TOL
 
 
+def _full_stack_teacher_forced(torch, wl, idx):
+    """Full-size stack, a few tokens.  fmoe_stack_forward must equal the same
+    layers chained through fmoe_layer_forward bit for bit, and every layer must
+    match the oracle applied to the GPU's own input of that layer (teacher
+    forcing; errors of earlier layers are not carried into later checks).
+    Layers whose oracle routing has a near-tie are not compared."""
+    from synth.gpu import tokens
+    T = len(idx)
+    x = tokens(wl, idx, tie_free_subseeds(wl, 0, idx))
+    with Model(wl) as m:
+        out = torch.empty_like(x)
+        m.fm.fmoe_stack_forward(m.ctx, 0, wl.n_layers, x.data_ptr(), T, out.data_ptr(), m.stream)
+        hs = [x]
+        for layer in range(wl.n_layers):
+            h = torch.empty_like(x)
+            m.fm.fmoe_layer_forward(m.ctx, layer, hs[-1].data_ptr(), T, h.data_ptr(), None, None, m.stream)
+            hs.append(h)
+        torch.cuda.synchronize()
+        st, word = m.fm.fmoe_poll_status(m.ctx, m.stream)
+        assert st == 0, hex(word)
+        got = [bf16_tensor_bits(h) for h in hs]
+        assert np.array_equal(bf16_tensor_bits(out), got[-1])
+        del m
+    torch.cuda.empty_cache()
+    checked = 0
+    for layer in range(wl.n_layers):
+        ol = OracleLayer(wl, layer)
+        for t in range(T):
+            r = ol.forward(got[layer][t])
+            if oracle.topk_gaps(r["logits"], wl.top_k) < 1e-4:
+                continue  # near-tie: the selection is not unique at this precision
+            err = rel_l2(oracle.bf16_to_f64(got[layer + 1][t]), oracle.bf16_to_f64(r["out"]))
+            assert err <= REL_L2_TOL, (layer, t, err)
+            checked += 1
+    assert checked >= wl.n_layers  # most (layer, token) pairs are compared
+
+
+@pytest.mark.slow
+def test_full_stack_4bit_teacher_forced(torch):
+    """24 layers x (H 4096, 512 experts, top-4 + shared, I 1024, 4-bit) with
+    RMSNorm between layers (about 87 GB resident), two tokens."""
+    _full_stack_teacher_forced(torch, synth.WORKLOADS["stack4"], [5, 9])
+
+
+@pytest.mark.slow
+def test_full_stack_2bit_teacher_forced(torch):
+    """60 layers of the same shape at 2 bits (about 116 GB resident), two tokens."""
+    _full_stack_teacher_forced(torch, synth.WORKLOADS["stack2"], [5, 9])
+
+
 def test_deterministic(torch):
     wl = RAGGED
     T = 3
