@@ -246,6 +246,23 @@ def test_full_stack_2bit_teacher_forced(torch):
     _full_stack_teacher_forced(torch, synth.WORKLOADS["stack2"], [5, 9])
 
 
+def test_overlapping_buffers_are_rejected(torch):
+    """h_out must not overlap h_in: rejected before any GPU work, for the layer
+    and the stack call, whole or partial overlap."""
+    wl = TINY
+    with Model(wl) as m:
+        x = torch.zeros((4, wl.hidden), dtype=torch.bfloat16, device="cuda")
+        calls = [lambda: m.fm.fmoe_layer_forward(m.ctx, 0, x.data_ptr(), 2, x.data_ptr(), None, None, m.stream),
+                 lambda: m.fm.fmoe_layer_forward(m.ctx, 0, x[0].data_ptr(), 2, x[1].data_ptr(), None, None, m.stream),
+                 lambda: m.fm.fmoe_stack_forward(m.ctx, 0, 1, x[0].data_ptr(), 2, x[1].data_ptr(), m.stream)]
+        for call in calls:
+            with pytest.raises(m.fm.FmoeError) as err:
+                call()
+            assert err.value.status == m.fm.FMOE_ERR_INVALID_ARG
+            assert "overlaps" in str(err.value)
+        m.fm.fmoe_layer_forward(m.ctx, 0, x[0].data_ptr(), 2, x[2].data_ptr(), None, None, m.stream)  # disjoint: fine
+
+
 def test_deterministic(torch):
     wl = RAGGED
     T = 3
