@@ -63,6 +63,7 @@ def lib():
             L.orc_topk.argtypes = [P, i32, i32, P, P, P]
             L.orc_expert.argtypes = [P, i32, i32, i32, P, P, P, P, P]
             L.orc_combine.argtypes = [P, P, P, P, i32, i32, P, P]
+            L.orc_requant_4to2.argtypes = [P, i32, i32, P]
             _lib = L
     return _lib
 
@@ -171,6 +172,14 @@ def layer_forward(h, *, router_w, router_bias, norm_w, eps, top_k, hidden, inter
     y_sh = expert(blob_of(E), hidden, inter, bits, z)[0]
     out64, out = combine(h, w, ys, y_sh)
     return dict(z=z, logits=logits, idx=idx, w=w, y=ys, y_shared=y_sh, out_f64=out64, out=out)
+
+
+def requant_4to2(blob: np.ndarray, hidden: int, inter: int) -> np.ndarray:
+    """Canonical 2-bit blob refitted from a canonical 4-bit blob (orc_requant_4to2)."""
+    blob = _c(blob, np.uint8)
+    out = np.zeros(blob_bytes(hidden, inter, 2), dtype=np.uint8)
+    lib().orc_requant_4to2(_ptr(blob), hidden, inter, _ptr(out))
+    return out
 
 
 def topk_gaps(logits: np.ndarray, k: int) -> float:

@@ -210,3 +210,76 @@ void orc_combine(const uint16_t* h, const double* w, const double* y_routed, con
     if (out) out[j] = orc_round_bf16(s);
   }
 }
+
+/* 4-bit -> 2-bit requantisation of one canonical expert blob.  The page
+ * "Flash-MoE Inference Engine", section "Weight Preparation" (step 3, optional
+ * 2-bit requantisation), converts the 4-bit expert files to 2-bit with a script
+ * but gives no algorithm.  Reading taken: every 64-column group of every row is
+ * refitted on its own with an affine grid spanning the group's smallest and
+ * largest dequantised weight, each step one IEEE fp32 operation rounded to
+ * nearest even (so that the integer codes are decided with the same arithmetic
+ * by any implementation):
+ *   w_c  = fmaf(q4_c, s4, b4)          s4, b4: the group's bf16 scale and bias
+ *   lo   = min_c w_c,  hi = max_c w_c
+ *   s2   = bf16((hi - lo) / 3)
+ *   b2   = bf16(lo)
+ *   inv  = s2 > 0 ? 1 / s2 : 0
+ *   q2_c = min(max(rint((w_c - b2) * inv), 0), 3)
+ * The output is the canonical 2-bit blob of the same matrices. */
+void orc_requant_4to2(const uint8_t* src, int hidden, int inter, uint8_t* dst) {
+  int64_t in_off = 0, out_off = 0;
+  for (int m = 0; m < 3; ++m) {
+    int64_t R, C;
+    matrix_shape(hidden, inter, m, &R, &C);
+    const int64_t ng = C / GROUP;
+    const uint8_t* in_codes = src + in_off;
+    const uint8_t* in_s = in_codes + R * C / 2;
+    const uint8_t* in_b = in_s + 2 * R * ng;
+    uint8_t* out_codes = dst + out_off;
+    uint8_t* out_s = out_codes + R * C / 4;
+    uint8_t* out_b = out_s + 2 * R * ng;
+    for (int64_t r = 0; r < R; ++r) {
+      for (int64_t g = 0; g < ng; ++g) {
+        uint16_t s16, b16;
+        memcpy(&s16, in_s + 2 * (r * ng + g), 2);
+        memcpy(&b16, in_b + 2 * (r * ng + g), 2);
+        const float s4 = (float)orc_bf16_value(s16), b4 = (float)orc_bf16_value(b16);
+        float w[GROUP];
+        for (int c = 0; c < GROUP; ++c) {
+          const int64_t col = g * GROUP + c;
+          uint32_t word;
+          memcpy(&word, in_codes + 4 * ((r * C + col) / 8), 4);
+          const uint32_t q = (word >> (4 * (col % 8))) & 15u;
+          w[c] = fmaf((float)q, s4, b4);
+        }
+        float lo = w[0], hi = w[0];
+        for (int c = 1; c < GROUP; ++c) {
+          if (w[c] < lo) lo = w[c];
+          if (w[c] > hi) hi = w[c];
+        }
+        const float span = hi - lo;
+        const float third = span / 3.0f;
+        const uint16_t s2b = orc_round_bf16((double)third);
+        const uint16_t b2b = orc_round_bf16((double)lo);
+        const float s2 = (float)orc_bf16_value(s2b), b2 = (float)orc_bf16_value(b2b);
+        const float inv = s2 > 0.0f ? 1.0f / s2 : 0.0f;
+        memcpy(out_s + 2 * (r * ng + g), &s2b, 2);
+        memcpy(out_b + 2 * (r * ng + g), &b2b, 2);
+        for (int c = 0; c < GROUP; c += 16) {
+          uint32_t word = 0;
+          for (int k = 0; k < 16; ++k) {
+            const float d = w[c + k] - b2;
+            const float t = d * inv;
+            float qf = rintf(t);
+            if (qf < 0.0f) qf = 0.0f;
+            if (qf > 3.0f) qf = 3.0f;
+            word |= (uint32_t)qf << (2 * k);
+          }
+          memcpy(out_codes + 4 * ((r * C + g * GROUP + c) / 16), &word, 4);
+        }
+      }
+    }
+    in_off += matrix_bytes(hidden, inter, 4, m);
+    out_off += matrix_bytes(hidden, inter, 2, m);
+  }
+}

@@ -38,6 +38,9 @@ uint16_t orc_round_bf16(double v);
 int64_t orc_blob_bytes(int hidden, int inter, int bits);
 /* Dequantised weight of matrix m (0 gate [I][H], 1 up [I][H], 2 down [H][I]). */
 double orc_weight(const uint8_t* blob, int hidden, int inter, int bits, int m, int r, int c);
+/* 4-bit -> 2-bit requantisation of one canonical expert blob: per 64-group an
+ * affine min/max refit decided in IEEE fp32 (steps at the definition). */
+void orc_requant_4to2(const uint8_t* src, int hidden, int inter, uint8_t* dst);
 /* z = bf16(h / sqrt(mean(h^2) + eps) * w); w may be NULL (treated as 1). */
 void orc_rmsnorm(const uint16_t* h, const uint16_t* w, int hidden, double eps, uint16_t* z);
 /* Router logits, fp32-rounded: logits[e] = fp32(sum_h Wr[e][h] z[h] + bias[e]). */

@@ -291,3 +291,65 @@ def test_round_bf16_ties_to_even():
     assert oracle.round_bf16(1.0 + 2.0**-8 + 2.0**-30) == 0x3F81
     assert oracle.round_bf16(-65.59384201648058) == 0xC283        # -65.5
     assert oracle.bf16_value(0x3F81) == 1.0078125
+
+
+# ---------------------------------------------------------------- 4-bit -> 2-bit requantisation
+
+def _two_bit_grid_blob(H, I, rng):
+    """A 2-bit blob whose every group holds codes 0 and 3 (so the group spans the
+    whole grid), scale 5 * 2^-6, and an exact bf16 bias per row; and its 4-bit
+    expansion q4 = 5 * q2 with scale 2^-6 and the same bias (the same weights)."""
+    mats2, mats4 = [], []
+    for R, C in ((I, H), (I, H), (H, I)):
+        q2 = rng.integers(0, 4, size=(R, C))
+        q2[:, 0::64] = 0
+        q2[:, 1::64] = 3
+        bias = ((np.arange(R) % 5) - 2.0)[:, None] * 2.0 ** -5
+        mats2.append((q2, 5 * 2.0 ** -6, bias))
+        mats4.append((5 * q2, 2.0 ** -6, bias))
+    return make_blob(H, I, 2, *mats2), make_blob(H, I, 4, *mats4)
+
+
+def test_requant_recovers_an_exact_two_bit_grid():
+    rng = np.random.default_rng(3)
+    H, I = 256, 128
+    b2, b4 = _two_bit_grid_blob(H, I, rng)
+    assert np.array_equal(oracle.requant_4to2(b4, H, I), b2)
+
+
+def test_requant_constant_group_keeps_its_value():
+    H, I = 128, 64
+    # every weight 7 * 2^-5 + 2^-4 = 0.28125 (exact in bf16)
+    b4 = make_blob(H, I, 4, (7, 2.0 ** -5, 2.0 ** -4), (7, 2.0 ** -5, 2.0 ** -4), (7, 2.0 ** -5, 2.0 ** -4))
+    out = oracle.requant_4to2(b4, H, I)
+    for m, (R, C) in enumerate(((I, H), (I, H), (H, I))):
+        for r, c in ((0, 0), (R - 1, C - 1), (R // 2, 65 % C)):
+            assert oracle.weight(out, H, I, 2, m, r, c) == 0.28125
+    two = make_blob(H, I, 2, (0, 0.0, 0.28125), (0, 0.0, 0.28125), (0, 0.0, 0.28125))
+    assert np.array_equal(out, two)
+
+
+def test_requant_error_bound_and_monotone_codes():
+    wl = synth.WORKLOADS["tiny"]
+    H, I = wl.hidden, wl.inter
+    src = synth.expert_blob(wl, 0, 3)
+    out = oracle.requant_4to2(src, H, I)
+    assert out.size == oracle.blob_bytes(H, I, 2)
+    for m, (R, C) in enumerate(((I, H), (I, H), (H, I))):
+        for r in (0, 1, R - 1):
+            for g in range(C // 64):
+                cols = range(64 * g, 64 * g + 64)
+                w4 = np.array([oracle.weight(src, H, I, 4, m, r, c) for c in cols])
+                w2 = np.array([oracle.weight(out, H, I, 2, m, r, c) for c in cols])
+                lo, hi = w4.min(), w4.max()
+                s2 = (w2.max() - w2.min()) / 3 if w2.max() > w2.min() else 0.0
+                step = (hi - lo) / 3
+                bound = 0.5 * step * (1 + 2.0 ** -7) + 2.0 ** -8 * (abs(lo) + (hi - lo)) + 1e-12
+                assert np.max(np.abs(w2 - w4)) <= bound, (m, r, g)
+                order = np.argsort(w4, kind="stable")
+                assert np.all(np.diff(w2[order]) >= 0), (m, r, g)  # codes follow the weights
+                assert s2 <= step * (1 + 2.0 ** -8) + 1e-12
+
+
+def test_requant_full_shape_size():
+    assert oracle.blob_bytes(4096, 1024, 2) == 3_932_160
