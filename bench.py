@@ -443,17 +443,71 @@ def run_gpu(args, wl, ws, rank, local):
     return 0
 
 
+# fp32/integer operations per weight of the requantisation kernel: code
+# extraction, int-to-float and fma in both passes, min/max, subtract, multiply,
+# round, clamp and packing
+REQUANT_OPS_PER_WEIGHT = 16
+
+
+def run_requant(args):
+    """4-bit -> 2-bit requantisation of one full layer's 513 expert blobs
+    (H 4096, I 1024), timed with CUDA events; one GPU."""
+    import torch
+
+    import quantised_expert_ffn_router_b200 as fm
+    from synth.gpu import DeviceLayer
+    wl = synth.WORKLOADS["layer"]
+    stream = torch.cuda.current_stream()
+    layer = DeviceLayer(wl, 0, stream.cuda_stream)
+    n = wl.n_experts + 1
+    out = torch.empty(n * fm.fmoe_expert_bytes(wl.hidden, wl.inter, 2), dtype=torch.uint8, device="cuda")
+    steps = args.steps or 20
+    for _ in range(max(args.warmup, 3)):
+        fm.fmoe_requant_4to2(layer.experts.data_ptr(), n, wl.hidden, wl.inter, out.data_ptr(), stream.cuda_stream)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    for a, b in evs:
+        a.record(stream)
+        fm.fmoe_requant_4to2(layer.experts.data_ptr(), n, wl.hidden, wl.inter, out.data_ptr(), stream.cuda_stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.summary()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    in_bytes = n * wl.blob_bytes
+    out_bytes = out.numel()
+    gbs = (in_bytes + out_bytes) / (ms * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+    weights = n * 3 * wl.hidden * wl.inter
+    # issue peak: 148 SMs x 128 lanes x the SM clock seen
+    alu_peak = 148 * 128 * (clocks.get("sm_mhz") or 1965) * 1e6 / 1e12
+    alu = weights * REQUANT_OPS_PER_WEIGHT / (ms * 1e-3) / 1e12
+    line = {"metric": "4-bit -> 2-bit expert requantisation (one full layer, 513 blobs)", "value": gbs,
+            "unit": "GB/s (bytes read + written)", "n_gpus": 1, "steps": steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
+            "data": "synthetic (seeded)", "config": {"workload": "requant", "shape": "H4096 I1024 513 blobs"},
+            "roofline": {"bound": "alu", "achieved": alu, "peak": alu_peak, "unit": "T ops/s", "frac": alu / alu_peak,
+                         "ops_per_weight": REQUANT_OPS_PER_WEIGHT, "hbm_gbs": gbs, "hbm_frac": gbs / peak,
+                         "hbm_peak_source": peak_kind},
+            "gpu_launches": steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer", "stack4", "stack2", "tiny", "batched"], default="layer")
+    ap.add_argument("--workload", choices=["layer", "stack4", "stack2", "tiny", "batched", "requant"], default="layer")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
+    if args.workload == "requant":
+        return run_requant(args)
     wl = synth.WORKLOADS[args.workload]
     if args.steps is None:
         args.steps = {"layer": 3000, "stack4": 256, "stack2": 256, "tiny": 1000, "batched": 100}[args.workload]

@@ -198,6 +198,28 @@ FMOE_API fmoe_status fmoe_unpack_expert(fmoe_ctx* ctx, int32_t layer, int32_t ex
 FMOE_API fmoe_status fmoe_poll_status(fmoe_ctx* ctx, void* stream, uint32_t* device_status);
 
 /*
+ * 4-bit -> 2-bit requantisation of canonical expert blobs: the conversion of
+ * the page "Flash-MoE Inference Engine", section "Weight Preparation" (step 3,
+ * optional 2-bit requantisation), which names the step but not its algorithm.
+ * Every 64-column group of every row of gate, up and down is refitted on its
+ * own with an affine grid spanning the group's smallest and largest weight,
+ * each step one IEEE fp32 operation rounded to nearest even:
+ *   w = fma(q4, s4, b4); lo, hi = min, max of the group's w;
+ *   s2 = bf16((hi - lo) / 3); b2 = bf16(lo); inv = s2 > 0 ? 1 / s2 : 0;
+ *   q2 = min(max(rint((w - b2) * inv), 0), 3).
+ *   src_dev : n_blobs contiguous canonical 4-bit blobs (fmoe_expert_bytes(H, I, 4)
+ *             bytes each), device memory, read only;
+ *   dst_dev : n_blobs contiguous canonical 2-bit blobs (fmoe_expert_bytes(H, I, 2)
+ *             bytes each), device memory, written; must not overlap src_dev.
+ * Needs no context; asynchronous on `stream` (a cudaStream_t as void*).  Both
+ * pointers 16-byte aligned, H and I positive multiples of 64.  Errors
+ * (INVALID_ARG, ALIGNMENT, UNSUPPORTED for H*I > 2^30, CUDA) are reported before
+ * any GPU work where possible, with detail in fmoe_last_error(NULL).
+ */
+FMOE_API fmoe_status fmoe_requant_4to2(const void* src_dev, int32_t n_blobs, int32_t hidden, int32_t inter,
+                                       void* dst_dev, void* stream);
+
+/*
  * Timing hook for the grouped (batched) path, for benchmarks; no counterpart on
  * the pages.  While set, every call that takes the grouped path records
  * events[0] / events[1] on its stream immediately before / after the grouped

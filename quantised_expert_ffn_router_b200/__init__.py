@@ -29,7 +29,7 @@ FMOE_FLAG_FORCE_GROUPED = 0x2
 FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE = 0x100
 
 EXPORTED_SYMBOLS = ["fmoe_expert_bytes", "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward",
-                    "fmoe_layer_forward", "fmoe_stack_forward", "fmoe_unpack_expert", "fmoe_set_gemm_events",
+                    "fmoe_layer_forward", "fmoe_stack_forward", "fmoe_unpack_expert", "fmoe_requant_4to2", "fmoe_set_gemm_events",
                     "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error"]
 
 
@@ -78,6 +78,7 @@ def lib():
             L.fmoe_unpack_expert.argtypes = [P, i32, i32, P, P]
             L.fmoe_poll_status.argtypes = [P, P, ctypes.POINTER(u32)]
             L.fmoe_set_gemm_events.argtypes = [P, P]
+            L.fmoe_requant_4to2.argtypes = [P, i32, i32, i32, P, P]
             L.fmoe_destroy.argtypes = [P]
             L.fmoe_last_error.argtypes = [P]
             L.fmoe_last_error.restype = ctypes.c_char_p
@@ -147,6 +148,11 @@ def fmoe_stack_forward(ctx, layer_begin, layer_end, h_in_dev, T, h_out_dev, stre
 def fmoe_unpack_expert(ctx, layer, expert, dst_dev, stream=0, *, check=True) -> int:
     st = lib().fmoe_unpack_expert(_vp(ctx), layer, expert, _vp(dst_dev), _vp(stream))
     return _check(ctx, st) if check else st
+
+
+def fmoe_requant_4to2(src_ptr, n_blobs: int, hidden: int, inter: int, dst_ptr, stream=0) -> int:
+    """Canonical 4-bit blobs at src_ptr -> canonical 2-bit blobs at dst_ptr."""
+    return _check(None, lib().fmoe_requant_4to2(_vp(src_ptr), n_blobs, hidden, inter, _vp(dst_ptr), _vp(stream)))
 
 
 def fmoe_set_gemm_events(ctx, handles=None) -> int:

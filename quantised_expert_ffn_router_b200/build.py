@@ -9,7 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libfmoe.so")
-SOURCES = ["fmoe_api.cu", "fmoe_decode.cu", "fmoe_repack.cu", "fmoe_static.cu", "fmoe_batched.cu", "fmoe_grouped_tc.cu"]
+SOURCES = ["fmoe_api.cu", "fmoe_decode.cu", "fmoe_repack.cu", "fmoe_static.cu", "fmoe_batched.cu", "fmoe_grouped_tc.cu",
+           "fmoe_requant.cu"]
 HEADERS = ["fmoe_internal.h"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]

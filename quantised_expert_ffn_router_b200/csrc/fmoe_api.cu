@@ -667,6 +667,33 @@ fmoe_status fmoe_unpack_expert(fmoe_ctx* ctx, int32_t layer, int32_t expert, voi
   return FMOE_OK;
 }
 
+fmoe_status fmoe_requant_4to2(const void* src_dev, int32_t n_blobs, int32_t hidden, int32_t inter, void* dst_dev,
+                              void* stream) {
+  if (n_blobs < 0) return fail(nullptr, FMOE_ERR_INVALID_ARG, "n_blobs=%d", n_blobs);
+  if (hidden <= 0 || hidden % kGroup || inter <= 0 || inter % kGroup)
+    return fail(nullptr, FMOE_ERR_INVALID_ARG, "hidden=%d / inter=%d must be positive multiples of 64", hidden, inter);
+  if ((int64_t)hidden * inter > (int64_t)1 << 30)
+    return fail(nullptr, FMOE_ERR_UNSUPPORTED, "hidden*inter=%lld above 2^30", (long long)hidden * inter);
+  if (n_blobs == 0) return FMOE_OK;
+  if (!src_dev || !dst_dev) return fail(nullptr, FMOE_ERR_INVALID_ARG, "NULL blob pointer");
+  if (misaligned(src_dev) || misaligned(dst_dev)) return fail(nullptr, FMOE_ERR_ALIGNMENT, "blobs not 16-byte aligned");
+  const size_t in_bytes = (size_t)n_blobs * (size_t)expert_bytes(hidden, inter, 4);
+  const size_t out_bytes = (size_t)n_blobs * (size_t)expert_bytes(hidden, inter, 2);
+  if (overlaps(src_dev, in_bytes, dst_dev, out_bytes))
+    return fail(nullptr, FMOE_ERR_INVALID_ARG, "destination overlaps the source blobs");
+  int dev = 0, n_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return fail(nullptr, FMOE_ERR_CUDA, "device query: %s", cudaGetErrorString(e));
+  const int rc = launch_requant(static_cast<const uint8_t*>(src_dev), static_cast<uint8_t*>(dst_dev), n_blobs, hidden,
+                                inter, n_sm, stream);
+  if (rc != 0) {
+    cudaGetLastError();
+    return fail(nullptr, FMOE_ERR_CUDA, "requant launch: %s", cudaGetErrorString((cudaError_t)rc));
+  }
+  return FMOE_OK;
+}
+
 fmoe_status fmoe_set_gemm_events(fmoe_ctx* ctx, void* const* events) {
   if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
   if (events == nullptr) {

@@ -61,7 +61,6 @@ namespace {
 
 constexpr int kTcWarps = 15;
 constexpr int kTcThreads = kTcWarps * 32;
-constexpr int kTcChunk = 128;                     // K columns per ring stage (2 tiles)
 constexpr int kTcBBytes = 2 * kGemmTokens * 128;  // X in a stage: 2 halves x up to 64 rows x 128 B (16 KB)
 constexpr int kTcABufs = 4;                       // A buffers in tensor memory (64 columns each)
 constexpr int kTcXMaps = kGemmTokens / 16;          // input tensor maps, one per box height

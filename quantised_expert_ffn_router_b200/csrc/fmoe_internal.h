@@ -299,6 +299,8 @@ int launch_decode(const DecodePlan& plan, void* stream, bool cooperative, bool p
 // a cudaError_t value.
 int launch_route_static(const uint16_t* wr, const float* bias, const uint16_t* norm_w, float eps,
                         const uint16_t* x, int T, int H, int E, int K, int32_t* idx_out, float* w_out, void* stream);
+// 4-bit -> 2-bit requantisation of n canonical blobs (fmoe_requant.cu).
+int launch_requant(const uint8_t* src, uint8_t* dst, int n_blobs, int H, int I, int n_sm, void* stream);
 int decode_max_smem_optin(int device);
 int decode_occupancy(int bits, int smem_bytes, int* blocks_per_sm);
 int zero_workspace(void* ws, size_t bytes, void* stream);
