@@ -64,7 +64,7 @@ int64_t orc_blob_bytes(int hidden, int inter, int bits) {
  * 64 consecutive columns of a row ("Flash-MoE: Running a 400 Billion Parameter Model on a MacBook",
  * section "The Architecture": the inner
  * loop dequantises with fused multiply-adds; the affine form, group size and
- * dtypes are the readings fixed for this build).  Code c of row r is field c % (32/bits) of little-endian 32-bit
+ * dtypes are readings taken where the pages are silent).  Code c of row r is field c % (32/bits) of little-endian 32-bit
  * word c / (32/bits) of that row. */
 double orc_weight(const uint8_t* blob, int hidden, int inter, int bits, int m, int r, int c) {
   int64_t off = 0;
@@ -89,7 +89,7 @@ double orc_weight(const uint8_t* blob, int hidden, int inter, int bits, int m, i
 /* RMSNorm ahead of the mixture-of-experts block (the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on a Laptop",
  * section "How the SSD expert streaming pipeline works":
  * the second command buffer normalises before it routes; the epsilon is the
- * build's reading). */
+ * reading taken where the pages are silent). */
 void orc_rmsnorm(const uint16_t* h, const uint16_t* w, int hidden, double eps, uint16_t* z) {
   double ss = 0.0;
   for (int i = 0; i < hidden; ++i) {
@@ -133,7 +133,7 @@ static int by_prob_desc(const void* a, const void* b) {
  * section "How the SSD expert streaming pipeline works":
  * the host takes the softmax and picks the top K; the themata summary "Flash-MoE: Running a 397B Parameter Model on a Laptop",
  * Key Takeaways: K = 4).
- * Renormalising the K selected probabilities is the build's reading. */
+ * Renormalising the K selected probabilities is a reading taken where the pages are silent. */
 void orc_topk(const float* logits, int n_experts, int top_k, int32_t* idx, double* w, double* p) {
   double mx = -INFINITY;
   for (int e = 0; e < n_experts; ++e) mx = fmax(mx, (double)logits[e]);
@@ -163,7 +163,7 @@ void orc_topk(const float* logits, int n_experts, int top_k, int32_t* idx, doubl
  * the third command buffer runs the experts; "Flash-MoE: Running a 400 Billion Parameter Model on a MacBook",
  * section "The Architecture":
  * dequantisation fused into the multiply-adds).  silu(t) = t/(1+e^-t) applied
- * to the gate projection, times the up projection, is the build's reading of
+ * to the gate projection, times the up projection, is the reading taken of
  * the activation. */
 void orc_expert(const uint8_t* blob, int hidden, int inter, int bits, const uint16_t* z, double* g, double* u,
                 double* a, double* y) {
