@@ -270,14 +270,17 @@ def run_gpu(args, wl, ws, rank, local):
     descs = [fm.LayerDesc(**d) for d in weights.descs()]
     batched = wl.name == "batched"
     B = wl.tokens if batched else 1          # tokens per step
-    cfg = fm.Config(wl.hidden, wl.n_experts, wl.top_k, wl.inter, wl.bits, 64, wl.n_layers, B, wl.rms_eps, 0, 0)
+    L = wl.n_layers
+    stacked = L > 1
+    # stacks: one launch per token through every layer, or (--stack-per-layer) one per layer
+    per_layer = stacked and args.stack_per_layer
+    flags = fm.FMOE_FLAG_STACK_PER_LAYER if per_layer else 0
+    cfg = fm.Config(wl.hidden, wl.n_experts, wl.top_k, wl.inter, wl.bits, 64, wl.n_layers, B, wl.rms_eps, flags, 0)
     _, ctx = fm.fmoe_create(cfg, descs, sp)
     n_batches = wl.steps if batched else wl.tokens   # distinct inputs cycled through
     X = tokens(wl, range(n_batches * B)).view(n_batches, B, wl.hidden)
     OUT = torch.empty_like(X)
     IDX = torch.zeros((n_batches, B, wl.top_k), dtype=torch.int32, device="cuda")
-    L = wl.n_layers
-    stacked = L > 1
 
     def step(i, x_ptr=None, out_ptr=None):
         x_ptr = X[i % n_batches].data_ptr() if x_ptr is None else x_ptr
@@ -416,20 +419,23 @@ def run_gpu(args, wl, ws, rank, local):
         "vs_baseline": None, "dtype": ("fp16 dequantised weights x fp16 inputs on tcgen05, fp32 accumulate (bf16 I/O)"
                                        if batched else "fp16 tensor-core MAC of exact integer codes, fp32 accumulate (bf16 I/O)"),
         "data": "synthetic (seeded, shaped like the pages' model; random weights)",
-        "config": config_dict(wl, flushed=not stacked),
+        "config": {**config_dict(wl, flushed=not stacked),
+                   **({"launch": "one per layer" if per_layer else "one per token through every layer"}
+                      if stacked else {})},
         "us_per_layer": us_layer, "hbm_gbs": achieved, "hbm_frac": achieved / peak,
         "roofline": ({"bound": "hbm", "achieved": tensor["gate_up_gemm"]["gbs"], "peak": peak, "unit": "GB/s",
                       "frac": tensor["gate_up_gemm"]["gbs"] / peak, "traffic": traffic, "peak_source": peak_kind,
                       "kernel": tensor["gate_up_gemm"]["kernel"],
                       "algorithmic_bytes_per_launch": tensor["gate_up_gemm"]["algorithmic_bytes"]} if batched else
                      {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                      "traffic": traffic, "peak_source": peak_kind, "kernel": f"decode_kernel<{wl.bits}>",
+                      "traffic": traffic, "peak_source": peak_kind,
+                      "kernel": f"decode_kernel<{wl.bits}, {'true' if stacked and not per_layer else 'false'}>",
                       "algorithmic_bytes_per_launch": bytes_launch}),
         "step_us_p10_p50_p90": [1e3 * q for q in statistics.quantiles(step_ms, n=10)[0::4]] if steps >= 10 else None,
         "warm_l2_us_per_layer": warm_us,
         "e2e": {"value": job_throughput(ws, e2e_steps * B, e2e_total), "unit": "tokens/s",
                 "h2d_bytes_per_step": B * wl.hidden * 2, "d2h_bytes_per_step": B * wl.hidden * 2},
-        "gpu_launches": steps * (BATCHED_LAUNCHES if batched else L),
+        "gpu_launches": steps * (BATCHED_LAUNCHES if batched else (L if per_layer or not stacked else 1)),
         "clocks": clocks,
     }
     if tensor is not None:
@@ -505,6 +511,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stack-per-layer", action="store_true",
+                    help="stacks: one launch per layer instead of one per token (the multi-layer kernel)")
     args = ap.parse_args(argv)
     if args.workload == "requant":
         return run_requant(args)

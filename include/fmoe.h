@@ -57,6 +57,9 @@ typedef enum fmoe_status {
 /* fmoe_config.flags */
 #define FMOE_FLAG_FORCE_PER_TOKEN 0x1u /* T > 1: run the batch-1 kernel once per token  */
 #define FMOE_FLAG_FORCE_GROUPED 0x2u   /* T >= 1: always use the grouped batched path   */
+/* fmoe_stack_forward on the batch-1 kernel: one launch per layer and token
+ * instead of one launch per token running every layer of the range. */
+#define FMOE_FLAG_STACK_PER_LAYER 0x4u
 /* The grouped batched path needs n_experts <= 1023 and max_tokens <= 16320:
  * beyond either a context runs every token count through the batch-1 kernel,
  * and FORCE_GROUPED makes fmoe_create fail with FMOE_ERR_UNSUPPORTED. */

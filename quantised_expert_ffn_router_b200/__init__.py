@@ -16,7 +16,7 @@ from . import build as _build
 
 __all__ = [
     "FMOE_OK", "FMOE_ERR_INVALID_ARG", "FMOE_ERR_UNSUPPORTED", "FMOE_ERR_ALIGNMENT", "FMOE_ERR_CUDA",
-    "FMOE_ERR_OOM", "FMOE_ERR_TIMEOUT", "FMOE_FLAG_FORCE_PER_TOKEN", "FMOE_FLAG_FORCE_GROUPED",
+    "FMOE_ERR_OOM", "FMOE_ERR_TIMEOUT", "FMOE_FLAG_FORCE_PER_TOKEN", "FMOE_FLAG_FORCE_GROUPED", "FMOE_FLAG_STACK_PER_LAYER",
     "FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE", "Config", "LayerDesc", "FmoeError", "lib", "fmoe_expert_bytes",
     "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward", "fmoe_layer_forward", "fmoe_stack_forward",
     "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error", "EXPORTED_SYMBOLS",
@@ -26,6 +26,7 @@ FMOE_OK, FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED, FMOE_ERR_ALIGNMENT = 0, 1, 
 FMOE_ERR_CUDA, FMOE_ERR_OOM, FMOE_ERR_TIMEOUT = 4, 5, 6
 FMOE_FLAG_FORCE_PER_TOKEN = 0x1
 FMOE_FLAG_FORCE_GROUPED = 0x2
+FMOE_FLAG_STACK_PER_LAYER = 0x4
 FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE = 0x100
 
 EXPORTED_SYMBOLS = ["fmoe_expert_bytes", "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward",

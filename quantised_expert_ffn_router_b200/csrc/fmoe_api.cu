@@ -29,6 +29,7 @@ struct fmoe_ctx {
   uint32_t* tasks = nullptr;   // device [3 modes][grid][kMaxTasks]
   int32_t* ntasks = nullptr;   // device [3 modes][grid]
   uint16_t* stack_buf[2] = {nullptr, nullptr};  // ping-pong activations, [max_tokens][H] bf16
+  LayerDev* layer_dev = nullptr;                // device [n_layers]: weights of every layer (multi-layer launches)
   void* bws_mem = nullptr;  // batched-path workspace (max_tokens > 1)
   BatchWs bws{};
   std::vector<TmaDesc> tc_maps;  // per layer: tensor maps of the packed gate/up and down matrices
@@ -344,14 +345,15 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   const int max_smem = decode_max_smem_optin(ctx->device);
   if (!plan_all(ctx, max_smem))
     return bail(fail(ctx, FMOE_ERR_UNSUPPORTED, "shared-memory plan does not fit (%d bytes available)", max_smem));
-  for (int m = 0; m < 3; ++m) {
+  for (int m = 0; m < 4; ++m) {  // three single-layer plans, then the multi-layer kernel with the layer plan
     int blocks = 0;
-    int rc = decode_occupancy(c.bits, (int)ctx->plan[m].smem_bytes, &blocks);
+    int rc = decode_occupancy(c.bits, m == 3, (int)ctx->plan[m == 3 ? kModeLayer : m].smem_bytes, &blocks);
     if (rc != 0) return bail(cuda_fail(ctx, (cudaError_t)rc, "occupancy query"));
     if (blocks < 1) return bail(fail(ctx, FMOE_ERR_UNSUPPORTED, "fused kernel cannot be resident"));
   }
 
-  // workspace: header | logits [E] | activations [kMaxSlots][I] | task lists | 2 x [max_tokens][H] bf16
+  // workspace: header | logits [E] | activations [kMaxSlots][I] | task lists | 2 x [max_tokens][H] bf16 |
+  // per-layer weight table
   size_t off = 256;
   size_t off_logits = off;
   off += ((size_t)c.n_experts * 8 + 255) / 256 * 256;
@@ -364,6 +366,8 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   size_t off_stack = off;
   size_t stack_bytes = ((size_t)std::max(c.max_tokens, 1) * c.hidden * 2 + 255) / 256 * 256;
   off += 2 * stack_bytes;
+  size_t off_layers = off;
+  off += ((size_t)c.n_layers * sizeof(LayerDev) + 255) / 256 * 256;
   ctx->ws_bytes = off;
   e = cudaMalloc(&ctx->ws, ctx->ws_bytes);
   if (e != cudaSuccess) {
@@ -379,6 +383,7 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   ctx->ntasks = reinterpret_cast<int32_t*>(base + off_ntasks);
   ctx->stack_buf[0] = reinterpret_cast<uint16_t*>(base + off_stack);
   ctx->stack_buf[1] = reinterpret_cast<uint16_t*>(base + off_stack + stack_bytes);
+  ctx->layer_dev = reinterpret_cast<LayerDev*>(base + off_layers);
   // batched path: sized for max_tokens, only when more than one token is allowed
   const bool grouped_ok = c.n_experts <= kBatchMaxExperts && c.max_tokens <= kBatchMaxTokens;
   if ((c.flags & FMOE_FLAG_FORCE_GROUPED) && !grouped_ok)
@@ -419,8 +424,16 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
       for (int b = 0; b < ctx->n_sm; ++b)
         nt[(size_t)m * ctx->n_sm + b] =
             build_task_list(ctx->plan[m], b, tl.data() + ((size_t)m * ctx->n_sm + b) * kMaxTasks);
+    std::vector<LayerDev> ld((size_t)c.n_layers);
+    for (int l = 0; l < c.n_layers; ++l) {
+      const fmoe_layer_desc& L = ctx->layers[l];
+      ld[l] = LayerDev{static_cast<const uint8_t*>(L.experts_dev), static_cast<const uint16_t*>(L.router_w_dev),
+                       L.router_bias_dev, static_cast<const uint16_t*>(L.norm_w_dev)};
+    }
     e = cudaMemcpyAsync(ctx->tasks, tl.data(), tl.size() * 4, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaMemcpyAsync(ctx->ntasks, nt.data(), nt.size() * 4, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(ctx->layer_dev, ld.data(), ld.size() * sizeof(LayerDev), cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "task table upload"));
   }
@@ -641,6 +654,23 @@ fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer
   if (misaligned(h_in_dev) || misaligned(h_out_dev)) return fail(ctx, FMOE_ERR_ALIGNMENT, "tensor not 16-byte aligned");
   const size_t bytes = (size_t)T * ctx->cfg.hidden * 2;
   if (overlaps(h_in_dev, bytes, h_out_dev, bytes)) return fail(ctx, FMOE_ERR_INVALID_ARG, "h_out overlaps h_in");
+  const int n_layers = layer_end - layer_begin;
+  if (n_layers > 1 && !use_batched(ctx, T) && !(ctx->cfg.flags & FMOE_FLAG_STACK_PER_LAYER)) {
+    // one launch per token runs every layer of the range
+    const int H = ctx->cfg.hidden;
+    for (int t = 0; t < T; ++t) {
+      DecodePlan P = bind(ctx, kModeLayer, layer_begin);
+      P.n_layers = n_layers;
+      P.layer_dev = ctx->layer_dev + layer_begin;
+      P.hbuf[0] = ctx->stack_buf[0];
+      P.hbuf[1] = ctx->stack_buf[1];
+      P.h_in = static_cast<const uint16_t*>(h_in_dev) + (size_t)t * H;
+      P.h_out = static_cast<uint16_t*>(h_out_dev) + (size_t)t * H;
+      s = launch(ctx, P, stream);
+      if (s != FMOE_OK) return s;
+    }
+    return FMOE_OK;
+  }
   const uint16_t* cur = static_cast<const uint16_t*>(h_in_dev);
   for (int l = layer_begin; l < layer_end; ++l) {
     uint16_t* dst = (l + 1 == layer_end) ? static_cast<uint16_t*>(h_out_dev) : ctx->stack_buf[(l - layer_begin) & 1];

@@ -359,7 +359,32 @@ __device__ __forceinline__ bool wait_flag(const volatile int* f, int value, uint
 
 
 
-template <int BITS>
+// Barrier of the consumer warps that also tells every one of them whether any
+// thread arrived with v set, so all take the same branch afterwards.
+__device__ __forceinline__ bool consumers_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(kConsumerWarps * 32)
+      : "memory");
+  return r != 0;
+}
+
+// Weights of layer l: the plan's own for a single-layer launch.
+template <bool MULTI>
+__device__ __forceinline__ LayerDev layer_of(const DecodePlan& P, int l) {
+  if (MULTI) return P.layer_dev[l];
+  return LayerDev{P.experts, P.router_w, P.router_bias, P.norm_w};
+}
+
+// MULTI: one launch runs layers 0..n_layers-1 of a stack for one token.  The
+// producer streams on into layer l+1 (its router rows, then the shared
+// expert's chunks, which need no routing) while the consumers finish layer l;
+// the consumers write layer l's output rows, count themselves done on a
+// device-wide counter and wait for every block before normalising layer l's
+// output as layer l+1's input.  Tags advance by one per layer.
+template <int BITS, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodePlan P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -378,6 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   float* dnpart = reinterpret_cast<float*>(smem + P.off_dnpart);
   float* ys = reinterpret_cast<float*>(smem + P.off_y);
   const uint64_t limit = P.timeout_ns;
+  const int NL = MULTI ? P.n_layers : 1;
 
   // this block's share of the work
   const int first_rb = G - 1 - cta;
@@ -439,13 +465,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // ============================================================ producer warp
     bool routed = false;
     bool waited_grid = false;
+    uint32_t tag0 = 0;
+    int cur = 0;  // layer being issued
+    LayerDev Ld = layer_of<MULTI>(P, 0);
     auto do_routing = [&]() {
-      if (P.pdl && !waited_grid) asm volatile("griddepcontrol.wait;" ::: "memory");
+      if (!waited_grid) {
+        if (P.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+        tag0 = *reinterpret_cast<volatile uint32_t*>(&P.ws->epoch) + 1u;
+      }
       waited_grid = true;
-      // Poll the tagged logits until every router row of this launch is
+      // Poll the tagged logits until every router row of this layer is
       // published; each round a lane reads experts lane, lane+32, ... (16 loads
       // issued back to back) and stages them in shared memory for top-K.
-      const uint32_t tag = *reinterpret_cast<volatile uint32_t*>(&P.ws->epoch) + 1u;
+      const uint32_t tag = tag0 + (uint32_t)cur;
       constexpr int kPollE = 16;  // logits per lane per load round
       float* lg = reinterpret_cast<float*>(smem + P.off_lg);
       const uint64_t t0 = gtimer();
@@ -505,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const int NI = P.n_issuers;
     auto issue = [&](int i, uint32_t t) -> int {
       int s, fill;
-      task_stage_of(P.nstage, NI, n_tasks, n_down, i, s, fill);
+      task_stage_of(P.nstage, NI, n_tasks, n_down, i, s, fill, cur);
       if (fill > 0 && !wait_mbar(bar_empty + 8u * s, (uint32_t)((fill - 1) & 1), limit, abort_flag)) {
         if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutTma);
         *abort_flag = 1;
@@ -517,24 +549,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       const uint32_t ty = task_type(t), idx = task_idx(t), slot = task_slot(t), c = task_chunk(t);
       if (ty == kTaskRouter) {
         const int c0 = (int)c * P.router_part_cols;
-        src = P.router_w + (int64_t)(cta + (int)idx * G) * P.H + c0;
+        src = Ld.router_w + (int64_t)(cta + (int)idx * G) * P.H + c0;
         bytes = (uint32_t)min(P.router_part_cols, P.H - c0) * 2;
       } else if (ty == kTaskGateUp) {
         const int u = cta + (int)idx * G, rb = u % P.units_per_slot;
         const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
-        src = P.experts + (int64_t)misc->slot_e[slot] * P.blob_bytes + ((int64_t)rb * P.gu_tiles + c * kChunkTiles) * TB;
+        src = Ld.experts + (int64_t)misc->slot_e[slot] * P.blob_bytes + ((int64_t)rb * P.gu_tiles + c * kChunkTiles) * TB;
         bytes = (uint32_t)(n * TB);
       } else {
         const int rbg = first_rb + (int)idx * G;
         const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
-        src = P.experts + (int64_t)misc->slot_e[slot] * P.blob_bytes + packed_gu_bytes(P.H, P.I, BITS) +
+        src = Ld.experts + (int64_t)misc->slot_e[slot] * P.blob_bytes + packed_gu_bytes(P.H, P.I, BITS) +
               ((int64_t)rbg * P.dn_tiles + c * kChunkTiles) * TB;
         bytes = (uint32_t)(n * TB);
       }
       mbar_expect_tx(bar_full + 8u * s, bytes);
       tma_load(dst, src, bytes, bar_full + 8u * s);
       // tells the consumer of task i that this fill is the one to wait for
-      reinterpret_cast<volatile int*>(misc->last_task)[s] = i;
+      reinterpret_cast<volatile int*>(misc->last_task)[s] = cur * kMaxTasks + i;
       return 1;
     };
     // Down jobs with stages of their own (the block's last n_down tasks) are all
@@ -542,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // their weights land early and nothing streams any more when the
     // activations are exchanged.
     const int ring_end = n_tasks - n_down;
-    bool downs_issued = n_down == 0;
+    bool downs_issued;
     auto issue_downs = [&]() -> bool {
       for (int r = 0; ring_end + r * NI < n_tasks; ++r) {
         const int i = ring_end + r * NI + lane;
@@ -552,320 +584,385 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       downs_issued = true;
       return true;
     };
-    bool failed = P.mode == kModeExpert && !downs_issued && !issue_downs();
-    for (int r = 0; r * NI < ring_end && !failed; ++r) {
-      if (__any_sync(0xffffffffu, *abort_flag)) break;
-      const int i = r * NI + lane;
-      const bool mine = lane < NI && i < ring_end && i >= pre_issued;
-      const uint32_t t = mine ? tasks[i] : 0u;
-      const bool needs_route = mine && P.mode == kModeLayer && !routed && task_type(t) != kTaskRouter &&
-                               (task_slot(t) >= 1 || P.route_first);
-      int ok = 1;
-      if (mine && !needs_route) ok = issue(i, t);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      if (__any_sync(0xffffffffu, needs_route)) {
-        if (!do_routing()) break;
-        routed = true;
-        if (!downs_issued && !issue_downs()) break;
-        if (needs_route) ok = issue(i, t);
-        if (!__all_sync(0xffffffffu, ok)) break;
+    for (cur = 0; cur < NL; ++cur) {
+      if (cur > 0) {
+        if (__any_sync(0xffffffffu, *abort_flag)) break;
+        Ld = layer_of<MULTI>(P, cur);
+        routed = false;
       }
+      downs_issued = n_down == 0;
+      bool failed = P.mode == kModeExpert && !downs_issued && !issue_downs();
+      const int pre = cur == 0 ? pre_issued : 0;
+      for (int r = 0; r * NI < ring_end && !failed; ++r) {
+        if (__any_sync(0xffffffffu, *abort_flag)) break;
+        const int i = r * NI + lane;
+        const bool mine = lane < NI && i < ring_end && i >= pre;
+        const uint32_t t = mine ? tasks[i] : 0u;
+        // past a launch's first layer the shared expert's chunks stream in
+        // while the previous layer finishes, so they never wait for routing
+        const bool needs_route = mine && P.mode == kModeLayer && !routed && task_type(t) != kTaskRouter &&
+                                 (task_slot(t) >= 1 || (P.route_first && cur == 0));
+        int ok = 1;
+        if (mine && !needs_route) ok = issue(i, t);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        if (__any_sync(0xffffffffu, needs_route)) {
+          if (!do_routing()) break;
+          routed = true;
+          if (!downs_issued && !issue_downs()) break;
+          if (needs_route) ok = issue(i, t);
+          if (!__all_sync(0xffffffffu, ok)) break;
+        }
+      }
+      // a block whose own list needed no routing still owes its down jobs
+      if (!downs_issued && !__any_sync(0xffffffffu, *abort_flag)) {
+        if (P.mode == kModeLayer && !routed) routed = do_routing();
+        if (routed || P.mode != kModeLayer) issue_downs();
+      }
+      // routing still owed for the output indices
+      if (!__any_sync(0xffffffffu, *abort_flag) && !routed && has_router && cta == 0 && (P.idx_out || P.w_out))
+        do_routing();
     }
-    // a block whose own list needed no routing still owes its down jobs
-    if (!downs_issued && !__any_sync(0xffffffffu, *abort_flag)) {
-      if (P.mode == kModeLayer && !routed) routed = do_routing();
-      if (routed || P.mode != kModeLayer) issue_downs();
-    }
-    // routing still owed for the output indices
-    if (!__any_sync(0xffffffffu, *abort_flag) && !routed && has_router && cta == 0 && (P.idx_out || P.w_out))
-      do_routing();
   } else {
     // ============================================================ consumer warps
     if (P.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
-    const uint32_t tag = *reinterpret_cast<volatile uint32_t*>(&P.ws->epoch) + 1u;
-    if (tid == 0) misc->tag = tag;
+    const uint32_t tag0 = *reinterpret_cast<volatile uint32_t*>(&P.ws->epoch) + 1u;
+    if (tid == 0) misc->tag = tag0 + (uint32_t)(NL - 1);
     // residual rows this block writes at the end
     if (P.mode == kModeLayer && tid < my_rb * 16)
       h_res = bf16f(P.h_in[(first_rb + (tid / 16) * G) * 16 + tid % 16]);
-    // ---- input: z = RMSNorm(h_in) or h_in (bf16, shared memory) and its fragments
-    {
-      // thread tid holds columns 8*(tid + j*threads) .. +7, j < kPrepChunks
-      constexpr int kCT = kConsumerWarps * 32;
-      constexpr int kPrepChunks = (kMaxHidden + 8 * kCT - 1) / (8 * kCT);
-      uint4 hv[kPrepChunks];
-#pragma unroll
-      for (int j = 0; j < kPrepChunks; ++j) {
-        const int c0 = (tid + j * kCT) * 8;
-        hv[j] = c0 < P.H ? *reinterpret_cast<const uint4*>(P.h_in + c0) : make_uint4(0u, 0u, 0u, 0u);
-      }
-      if (P.norm_w != nullptr) {
-        float ss = 0.f;
-#pragma unroll
-        for (int j = 0; j < kPrepChunks; ++j) {
-          const uint32_t hw[4] = {hv[j].x, hv[j].y, hv[j].z, hv[j].w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            ss = fmaf(bf16lo(hw[k]), bf16lo(hw[k]), ss);
-            ss = fmaf(bf16hi(hw[k]), bf16hi(hw[k]), ss);
+    for (int cur = 0; cur < NL; ++cur) {
+      const uint32_t tag = tag0 + (uint32_t)cur;
+      const LayerDev Ld = layer_of<MULTI>(P, cur);
+      const uint16_t* h_in = (!MULTI || cur == 0) ? P.h_in : P.hbuf[(cur - 1) & 1];
+      if (MULTI && cur > 0) {
+        // every block has written its rows of the previous layer's output
+        bool ok = true;
+        if (tid == 0) {
+          const uint32_t target = (uint32_t)G * (uint32_t)cur;
+          const uint64_t t0 = gtimer();
+          for (uint32_t it = 0;; ++it) {
+            uint32_t v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&P.ws->layer_cnt) : "memory");
+            if (v >= target) break;
+            if ((it & 7) == 7 && (*abort_flag || gtimer() - t0 > limit)) {
+              ok = false;
+              if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutLayer);
+              *abort_flag = 1;
+              break;
+            }
+            __nanosleep(64);
           }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (lane == 0) misc->red[warp] = ss;
-        asm volatile("bar.sync 1, %0;" ::"r"(kCT) : "memory");
-        float tot = 0.f;
-        for (int w = 0; w < kConsumerWarps; ++w) tot += misc->red[w];
-        const float r = 1.0f / sqrtf(tot / (float)P.H + P.eps);
-#pragma unroll
+        if (consumers_any(!ok || *abort_flag != 0)) break;
+      }
+      // ---- input: z = RMSNorm(h_in) or h_in (bf16, shared memory) and its fragments
+      {
+        // thread tid holds columns 8*(tid + j*threads) .. +7, j < kPrepChunks
+        constexpr int kCT = kConsumerWarps * 32;
+        constexpr int kPrepChunks = (kMaxHidden + 8 * kCT - 1) / (8 * kCT);
+        uint4 hv[kPrepChunks];
+  #pragma unroll
         for (int j = 0; j < kPrepChunks; ++j) {
           const int c0 = (tid + j * kCT) * 8;
-          if (c0 < P.H) {
-            const uint4 wv = *reinterpret_cast<const uint4*>(P.norm_w + c0);
+          // another block's output when MULTI and cur > 0: read it from L2
+          hv[j] = c0 >= P.H ? make_uint4(0u, 0u, 0u, 0u)
+                  : MULTI   ? __ldcg(reinterpret_cast<const uint4*>(h_in + c0))
+                            : *reinterpret_cast<const uint4*>(h_in + c0);
+        }
+        if (Ld.norm_w != nullptr) {
+          float ss = 0.f;
+  #pragma unroll
+          for (int j = 0; j < kPrepChunks; ++j) {
             const uint32_t hw[4] = {hv[j].x, hv[j].y, hv[j].z, hv[j].w};
-            const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-            uint32_t zz[4];
-#pragma unroll
+  #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const uint32_t lo = f2bf16(bf16lo(hw[k]) * r * bf16lo(ww[k]));
-              const uint32_t hi = f2bf16(bf16hi(hw[k]) * r * bf16hi(ww[k]));
-              zz[k] = lo | (hi << 16);
-            }
-            hv[j] = make_uint4(zz[0], zz[1], zz[2], zz[3]);
-          }
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < kPrepChunks; ++j) {
-        const int c0 = (tid + j * kCT) * 8;
-        if (c0 < P.H) *reinterpret_cast<uint4*>(zs + c0) = hv[j];
-      }
-      asm volatile("bar.sync 1, %0;" ::"r"(kCT) : "memory");
-      if (P.n_slots > 0) {
-        // warp w builds groups 4w..4w+3, then 4(w+W).., so a batch is contiguous
-        const int ngz = P.H / kGroup;
-        for (int G0 = 4 * warp; G0 < ngz; G0 += 4 * kConsumerWarps) {
-          float lo[4], hi[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t zz = (G0 + k < ngz) ? *reinterpret_cast<const uint32_t*>(zs + (G0 + k) * kGroup + 2 * lane) : 0u;
-            lo[k] = bf16lo(zz);
-            hi[k] = bf16hi(zz);
-          }
-          frag_batch<4>(lo, hi, G0, ngz, BITS, zfrag, zinfo, lane);
-        }
-      }
-      asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
-    }
-
-    // The producer selects the routed experts once per launch, late; running
-    // the same selection code here on whatever the logit buffer holds (it
-    // writes nothing) brings that code into the instruction cache meanwhile.
-    if (warp == kConsumerWarps - 1 && P.mode != kModeExpert) {
-      const TopPick dummy = topk_select(reinterpret_cast<const float*>(smem + P.off_lg), P.E, P.K, lane);
-      if (dummy.expert < 0) misc->pad[0] = dummy.expert;  // never true; keeps the call
-    }
-    // ---- task loop: warp w takes tasks w, w+16, ...
-    for (int i = warp; i < n_tasks; i += kConsumerWarps) {
-      int s, fill;
-      task_stage_of(P.nstage, P.n_issuers, n_tasks, n_down, i, s, fill);
-      // A stage's fills are consumed by different warps, so first make sure
-      // task i is the stage's current fill (all earlier fills consumed); only
-      // then is the parity wait unambiguous.  Every lane observes the phase,
-      // so the copied bytes are visible to it.
-      const bool issued = wait_flag(reinterpret_cast<volatile int*>(misc->last_task) + s, i, limit, abort_flag);
-      if (!__all_sync(0xffffffffu, issued && wait_mbar(bar_full + 8u * s, (uint32_t)(fill & 1), limit, abort_flag))) {
-        if (lane == 0) {
-          if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutTma);
-          *abort_flag = 1;
-        }
-        break;
-      }
-      const uint8_t* stage = smem + P.off_ring + (uint32_t)s * P.stage_bytes;
-      const uint32_t t = tasks[i];
-      const uint32_t ty = task_type(t), idx = task_idx(t), slot = task_slot(t), c = task_chunk(t);
-      if (ty == kTaskRouter) {
-        const int c0 = (int)c * P.router_part_cols, width = min(P.router_part_cols, P.H - c0);
-        float acc = 0.f;
-        for (int col = lane * 8; col < width; col += 256) {
-          const uint4 w = *reinterpret_cast<const uint4*>(stage + col * 2);
-          const uint4 z = *reinterpret_cast<const uint4*>(zs + c0 + col);
-          acc = fmaf(bf16lo(w.x), bf16lo(z.x), acc);
-          acc = fmaf(bf16hi(w.x), bf16hi(z.x), acc);
-          acc = fmaf(bf16lo(w.y), bf16lo(z.y), acc);
-          acc = fmaf(bf16hi(w.y), bf16hi(z.y), acc);
-          acc = fmaf(bf16lo(w.z), bf16lo(z.z), acc);
-          acc = fmaf(bf16hi(w.z), bf16hi(z.z), acc);
-          acc = fmaf(bf16lo(w.w), bf16lo(z.w), acc);
-          acc = fmaf(bf16hi(w.w), bf16hi(z.w), acc);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) {
-          // parts of a row are summed, in part order, by whichever warp ends last
-          misc->rpart[idx][c] = acc;
-          __threadfence_block();
-          const int old = atomicAdd(&misc->rcnt[idx], 1);
-          if (old == P.router_parts - 1) {
-            __threadfence_block();
-            const volatile float* rp = misc->rpart[idx];
-            float l = 0.f;
-            for (int q = 0; q < P.router_parts; ++q) l += rp[q];
-            const int e = cta + (int)idx * G;
-            if (P.router_bias) l += P.router_bias[e];
-            // fault injection publishes with a stale tag, so no reader accepts it
-            st_tagged(P.ws_logits + e, l, (P.flags & FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE) ? tag - 1u : tag);
-            red_relaxed_add(&P.ws->router_cnt, 1u);
-          }
-        }
-      } else if (ty == kTaskGateUp) {
-        const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
-        const float2 acc = chunk_dot<BITS>(stage, n, zfrag, zinfo, (int)c * kChunkTiles, lane);
-        float acc0 = acc.x, acc1 = acc.y;
-        const int u = cta + (int)idx * G, rb = u % P.units_per_slot;
-        bool last = true;
-        if (P.gu_chunks > 1) {
-          float* part = gupart + ((int)idx * P.gu_chunks + (int)c) * 16;
-          if ((lane & 3) == 0) { part[lane >> 2] = acc0; part[8 + (lane >> 2)] = acc1; }
-          __syncwarp();
-          int old = 0;
-          if (lane == 0) {
-            __threadfence_block();
-            old = atomicAdd(&misc->unit_cnt[idx], 1);
-            __threadfence_block();
-          }
-          old = __shfl_sync(0xffffffffu, old, 0);
-          last = old == P.gu_chunks - 1;
-          if (last && lane < 8) {
-            acc0 = 0.f;
-            acc1 = 0.f;
-            for (int k = 0; k < P.gu_chunks; ++k) {
-              const volatile float* pk = gupart + ((int)idx * P.gu_chunks + k) * 16;
-              acc0 += pk[lane];
-              acc1 += pk[8 + lane];
+              ss = fmaf(bf16lo(hw[k]), bf16lo(hw[k]), ss);
+              ss = fmaf(bf16hi(hw[k]), bf16hi(hw[k]), ss);
             }
           }
-        }
-        if (last) {
-          // lanes 0..7 (gu_chunks > 1) or lanes 4g (gu_chunks == 1) hold row g
-          const int row = P.gu_chunks > 1 ? lane : (lane >> 2);
-          const bool writer = P.gu_chunks > 1 ? lane < 8 : (lane & 3) == 0;
-          const float av = writer ? acc0 / (1.0f + expf(-acc0)) * acc1 : 0.f;
-          if (writer) st_tagged(P.ws_a + (int64_t)slot * P.I + rb * 8 + row, av, tag);
-          if (lane == 0) red_relaxed_add(&P.ws->h_cnt[slot], 1u);
-        }
-      } else {
-        // activations of this slot as fragments, built once per block in two
-        // halves of the slot's groups: the block's two down jobs of a slot
-        // usually run on two warps, which then fetch and build a half each.
-        uint32_t* af = reinterpret_cast<uint32_t*>(smem + P.off_afrag + slot * P.afrag_bytes);
-        float2* ai = reinterpret_cast<float2*>(smem + P.off_ainfo + slot * P.ainfo_bytes);
-        const uint64_t* act = P.ws_a + (int64_t)slot * P.I;
-        const int ng = P.I / kGroup, half_g = (ng + 1) / 2;
-        int good = 1;
-        for (int h = 0; h < 2 && good; ++h) {
-          const int gb = h * half_g, ge = min(ng, gb + half_g);
-          int* flag = &misc->aflag[2 * (int)slot + h];
-          int claimed = 0;
-          if (lane == 0 && *reinterpret_cast<volatile int*>(flag) == 0 && atomicCAS(flag, 0, 1) == 0) claimed = 1;
-          claimed = __shfl_sync(0xffffffffu, claimed, 0);
-          if (!claimed) continue;
-          // The slot's activations are tagged words published by every block's
-          // gate/up units.  Each lane fetches its pair (2*lane, 2*lane+1) of up
-          // to kFetchGroups groups in one round trip and the round is repeated
-          // until every tag is current; the published count only paces the
-          // retries.  Each group then gets its own power-of-two scale and sum,
-          // exactly as the input z does.
-          const uint64_t t0 = gtimer();
-          for (int g0 = gb; g0 < ge && good; g0 += kFetchGroups) {
-            ulonglong2 v[kFetchGroups];
-            for (int attempt = 0;; ++attempt) {
-              // every load is issued before any result is examined: the loads
-              // are volatile, so a check between two of them would wait for
-              // the first one's round trip before issuing the second
-#pragma unroll
-              for (int k = 0; k < kFetchGroups; ++k)  // past the end: re-read the last group, ignored below
-                v[k] = ld_tagged2(act + min(g0 + k, ge - 1) * kGroup + 2 * lane);
-              bool mine = true;
-#pragma unroll
-              for (int k = 0; k < kFetchGroups; ++k)
-                if (g0 + k < ge) mine = mine && tagged_tag(v[k].x) == tag && tagged_tag(v[k].y) == tag;
-              if (__all_sync(0xffffffffu, mine)) break;
-              // not all published yet: wait for the count, then fetch again
-              const bool counted =
-                  wait_count(&P.ws->h_cnt[slot], (uint32_t)P.units_per_slot, limit, abort_flag);
-              if (__any_sync(0xffffffffu, !counted || *abort_flag != 0 || gtimer() - t0 > limit)) {
-                good = 0;
-                break;
+  #pragma unroll
+          for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          if (lane == 0) misc->red[warp] = ss;
+          asm volatile("bar.sync 1, %0;" ::"r"(kCT) : "memory");
+          float tot = 0.f;
+          for (int w = 0; w < kConsumerWarps; ++w) tot += misc->red[w];
+          const float r = 1.0f / sqrtf(tot / (float)P.H + P.eps);
+  #pragma unroll
+          for (int j = 0; j < kPrepChunks; ++j) {
+            const int c0 = (tid + j * kCT) * 8;
+            if (c0 < P.H) {
+              const uint4 wv = *reinterpret_cast<const uint4*>(Ld.norm_w + c0);
+              const uint32_t hw[4] = {hv[j].x, hv[j].y, hv[j].z, hv[j].w};
+              const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+              uint32_t zz[4];
+  #pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint32_t lo = f2bf16(bf16lo(hw[k]) * r * bf16lo(ww[k]));
+                const uint32_t hi = f2bf16(bf16hi(hw[k]) * r * bf16hi(ww[k]));
+                zz[k] = lo | (hi << 16);
               }
-              if (attempt > 0) __nanosleep(256);
+              hv[j] = make_uint4(zz[0], zz[1], zz[2], zz[3]);
             }
-            if (!good) break;
-            float lo[kFetchGroups], hi[kFetchGroups];
-#pragma unroll
-            for (int k = 0; k < kFetchGroups; ++k) {
-              lo[k] = tagged_value(v[k].x);
-              hi[k] = tagged_value(v[k].y);
-            }
-            frag_batch<kFetchGroups>(lo, hi, g0, ge, BITS, af, ai, lane);
           }
-          if (!good && lane == 0) {
-            if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
+        }
+  #pragma unroll
+        for (int j = 0; j < kPrepChunks; ++j) {
+          const int c0 = (tid + j * kCT) * 8;
+          if (c0 < P.H) *reinterpret_cast<uint4*>(zs + c0) = hv[j];
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(kCT) : "memory");
+        if (P.n_slots > 0) {
+          // warp w builds groups 4w..4w+3, then 4(w+W).., so a batch is contiguous
+          const int ngz = P.H / kGroup;
+          for (int G0 = 4 * warp; G0 < ngz; G0 += 4 * kConsumerWarps) {
+            float lo[4], hi[4];
+  #pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t zz = (G0 + k < ngz) ? *reinterpret_cast<const uint32_t*>(zs + (G0 + k) * kGroup + 2 * lane) : 0u;
+              lo[k] = bf16lo(zz);
+              hi[k] = bf16hi(zz);
+            }
+            frag_batch<4>(lo, hi, G0, ngz, BITS, zfrag, zinfo, lane);
+          }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
+      }
+
+      // The producer selects the routed experts once per launch, late; running
+      // the same selection code here on whatever the logit buffer holds (it
+      // writes nothing) brings that code into the instruction cache meanwhile.
+      if (warp == kConsumerWarps - 1 && P.mode != kModeExpert && cur == 0) {
+        const TopPick dummy = topk_select(reinterpret_cast<const float*>(smem + P.off_lg), P.E, P.K, lane);
+        if (dummy.expert < 0) misc->pad[0] = dummy.expert;  // never true; keeps the call
+      }
+      // ---- task loop: warp w takes tasks w, w+16, ...
+      for (int i = warp; i < n_tasks; i += kConsumerWarps) {
+        int s, fill;
+        task_stage_of(P.nstage, P.n_issuers, n_tasks, n_down, i, s, fill, cur);
+        // A stage's fills are consumed by different warps, so first make sure
+        // task i is the stage's current fill (all earlier fills consumed); only
+        // then is the parity wait unambiguous.  Every lane observes the phase,
+        // so the copied bytes are visible to it.
+        const bool issued =
+            wait_flag(reinterpret_cast<volatile int*>(misc->last_task) + s, cur * kMaxTasks + i, limit, abort_flag);
+        if (!__all_sync(0xffffffffu, issued && wait_mbar(bar_full + 8u * s, (uint32_t)(fill & 1), limit, abort_flag))) {
+          if (lane == 0) {
+            if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutTma);
             *abort_flag = 1;
           }
-          if (good) {
+          break;
+        }
+        const uint8_t* stage = smem + P.off_ring + (uint32_t)s * P.stage_bytes;
+        const uint32_t t = tasks[i];
+        const uint32_t ty = task_type(t), idx = task_idx(t), slot = task_slot(t), c = task_chunk(t);
+        if (ty == kTaskRouter) {
+          const int c0 = (int)c * P.router_part_cols, width = min(P.router_part_cols, P.H - c0);
+          float acc = 0.f;
+          for (int col = lane * 8; col < width; col += 256) {
+            const uint4 w = *reinterpret_cast<const uint4*>(stage + col * 2);
+            const uint4 z = *reinterpret_cast<const uint4*>(zs + c0 + col);
+            acc = fmaf(bf16lo(w.x), bf16lo(z.x), acc);
+            acc = fmaf(bf16hi(w.x), bf16hi(z.x), acc);
+            acc = fmaf(bf16lo(w.y), bf16lo(z.y), acc);
+            acc = fmaf(bf16hi(w.y), bf16hi(z.y), acc);
+            acc = fmaf(bf16lo(w.z), bf16lo(z.z), acc);
+            acc = fmaf(bf16hi(w.z), bf16hi(z.z), acc);
+            acc = fmaf(bf16lo(w.w), bf16lo(z.w), acc);
+            acc = fmaf(bf16hi(w.w), bf16hi(z.w), acc);
+          }
+  #pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (lane == 0) {
+            // parts of a row are summed, in part order, by whichever warp ends last
+            misc->rpart[idx][c] = acc;
+            __threadfence_block();
+            const int old = atomicAdd(&misc->rcnt[idx], 1);
+            if (old == P.router_parts - 1) {
+              __threadfence_block();
+              const volatile float* rp = misc->rpart[idx];
+              float l = 0.f;
+              for (int q = 0; q < P.router_parts; ++q) l += rp[q];
+              const int e = cta + (int)idx * G;
+              if (Ld.router_bias) l += Ld.router_bias[e];
+              // fault injection publishes with a stale tag, so no reader accepts it
+              st_tagged(P.ws_logits + e, l, (P.flags & FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE) ? tag - 1u : tag);
+              red_relaxed_add(&P.ws->router_cnt, 1u);
+            }
+          }
+        } else if (ty == kTaskGateUp) {
+          const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
+          const float2 acc = chunk_dot<BITS>(stage, n, zfrag, zinfo, (int)c * kChunkTiles, lane);
+          float acc0 = acc.x, acc1 = acc.y;
+          const int u = cta + (int)idx * G, rb = u % P.units_per_slot;
+          bool last = true;
+          if (P.gu_chunks > 1) {
+            float* part = gupart + ((int)idx * P.gu_chunks + (int)c) * 16;
+            if ((lane & 3) == 0) { part[lane >> 2] = acc0; part[8 + (lane >> 2)] = acc1; }
             __syncwarp();
+            int old = 0;
             if (lane == 0) {
               __threadfence_block();
-              *reinterpret_cast<volatile int*>(flag) = 2;
+              old = atomicAdd(&misc->unit_cnt[idx], 1);
+              __threadfence_block();
+            }
+            old = __shfl_sync(0xffffffffu, old, 0);
+            last = old == P.gu_chunks - 1;
+            if (last && lane < 8) {
+              acc0 = 0.f;
+              acc1 = 0.f;
+              for (int k = 0; k < P.gu_chunks; ++k) {
+                const volatile float* pk = gupart + ((int)idx * P.gu_chunks + k) * 16;
+                acc0 += pk[lane];
+                acc1 += pk[8 + lane];
+              }
+            }
+          }
+          if (last) {
+            // lanes 0..7 (gu_chunks > 1) or lanes 4g (gu_chunks == 1) hold row g
+            const int row = P.gu_chunks > 1 ? lane : (lane >> 2);
+            const bool writer = P.gu_chunks > 1 ? lane < 8 : (lane & 3) == 0;
+            const float av = writer ? acc0 / (1.0f + expf(-acc0)) * acc1 : 0.f;
+            if (writer) st_tagged(P.ws_a + (int64_t)slot * P.I + rb * 8 + row, av, tag);
+            if (lane == 0) red_relaxed_add(&P.ws->h_cnt[slot], 1u);
+          }
+        } else {
+          // activations of this slot as fragments, built once per block in two
+          // halves of the slot's groups: the block's two down jobs of a slot
+          // usually run on two warps, which then fetch and build a half each.
+          uint32_t* af = reinterpret_cast<uint32_t*>(smem + P.off_afrag + slot * P.afrag_bytes);
+          float2* ai = reinterpret_cast<float2*>(smem + P.off_ainfo + slot * P.ainfo_bytes);
+          const uint64_t* act = P.ws_a + (int64_t)slot * P.I;
+          const int ng = P.I / kGroup, half_g = (ng + 1) / 2;
+          int good = 1;
+          for (int h = 0; h < 2 && good; ++h) {
+            const int gb = h * half_g, ge = min(ng, gb + half_g);
+            int* flag = &misc->aflag[2 * (int)slot + h];
+            int claimed = 0;
+            if (lane == 0 && *reinterpret_cast<volatile int*>(flag) == 0 && atomicCAS(flag, 0, 1) == 0) claimed = 1;
+            claimed = __shfl_sync(0xffffffffu, claimed, 0);
+            if (!claimed) continue;
+            // The slot's activations are tagged words published by every block's
+            // gate/up units.  Each lane fetches its pair (2*lane, 2*lane+1) of up
+            // to kFetchGroups groups in one round trip and the round is repeated
+            // until every tag is current; the published count only paces the
+            // retries.  Each group then gets its own power-of-two scale and sum,
+            // exactly as the input z does.
+            const uint64_t t0 = gtimer();
+            for (int g0 = gb; g0 < ge && good; g0 += kFetchGroups) {
+              ulonglong2 v[kFetchGroups];
+              for (int attempt = 0;; ++attempt) {
+                // every load is issued before any result is examined: the loads
+                // are volatile, so a check between two of them would wait for
+                // the first one's round trip before issuing the second
+  #pragma unroll
+                for (int k = 0; k < kFetchGroups; ++k)  // past the end: re-read the last group, ignored below
+                  v[k] = ld_tagged2(act + min(g0 + k, ge - 1) * kGroup + 2 * lane);
+                bool mine = true;
+  #pragma unroll
+                for (int k = 0; k < kFetchGroups; ++k)
+                  if (g0 + k < ge) mine = mine && tagged_tag(v[k].x) == tag && tagged_tag(v[k].y) == tag;
+                if (__all_sync(0xffffffffu, mine)) break;
+                // not all published yet: wait for the count, then fetch again
+                const bool counted =
+                    wait_count(&P.ws->h_cnt[slot], (uint32_t)(P.units_per_slot * (cur + 1)), limit, abort_flag);
+                if (__any_sync(0xffffffffu, !counted || *abort_flag != 0 || gtimer() - t0 > limit)) {
+                  good = 0;
+                  break;
+                }
+                if (attempt > 0) __nanosleep(256);
+              }
+              if (!good) break;
+              float lo[kFetchGroups], hi[kFetchGroups];
+  #pragma unroll
+              for (int k = 0; k < kFetchGroups; ++k) {
+                lo[k] = tagged_value(v[k].x);
+                hi[k] = tagged_value(v[k].y);
+              }
+              frag_batch<kFetchGroups>(lo, hi, g0, ge, BITS, af, ai, lane);
+            }
+            if (!good && lane == 0) {
+              if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
+              *abort_flag = 1;
+            }
+            if (good) {
+              __syncwarp();
+              if (lane == 0) {
+                __threadfence_block();
+                *reinterpret_cast<volatile int*>(flag) = 2;
+              }
+            }
+          }
+          // both halves ready (built here or by another warp)
+          for (int h = 0; h < 2 && good; ++h) {
+            if (h * half_g >= ng) continue;
+            if (lane == 0 && !wait_flag(&misc->aflag[2 * (int)slot + h], 2, limit, abort_flag)) {
+              if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
+              *abort_flag = 1;
+              good = 0;
+            }
+            good = __shfl_sync(0xffffffffu, good, 0);
+          }
+          __threadfence_block();
+          if (!good) break;
+          const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
+          const float2 acc = chunk_dot<BITS>(stage, n, af, ai, (int)c * kChunkTiles, lane);
+          const float acc0 = acc.x, acc1 = acc.y;
+          float* y = ys + ((int)idx * P.n_slots + (int)slot) * 16;
+          if (P.dn_chunks == 1) {
+            if ((lane & 3) == 0) { y[lane >> 2] = acc0; y[8 + (lane >> 2)] = acc1; }
+          } else {
+            const int job = (int)idx * P.n_slots + (int)slot;
+            float* part = dnpart + (job * P.dn_chunks + (int)c) * 16;
+            if ((lane & 3) == 0) { part[lane >> 2] = acc0; part[8 + (lane >> 2)] = acc1; }
+            __syncwarp();
+            int old = 0;
+            if (lane == 0) {
+              __threadfence_block();
+              old = atomicAdd(&misc->dn_cnt[job], 1);
+              __threadfence_block();
+            }
+            old = __shfl_sync(0xffffffffu, old, 0);
+            if (old == P.dn_chunks - 1 && lane < 16) {
+              float v = 0.f;
+              for (int k = 0; k < P.dn_chunks; ++k) v += reinterpret_cast<volatile float*>(dnpart)[(job * P.dn_chunks + k) * 16 + lane];
+              y[lane] = v;
             }
           }
         }
-        // both halves ready (built here or by another warp)
-        for (int h = 0; h < 2 && good; ++h) {
-          if (h * half_g >= ng) continue;
-          if (lane == 0 && !wait_flag(&misc->aflag[2 * (int)slot + h], 2, limit, abort_flag)) {
-            if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutH);
-            *abort_flag = 1;
-            good = 0;
-          }
-          good = __shfl_sync(0xffffffffu, good, 0);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty + 8u * s);
+      }
+      if (MULTI) {
+        // all consumer warps are done with this layer's tasks
+        if (consumers_any(*abort_flag != 0)) break;
+        uint16_t* h_out = cur == NL - 1 ? P.h_out : P.hbuf[cur & 1];
+        if (tid < my_rb * 16) {
+          const int jb = tid / 16, row = tid % 16;
+          float acc = h_res + ys[(jb * P.n_slots + 0) * 16 + row];
+          for (int k = 1; k < P.n_slots; ++k) acc = fmaf(misc->slot_w[k], ys[(jb * P.n_slots + k) * 16 + row], acc);
+          const uint16_t o = f2bf16(acc);
+          h_out[(first_rb + jb * G) * 16 + row] = o;
+          h_res = bf16f(o);  // the next layer's residual input of this row
         }
-        __threadfence_block();
-        if (!good) break;
-        const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
-        const float2 acc = chunk_dot<BITS>(stage, n, af, ai, (int)c * kChunkTiles, lane);
-        const float acc0 = acc.x, acc1 = acc.y;
-        float* y = ys + ((int)idx * P.n_slots + (int)slot) * 16;
-        if (P.dn_chunks == 1) {
-          if ((lane & 3) == 0) { y[lane >> 2] = acc0; y[8 + (lane >> 2)] = acc1; }
-        } else {
-          const int job = (int)idx * P.n_slots + (int)slot;
-          float* part = dnpart + (job * P.dn_chunks + (int)c) * 16;
-          if ((lane & 3) == 0) { part[lane >> 2] = acc0; part[8 + (lane >> 2)] = acc1; }
-          __syncwarp();
-          int old = 0;
-          if (lane == 0) {
-            __threadfence_block();
-            old = atomicAdd(&misc->dn_cnt[job], 1);
-            __threadfence_block();
-          }
-          old = __shfl_sync(0xffffffffu, old, 0);
-          if (old == P.dn_chunks - 1 && lane < 16) {
-            float v = 0.f;
-            for (int k = 0; k < P.dn_chunks; ++k) v += reinterpret_cast<volatile float*>(dnpart)[(job * P.dn_chunks + k) * 16 + lane];
-            y[lane] = v;
-          }
+        if (warp == 1) {
+          misc->aflag[lane] = 0;
+          misc->unit_cnt[lane] = 0;
+          misc->dn_cnt[lane] = 0;
+          if (lane < 16) misc->rcnt[lane] = 0;
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
+        if (tid == 0 && cur + 1 < NL) {
+          __threadfence();
+          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&P.ws->layer_cnt) : "memory");
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_empty + 8u * s);
     }
   }
   __syncthreads();
 
   // ---------------------------------------------------------------- combine + output
   const bool aborted = *abort_flag != 0;
-  if (!aborted && tid < kConsumerWarps * 32) {
+  if (!MULTI && !aborted && tid < kConsumerWarps * 32) {
     for (int r = tid; r < my_rb * 16; r += kConsumerWarps * 32) {
       const int jb = r / 16, row = r % 16;
       const int out_row = (first_rb + jb * G) * 16 + row;
@@ -884,10 +981,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // After an abort the latest copy into every stage must land before the
     // block exits (without one, every issued copy was consumed already).
     for (int s = 0; s < n_stages_all && aborted; ++s) {
-      const int i = misc->last_task[s];
-      if (i < 0) continue;
+      const int uid = misc->last_task[s];
+      if (uid < 0) continue;
       int s2, fill;
-      task_stage_of(P.nstage, P.n_issuers, n_tasks, n_down, i, s2, fill);
+      task_stage_of(P.nstage, P.n_issuers, n_tasks, n_down, uid % kMaxTasks, s2, fill, uid / kMaxTasks);
       const uint64_t t0 = gtimer();
       while (!mbar_try_wait(bar_full + 8u * s, (uint32_t)(fill & 1)))
         if (gtimer() - t0 > limit) {
@@ -901,6 +998,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (old == (uint32_t)G - 1) {
       P.ws->exit_count = 0;
       P.ws->router_cnt = 0;
+      P.ws->layer_cnt = 0;
       for (int k = 0; k < 16; ++k) P.ws->h_cnt[k] = 0;
       P.ws->epoch = misc->tag;
     }
@@ -909,8 +1007,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
 }  // namespace
 
-int decode_occupancy(int bits, int smem_bytes, int* blocks_per_sm) {
-  void (*kern)(DecodePlan) = bits == 4 ? decode_kernel<4> : decode_kernel<2>;
+using DecodeFn = void (*)(DecodePlan);
+DecodeFn decode_fn(int bits, bool multi) {
+  if (bits == 4) return multi ? decode_kernel<4, true> : decode_kernel<4, false>;
+  return multi ? decode_kernel<2, true> : decode_kernel<2, false>;
+}
+
+int decode_occupancy(int bits, bool multi, int smem_bytes, int* blocks_per_sm) {
+  DecodeFn kern = decode_fn(bits, multi);
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (err != cudaSuccess) return (int)err;
   return (int)cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, kern, kThreads, smem_bytes);
@@ -925,7 +1029,7 @@ int decode_max_smem_optin(int device) {
 int launch_decode(const DecodePlan& plan, void* stream, bool cooperative, bool pdl) {
   DecodePlan p = plan;
   p.pdl = pdl ? 1 : 0;
-  void (*kern)(DecodePlan) = p.bits == 4 ? decode_kernel<4> : decode_kernel<2>;
+  DecodeFn kern = decode_fn(p.bits, p.n_layers > 0);
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem_bytes);
   if (err != cudaSuccess) return (int)err;
   cudaLaunchConfig_t cfg = {};

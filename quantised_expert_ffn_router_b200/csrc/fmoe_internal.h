@@ -70,7 +70,9 @@ struct WsHeader {
   uint32_t exit_count;      // blocks finished in the current launch
   uint32_t status;          // kStatus* bits, cleared by fmoe_poll_status
   uint32_t router_cnt;      // router rows published in this launch (hint for pollers)
-  uint32_t h_cnt[16];       // gate/up units published per slot in this launch (hint)
+  uint32_t h_cnt[16];       // gate/up units published per slot in this launch (hint; cumulative over
+                            // the layers of a multi-layer launch)
+  uint32_t layer_cnt;       // blocks done with a layer's combine, cumulative over a multi-layer launch
 };
 static_assert(sizeof(WsHeader) <= 256, "header");
 
@@ -79,6 +81,7 @@ constexpr uint32_t kStatusTimeoutRouter = 0x1;
 constexpr uint32_t kStatusTimeoutH = 0x2;
 constexpr uint32_t kStatusTimeoutTma = 0x4;
 constexpr uint32_t kStatusTimeoutTc = 0x8;   // a bounded wait of the grouped tensor-core GEMM ran out
+constexpr uint32_t kStatusTimeoutLayer = 0x10;  // a multi-layer launch waited too long for the previous layer
 
 
 enum DecodeMode : int { kModeLayer = 0, kModeExpert = 1, kModeRoute = 2 };
@@ -108,6 +111,14 @@ struct Misc {
   int dn_cnt[32];       // K-chunks finished per (row block, slot) down job
   int last_task[64];    // last task issued into each ring stage (-1: none)
   float red[16];        // RMSNorm scratch
+};
+
+// Per-layer weights of a multi-layer launch (device array, one entry per layer).
+struct LayerDev {
+  const uint8_t* experts;
+  const uint16_t* router_w;
+  const float* router_bias;
+  const uint16_t* norm_w;
 };
 
 // Everything the fused single-token kernel needs, computed on the host.
@@ -168,6 +179,12 @@ struct DecodePlan {
   uint32_t flags;
   uint64_t timeout_ns;
   int pdl;                 // launched with programmatic stream serialisation
+  // multi-layer launch (n_layers > 0): layers 0..n_layers-1 take their weights
+  // from layer_dev[l]; layer 0 reads h_in, the last writes h_out, layer l writes
+  // hbuf[l & 1] in between.  n_layers == 0: one layer from the fields above.
+  int n_layers;
+  const LayerDev* layer_dev;
+  uint16_t* hbuf[2];
 };
 
 // Ring position of task i: issued by producer lane i % n_issuers into that
@@ -179,17 +196,22 @@ inline __host__ __device__ void task_stage(int nstage, int n_issuers, int i, int
   fill = j / L;
 }
 
-// Stage and fill of task i of a block whose last n_down tasks are its down
-// jobs: those sit in dedicated stages after the ring (one fill each), the other
-// tasks cycle through the ring.
+// Stage and fill of task i of layer l (0 for a single-layer launch) of a block
+// whose last n_down tasks are its down jobs: those sit in dedicated stages after
+// the ring (one fill per layer), the other tasks cycle through the ring.  Layer
+// by layer, producer lane i % n_issuers issues the same ring_end-task list, so
+// its k-th issue of the launch is issue i / n_issuers of layer l plus the
+// ceil((ring_end - lane) / n_issuers) issues it made in each earlier layer: a
+// stage is always refilled by the same lane, in order.
 inline __host__ __device__ void task_stage_of(int nstage, int n_issuers, int n_tasks, int n_down, int i, int& stage,
-                                              int& fill) {
+                                              int& fill, int layer = 0) {
   const int ring_end = n_tasks - n_down;
   if (i >= ring_end) {
     stage = nstage + (i - ring_end);
-    fill = 0;
+    fill = layer;
   } else {
-    task_stage(nstage, n_issuers, i, stage, fill);
+    const int lane = i % n_issuers, per_layer = (ring_end - lane + n_issuers - 1) / n_issuers;
+    task_stage(nstage, n_issuers, (layer * per_layer + i / n_issuers) * n_issuers + lane, stage, fill);
   }
 }
 
@@ -302,7 +324,7 @@ int launch_route_static(const uint16_t* wr, const float* bias, const uint16_t* n
 // 4-bit -> 2-bit requantisation of n canonical blobs (fmoe_requant.cu).
 int launch_requant(const uint8_t* src, uint8_t* dst, int n_blobs, int H, int I, int n_sm, void* stream);
 int decode_max_smem_optin(int device);
-int decode_occupancy(int bits, int smem_bytes, int* blocks_per_sm);
+int decode_occupancy(int bits, bool multi, int smem_bytes, int* blocks_per_sm);
 int zero_workspace(void* ws, size_t bytes, void* stream);
 
 }  // namespace fmoe
