@@ -30,6 +30,7 @@ struct fmoe_ctx {
   int32_t* ntasks = nullptr;   // device [3 modes][grid]
   uint16_t* stack_buf[2] = {nullptr, nullptr};  // ping-pong activations, [max_tokens][H] bf16
   LayerDev* layer_dev = nullptr;                // device [n_layers]: weights of every layer (multi-layer launches)
+  uint64_t* hwords = nullptr;                   // device [H] tagged: a multi-layer launch's intermediate outputs
   void* bws_mem = nullptr;  // batched-path workspace (max_tokens > 1)
   BatchWs bws{};
   std::vector<TmaDesc> tc_maps;  // per layer: tensor maps of the packed gate/up and down matrices
@@ -353,7 +354,7 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   }
 
   // workspace: header | logits [E] | activations [kMaxSlots][I] | task lists | 2 x [max_tokens][H] bf16 |
-  // per-layer weight table
+  // per-layer weight table | tagged layer outputs [H]
   size_t off = 256;
   size_t off_logits = off;
   off += ((size_t)c.n_experts * 8 + 255) / 256 * 256;
@@ -368,6 +369,8 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   off += 2 * stack_bytes;
   size_t off_layers = off;
   off += ((size_t)c.n_layers * sizeof(LayerDev) + 255) / 256 * 256;
+  size_t off_hwords = off;
+  off += ((size_t)c.hidden * 8 + 255) / 256 * 256;
   ctx->ws_bytes = off;
   e = cudaMalloc(&ctx->ws, ctx->ws_bytes);
   if (e != cudaSuccess) {
@@ -384,6 +387,7 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   ctx->stack_buf[0] = reinterpret_cast<uint16_t*>(base + off_stack);
   ctx->stack_buf[1] = reinterpret_cast<uint16_t*>(base + off_stack + stack_bytes);
   ctx->layer_dev = reinterpret_cast<LayerDev*>(base + off_layers);
+  ctx->hwords = reinterpret_cast<uint64_t*>(base + off_hwords);
   // batched path: sized for max_tokens, only when more than one token is allowed
   const bool grouped_ok = c.n_experts <= kBatchMaxExperts && c.max_tokens <= kBatchMaxTokens;
   if ((c.flags & FMOE_FLAG_FORCE_GROUPED) && !grouped_ok)
@@ -662,8 +666,7 @@ fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer
       DecodePlan P = bind(ctx, kModeLayer, layer_begin);
       P.n_layers = n_layers;
       P.layer_dev = ctx->layer_dev + layer_begin;
-      P.hbuf[0] = ctx->stack_buf[0];
-      P.hbuf[1] = ctx->stack_buf[1];
+      P.ws_h = ctx->hwords;
       P.h_in = static_cast<const uint16_t*>(h_in_dev) + (size_t)t * H;
       P.h_out = static_cast<uint16_t*>(h_out_dev) + (size_t)t * H;
       s = launch(ctx, P, stream);

@@ -381,9 +381,9 @@ __device__ __forceinline__ LayerDev layer_of(const DecodePlan& P, int l) {
 // MULTI: one launch runs layers 0..n_layers-1 of a stack for one token.  The
 // producer streams on into layer l+1 (its router rows, then the shared
 // expert's chunks, which need no routing) while the consumers finish layer l;
-// the consumers write layer l's output rows, count themselves done on a
-// device-wide counter and wait for every block before normalising layer l's
-// output as layer l+1's input.  Tags advance by one per layer.
+// each block publishes its rows of layer l's output as tagged words, and every
+// block reads all of them back (until every tag is layer l's) as layer l+1's
+// input.  Tags advance by one per layer.
 template <int BITS, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodePlan P) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -409,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int first_rb = G - 1 - cta;
   const int my_rb = (P.n_slots > 0 && first_rb < P.n_rb) ? (P.n_rb - first_rb + G - 1) / G : 0;
   const bool has_router = P.mode != kModeExpert;
+  const int my_rrows = (has_router && cta < P.E) ? (P.E - cta + G - 1) / G : 0;
   const int n_down = P.n_down_max > 0 ? my_rb * P.n_slots * P.dn_chunks : 0;
   float h_res = 0.f;  // residual input of the row this thread combines
 
@@ -424,7 +425,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     asm volatile("fence.mbarrier_init.release.cluster;\n fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
     if (has_router && P.router_parts == 1) {
-      const int my_rrows = cta < P.E ? (P.E - cta + G - 1) / G : 0;
       pre_issued = min(my_rrows, P.n_issuers);
       if (lane < pre_issued) {
         int s, fill;
@@ -445,7 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
     misc->unit_cnt[lane] = 0;
     misc->dn_cnt[lane] = 0;
-    if (lane == 0) misc->abort = 0;
+    if (lane == 0) {
+      misc->abort = 0;
+      misc->rdone = 0;
+    }
   } else if (warp == 2) {
     // this block's ordered task list, global -> shared
     const uint32_t* src = P.tasks + (int64_t)cta * kMaxTasks;
@@ -633,69 +636,100 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     for (int cur = 0; cur < NL; ++cur) {
       const uint32_t tag = tag0 + (uint32_t)cur;
       const LayerDev Ld = layer_of<MULTI>(P, cur);
-      const uint16_t* h_in = (!MULTI || cur == 0) ? P.h_in : P.hbuf[(cur - 1) & 1];
-      if (MULTI && cur > 0) {
-        // every block has written its rows of the previous layer's output
-        bool ok = true;
-        if (tid == 0) {
-          const uint32_t target = (uint32_t)G * (uint32_t)cur;
-          const uint64_t t0 = gtimer();
-          for (uint32_t it = 0;; ++it) {
-            uint32_t v;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&P.ws->layer_cnt) : "memory");
-            if (v >= target) break;
-            if ((it & 7) == 7 && (*abort_flag || gtimer() - t0 > limit)) {
-              ok = false;
-              if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutLayer);
-              *abort_flag = 1;
-              break;
-            }
-            __nanosleep(64);
-          }
-        }
-        if (consumers_any(!ok || *abort_flag != 0)) break;
+      // thread tid holds columns 8*(tid + j*threads) .. +7, j < kPrepChunks
+      constexpr int kCT = kConsumerWarps * 32;
+      constexpr int kPrepChunks = (kMaxHidden + 8 * kCT - 1) / (8 * kCT);
+      // the layer's RMSNorm weights do not depend on the previous layer: their
+      // loads are in flight while the block waits for it
+      uint4 nw[kPrepChunks];
+#pragma unroll
+      for (int j = 0; j < kPrepChunks; ++j) {
+        const int c0 = (tid + j * kCT) * 8;
+        nw[j] = (Ld.norm_w != nullptr && c0 < P.H) ? *reinterpret_cast<const uint4*>(Ld.norm_w + c0)
+                                                   : make_uint4(0u, 0u, 0u, 0u);
       }
       // ---- input: z = RMSNorm(h_in) or h_in (bf16, shared memory) and its fragments
       {
-        // thread tid holds columns 8*(tid + j*threads) .. +7, j < kPrepChunks
-        constexpr int kCT = kConsumerWarps * 32;
-        constexpr int kPrepChunks = (kMaxHidden + 8 * kCT - 1) / (8 * kCT);
         uint4 hv[kPrepChunks];
-  #pragma unroll
-        for (int j = 0; j < kPrepChunks; ++j) {
-          const int c0 = (tid + j * kCT) * 8;
-          // another block's output when MULTI and cur > 0: read it from L2
-          hv[j] = c0 >= P.H ? make_uint4(0u, 0u, 0u, 0u)
-                  : MULTI   ? __ldcg(reinterpret_cast<const uint4*>(h_in + c0))
-                            : *reinterpret_cast<const uint4*>(h_in + c0);
+        if (!MULTI || cur == 0) {
+#pragma unroll
+          for (int j = 0; j < kPrepChunks; ++j) {
+            const int c0 = (tid + j * kCT) * 8;
+            hv[j] = c0 < P.H ? *reinterpret_cast<const uint4*>(P.h_in + c0) : make_uint4(0u, 0u, 0u, 0u);
+          }
+        } else {
+          // The previous layer's output: tagged words that every block's
+          // combine publishes.  All of a thread's loads are issued before any
+          // tag is examined, and the round is repeated until every tag is the
+          // previous layer's.
+          const uint32_t want = tag - 1u;
+          const uint64_t t0 = gtimer();
+          bool ok = true;
+          for (uint32_t it = 0;; ++it) {
+            ulonglong2 v[kPrepChunks][4];
+#pragma unroll
+            for (int j = 0; j < kPrepChunks; ++j) {
+              const int c0 = min((tid + j * kCT) * 8, P.H - 8);  // past the end: re-read the last chunk, ignored
+#pragma unroll
+              for (int q = 0; q < 4; ++q) v[j][q] = ld_tagged2(P.ws_h + c0 + 2 * q);
+            }
+            bool all = true;
+#pragma unroll
+            for (int j = 0; j < kPrepChunks; ++j) {
+              if ((tid + j * kCT) * 8 < P.H) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) all = all && tagged_tag(v[j][q].x) == want && tagged_tag(v[j][q].y) == want;
+              }
+            }
+            if (all) {
+              // the words hold bf16 values exactly; keep their bf16 bits
+#pragma unroll
+              for (int j = 0; j < kPrepChunks; ++j) {
+                uint32_t hw[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  hw[q] = ((uint32_t)v[j][q].x >> 16) | ((uint32_t)v[j][q].y & 0xFFFF0000u);
+                hv[j] = (tid + j * kCT) * 8 < P.H ? make_uint4(hw[0], hw[1], hw[2], hw[3]) : make_uint4(0u, 0u, 0u, 0u);
+              }
+              break;
+            }
+            if (*abort_flag || gtimer() - t0 > limit) {
+              if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutLayer);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            if (it > 0) __nanosleep(128);
+          }
+          if (consumers_any(!ok || *abort_flag != 0)) break;
         }
         if (Ld.norm_w != nullptr) {
           float ss = 0.f;
-  #pragma unroll
+#pragma unroll
           for (int j = 0; j < kPrepChunks; ++j) {
             const uint32_t hw[4] = {hv[j].x, hv[j].y, hv[j].z, hv[j].w};
-  #pragma unroll
+#pragma unroll
             for (int k = 0; k < 4; ++k) {
               ss = fmaf(bf16lo(hw[k]), bf16lo(hw[k]), ss);
               ss = fmaf(bf16hi(hw[k]), bf16hi(hw[k]), ss);
             }
           }
-  #pragma unroll
+#pragma unroll
           for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
           if (lane == 0) misc->red[warp] = ss;
           asm volatile("bar.sync 1, %0;" ::"r"(kCT) : "memory");
           float tot = 0.f;
           for (int w = 0; w < kConsumerWarps; ++w) tot += misc->red[w];
           const float r = 1.0f / sqrtf(tot / (float)P.H + P.eps);
-  #pragma unroll
+#pragma unroll
           for (int j = 0; j < kPrepChunks; ++j) {
             const int c0 = (tid + j * kCT) * 8;
             if (c0 < P.H) {
-              const uint4 wv = *reinterpret_cast<const uint4*>(Ld.norm_w + c0);
+              const uint4 wv = nw[j];
               const uint32_t hw[4] = {hv[j].x, hv[j].y, hv[j].z, hv[j].w};
               const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
               uint32_t zz[4];
-  #pragma unroll
+#pragma unroll
               for (int k = 0; k < 4; ++k) {
                 const uint32_t lo = f2bf16(bf16lo(hw[k]) * r * bf16lo(ww[k]));
                 const uint32_t hi = f2bf16(bf16hi(hw[k]) * r * bf16hi(ww[k]));
@@ -705,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
           }
         }
-  #pragma unroll
+#pragma unroll
         for (int j = 0; j < kPrepChunks; ++j) {
           const int c0 = (tid + j * kCT) * 8;
           if (c0 < P.H) *reinterpret_cast<uint4*>(zs + c0) = hv[j];
@@ -716,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const int ngz = P.H / kGroup;
           for (int G0 = 4 * warp; G0 < ngz; G0 += 4 * kConsumerWarps) {
             float lo[4], hi[4];
-  #pragma unroll
+#pragma unroll
             for (int k = 0; k < 4; ++k) {
               const uint32_t zz = (G0 + k < ngz) ? *reinterpret_cast<const uint32_t*>(zs + (G0 + k) * kGroup + 2 * lane) : 0u;
               lo[k] = bf16lo(zz);
@@ -755,6 +789,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const uint8_t* stage = smem + P.off_ring + (uint32_t)s * P.stage_bytes;
         const uint32_t t = tasks[i];
         const uint32_t ty = task_type(t), idx = task_idx(t), slot = task_slot(t), c = task_chunk(t);
+        // Past a launch's first layer the shared expert's chunks are already
+        // in shared memory when the layer starts: they wait until this block's
+        // router rows are published, so that the router rows have the SM to
+        // themselves and the chunks fill the logit exchange instead.
+        if (MULTI && cur > 0 && ty != kTaskRouter && my_rrows > 0 &&
+            !__all_sync(0xffffffffu, wait_flag(&misc->rdone, my_rrows, limit, abort_flag))) {
+          if (lane == 0) {
+            if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutRouter);
+            *abort_flag = 1;
+          }
+          break;
+        }
         if (ty == kTaskRouter) {
           const int c0 = (int)c * P.router_part_cols, width = min(P.router_part_cols, P.H - c0);
           float acc = 0.f;
@@ -770,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             acc = fmaf(bf16lo(w.w), bf16lo(z.w), acc);
             acc = fmaf(bf16hi(w.w), bf16hi(z.w), acc);
           }
-  #pragma unroll
+#pragma unroll
           for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
           if (lane == 0) {
             // parts of a row are summed, in part order, by whichever warp ends last
@@ -787,6 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
               // fault injection publishes with a stale tag, so no reader accepts it
               st_tagged(P.ws_logits + e, l, (P.flags & FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE) ? tag - 1u : tag);
               red_relaxed_add(&P.ws->router_cnt, 1u);
+            if (MULTI) atomicAdd(&misc->rdone, 1);
             }
           }
         } else if (ty == kTaskGateUp) {
@@ -854,11 +901,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 // every load is issued before any result is examined: the loads
                 // are volatile, so a check between two of them would wait for
                 // the first one's round trip before issuing the second
-  #pragma unroll
+#pragma unroll
                 for (int k = 0; k < kFetchGroups; ++k)  // past the end: re-read the last group, ignored below
                   v[k] = ld_tagged2(act + min(g0 + k, ge - 1) * kGroup + 2 * lane);
                 bool mine = true;
-  #pragma unroll
+#pragma unroll
                 for (int k = 0; k < kFetchGroups; ++k)
                   if (g0 + k < ge) mine = mine && tagged_tag(v[k].x) == tag && tagged_tag(v[k].y) == tag;
                 if (__all_sync(0xffffffffu, mine)) break;
@@ -873,7 +920,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
               }
               if (!good) break;
               float lo[kFetchGroups], hi[kFetchGroups];
-  #pragma unroll
+#pragma unroll
               for (int k = 0; k < kFetchGroups; ++k) {
                 lo[k] = tagged_value(v[k].x);
                 hi[k] = tagged_value(v[k].y);
@@ -935,25 +982,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       if (MULTI) {
         // all consumer warps are done with this layer's tasks
         if (consumers_any(*abort_flag != 0)) break;
-        uint16_t* h_out = cur == NL - 1 ? P.h_out : P.hbuf[cur & 1];
         if (tid < my_rb * 16) {
-          const int jb = tid / 16, row = tid % 16;
+          const int jb = tid / 16, row = tid % 16, out_row = (first_rb + jb * G) * 16 + row;
           float acc = h_res + ys[(jb * P.n_slots + 0) * 16 + row];
           for (int k = 1; k < P.n_slots; ++k) acc = fmaf(misc->slot_w[k], ys[(jb * P.n_slots + k) * 16 + row], acc);
           const uint16_t o = f2bf16(acc);
-          h_out[(first_rb + jb * G) * 16 + row] = o;
           h_res = bf16f(o);  // the next layer's residual input of this row
+          if (cur == NL - 1)
+            P.h_out[out_row] = o;
+          else
+            st_tagged(P.ws_h + out_row, h_res, tag);
         }
         if (warp == 1) {
           misc->aflag[lane] = 0;
           misc->unit_cnt[lane] = 0;
           misc->dn_cnt[lane] = 0;
           if (lane < 16) misc->rcnt[lane] = 0;
-        }
-        asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
-        if (tid == 0 && cur + 1 < NL) {
-          __threadfence();
-          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&P.ws->layer_cnt) : "memory");
+          if (lane == 0) misc->rdone = 0;
         }
       }
     }
@@ -998,7 +1043,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (old == (uint32_t)G - 1) {
       P.ws->exit_count = 0;
       P.ws->router_cnt = 0;
-      P.ws->layer_cnt = 0;
       for (int k = 0; k < 16; ++k) P.ws->h_cnt[k] = 0;
       P.ws->epoch = misc->tag;
     }

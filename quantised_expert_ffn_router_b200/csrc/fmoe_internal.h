@@ -72,7 +72,6 @@ struct WsHeader {
   uint32_t router_cnt;      // router rows published in this launch (hint for pollers)
   uint32_t h_cnt[16];       // gate/up units published per slot in this launch (hint; cumulative over
                             // the layers of a multi-layer launch)
-  uint32_t layer_cnt;       // blocks done with a layer's combine, cumulative over a multi-layer launch
 };
 static_assert(sizeof(WsHeader) <= 256, "header");
 
@@ -103,7 +102,8 @@ struct Misc {
   int abort;
   uint32_t tag;         // epoch + 1 of this launch
   int n_tasks;          // length of this block's task list
-  int pad[13];
+  int rdone;            // router rows of this block published in the current layer
+  int pad[12];
   int aflag[32];        // per (slot, half) activation fragments: 0 none, 1 building, 2 ready
   int rcnt[16];         // parts finished per router row of this block
   float rpart[16][4];   // partial logits per router row and part
@@ -180,11 +180,12 @@ struct DecodePlan {
   uint64_t timeout_ns;
   int pdl;                 // launched with programmatic stream serialisation
   // multi-layer launch (n_layers > 0): layers 0..n_layers-1 take their weights
-  // from layer_dev[l]; layer 0 reads h_in, the last writes h_out, layer l writes
-  // hbuf[l & 1] in between.  n_layers == 0: one layer from the fields above.
+  // from layer_dev[l]; layer 0 reads h_in, the last writes h_out, and each
+  // layer in between publishes its output as tagged words in ws_h.
+  // n_layers == 0: one layer from the fields above.
   int n_layers;
   const LayerDev* layer_dev;
-  uint16_t* hbuf[2];
+  uint64_t* ws_h;          // [H] tagged
 };
 
 // Ring position of task i: issued by producer lane i % n_issuers into that
