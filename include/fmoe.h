@@ -177,8 +177,13 @@ FMOE_API fmoe_status fmoe_layer_forward(fmoe_ctx* ctx, int32_t layer, const void
 /*
  * Layers layer_begin .. layer_end-1 in sequence (a mixture-of-experts-only
  * stack: each layer's output is the next layer's input), equivalent to
- * chaining fmoe_layer_forward; intermediate activations live in the context
- * workspace.  h_in_dev and h_out_dev (bf16 [T][H]) must not overlap.
+ * chaining fmoe_layer_forward bit for bit; intermediate activations live in
+ * the context workspace.  h_in_dev and h_out_dev (bf16 [T][H]) must not
+ * overlap.  On the batch-1 kernel a range of two or more layers runs as one
+ * launch per token through every layer (the next layer's router rows and
+ * shared expert stream in while a layer finishes); FMOE_FLAG_STACK_PER_LAYER
+ * makes it one launch per layer and token.  The grouped path runs layer by
+ * layer.  Launches are serialised per context, like every call.
  */
 FMOE_API fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer_end, const void* h_in_dev,
                                int32_t T, void* h_out_dev, void* stream);
