@@ -183,7 +183,7 @@ FMOE_API fmoe_status fmoe_layer_forward(fmoe_ctx* ctx, int32_t layer, const void
  * launch per token through every layer (the next layer's router rows and
  * shared expert stream in while a layer finishes); FMOE_FLAG_STACK_PER_LAYER
  * makes it one launch per layer and token.  The grouped path runs layer by
- * layer.  Launches are serialised per context, like every call.
+ * layer.
  */
 FMOE_API fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer_end, const void* h_in_dev,
                                int32_t T, void* h_out_dev, void* stream);
