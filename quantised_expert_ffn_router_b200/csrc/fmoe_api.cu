@@ -169,7 +169,6 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
   nstage = best_ns;
   P.n_issuers = best_ni;
   P.nstage = nstage;
-  P.route_first = kRouteFirst;
   P.off_ring = off;
   off = align_up((uint32_t)(nstage + P.n_down_max) * P.stage_bytes, 128);
   P.off_z = off + r_z;

@@ -601,10 +601,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const int i = r * NI + lane;
         const bool mine = lane < NI && i < ring_end && i >= pre;
         const uint32_t t = mine ? tasks[i] : 0u;
-        // past a launch's first layer the shared expert's chunks stream in
-        // while the previous layer finishes, so they never wait for routing
-        const bool needs_route = mine && P.mode == kModeLayer && !routed && task_type(t) != kTaskRouter &&
-                                 (task_slot(t) >= 1 || (P.route_first && cur == 0));
+        // the shared expert's chunks never wait for routing: they stream in
+        // during routing (and, past a launch's first layer, while the
+        // previous layer finishes)
+        const bool needs_route =
+            mine && P.mode == kModeLayer && !routed && task_type(t) != kTaskRouter && task_slot(t) >= 1;
         int ok = 1;
         if (mine && !needs_route) ok = issue(i, t);
         if (!__all_sync(0xffffffffu, ok)) break;
@@ -789,11 +790,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const uint8_t* stage = smem + P.off_ring + (uint32_t)s * P.stage_bytes;
         const uint32_t t = tasks[i];
         const uint32_t ty = task_type(t), idx = task_idx(t), slot = task_slot(t), c = task_chunk(t);
-        // Past a launch's first layer the shared expert's chunks are already
-        // in shared memory when the layer starts: they wait until this block's
+        // The shared expert's chunks arrive with the router rows (or before
+        // them, past a launch's first layer): they wait until this block's
         // router rows are published, so that the router rows have the SM to
-        // themselves and the chunks fill the logit exchange instead.
-        if (MULTI && cur > 0 && ty != kTaskRouter && my_rrows > 0 &&
+        // themselves and the chunks fill the logit exchange instead.  (In a
+        // multi-layer launch's first layer the wait measured slower.)
+        if (P.mode == kModeLayer && (!MULTI || cur > 0) && ty != kTaskRouter && my_rrows > 0 &&
             !__all_sync(0xffffffffu, wait_flag(&misc->rdone, my_rrows, limit, abort_flag))) {
           if (lane == 0) {
             if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutRouter);
@@ -833,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
               // fault injection publishes with a stale tag, so no reader accepts it
               st_tagged(P.ws_logits + e, l, (P.flags & FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE) ? tag - 1u : tag);
               red_relaxed_add(&P.ws->router_cnt, 1u);
-            if (MULTI) atomicAdd(&misc->rdone, 1);
+            atomicAdd(&misc->rdone, 1);
             }
           }
         } else if (ty == kTaskGateUp) {

@@ -44,7 +44,6 @@ constexpr int kStaticRouteLogits = 32768; // fp32 logits in the fixed scratch of
 constexpr int kStaticRouteMaxTokens = 4096;  // tokens per fmoe_route_static call
 constexpr int kMaxDevices = 64;          // devices fmoe_route_static caches a scratch address for
 constexpr int kMinRingStages = 20;       // ring stages kept when down jobs get stages of their own
-constexpr int kRouteFirst = 1;          // see DecodePlan::route_first
 constexpr int kFetchGroups = 8;          // activation groups a warp fetches per round trip
 
 inline __host__ __device__ int tile_code_bytes(int bits) { return 16 * kGroup * bits / 8; }
@@ -143,7 +142,6 @@ struct DecodePlan {
   int nstage;              // ring stages for router and gate/up tasks (a multiple of n_issuers)
   int n_down_max;          // stages after the ring, one per down job (filled once per launch)
   int n_issuers;           // producer lanes issuing copies; lane l owns stages l, l+n_issuers, ...
-  int route_first;         // 1: route before issuing any expert copy (keeps the logit exchange off a busy memory pipe)
   uint32_t stage_bytes;
   // shared-memory layout (byte offsets)
   uint32_t off_ring;
