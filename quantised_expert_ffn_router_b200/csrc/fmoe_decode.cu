@@ -20,12 +20,13 @@
 // HBM -> shared memory with bulk-async (TMA) copies into a ring of stages
 // (full/empty mbarriers); it also waits (bounded) for every block's router
 // rows and runs softmax + top-K itself before the first task that needs a
-// routed expert.  Sixteen consumer warps take tasks round-robin and never wait
+// routed expert.  Fifteen consumer warps take tasks round-robin and never wait
 // for each other: K-chunks of a unit are summed by whichever warp finishes
 // last (shared-memory counter, fixed order), which writes a = silu(g)*u and
-// publishes the unit with a release counter; a down job waits (bounded) for its
-// expert's activations to be published by every block, turns them into
-// fragments once per block and reduces its rows.
+// publishes the unit's values as tagged words (plus a relaxed count that
+// paces readers); a down job waits (bounded) for its expert's activations to
+// be published by every block, turns them into fragments once per block and
+// reduces its rows.
 //
 // Inner loop.  A tile is 16 rows x 64 columns (one quantisation group per
 // row); its codes go into mma.sync fragments exactly (lop3 into the mantissa
