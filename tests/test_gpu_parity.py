@@ -130,6 +130,33 @@ def test_layer_forward_matches_oracle(torch, wl):
         _check_layer(torch, m, wl, 0, x, T)
 
 
+# more experts than one lane-per-16-entries pass covers (the fused kernel's
+# top-K then runs in passes); 2048 is above the grouped path's limit, so T >= 8
+# runs token by token there
+MANY_E = [dataclasses.replace(TINY, name="experts1000", n_experts=1000, top_k=4, seed=15),
+          dataclasses.replace(TINY, name="experts2048k8", n_experts=2048, top_k=8, seed=16)]
+
+
+@pytest.mark.parametrize("wl", MANY_E, ids=lambda w: w.name)
+def test_many_experts_match_oracle(torch, wl):
+    for T in (3, 8):
+        _, _, x = _tokens(wl, T, start=80)
+        with Model(wl) as m:
+            _check_layer(torch, m, wl, 0, x, T)
+            idx = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+            w = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+            m.fm.fmoe_route(m.ctx, 0, x.data_ptr(), T, idx.data_ptr(), w.data_ptr(), m.stream)
+            st, word = m.fm.fmoe_poll_status(m.ctx, m.stream)
+            assert st == 0, hex(word)
+            gi, gw = idx.cpu().numpy(), w.cpu().numpy()
+        ol = OracleLayer(wl, 0)
+        xb = bf16_tensor_bits(x)
+        for t in range(T):
+            r = ol.forward(xb[t])
+            assert list(gi[t]) == list(r["idx"]), (T, t)
+            assert np.max(np.abs(gw[t] - r["w"])) <= W_TOL, (T, t)
+
+
 def test_layer_equals_sum_of_route_and_experts(torch):
     """layer(h) = bf16(h + y_shared + sum_k w_k y_k) using the library's own
     route and expert calls (fp32, same accumulation order)."""
