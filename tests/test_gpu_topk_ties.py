@@ -25,6 +25,10 @@ CASES = [
     dataclasses.replace(TINY, name="ties37", n_experts=37, top_k=3, zipf=1.0, seed=32),
     dataclasses.replace(TINY, name="ties512", n_experts=512, top_k=4, zipf=1.0, seed=33),
     dataclasses.replace(TINY, name="ties512k8", n_experts=512, top_k=8, zipf=1.0, seed=34),
+    # above 512 experts the fused kernel selects in passes over the logits; above
+    # 1023 the grouped path is not available and T >= 8 runs token by token
+    dataclasses.replace(TINY, name="ties1000", n_experts=1000, top_k=4, zipf=1.0, seed=35),
+    dataclasses.replace(TINY, name="ties2048k8", n_experts=2048, top_k=8, zipf=1.0, seed=36),
 ]
 
 
