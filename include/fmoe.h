@@ -189,6 +189,26 @@ FMOE_API fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int3
                                int32_t T, void* h_out_dev, void* stream);
 
 /*
+ * fmoe_layer_forward / fmoe_stack_forward on HOST buffers: h_in_host (bf16
+ * [T][H]) is copied into the context's device staging buffer, the device path
+ * runs on it, and h_out_host (bf16 [T][H]) and, when not NULL, idx_out_host
+ * (int32 [T][K]) and w_out_host (fp32 [T][K]) are copied back.  Everything is
+ * enqueued on `stream` with one cudaMemcpyAsync per buffer and the call
+ * returns without synchronising; the caller synchronises `stream` before
+ * reading the outputs and keeps the buffers alive until then.  Page-locked
+ * buffers (cudaHostAlloc / cudaHostRegister) keep the copies asynchronous;
+ * pageable ones work but their copies block the host.  The staging buffers
+ * are per context, so h_in_host and h_out_host may be the same buffer.
+ * Results are bit-identical to the device-pointer calls.  Errors: as the
+ * device-pointer calls (no alignment rule on host buffers), FMOE_ERR_CUDA when
+ * a copy cannot be enqueued.
+ */
+FMOE_API fmoe_status fmoe_layer_forward_host(fmoe_ctx* ctx, int32_t layer, const void* h_in_host, int32_t T,
+                                             void* h_out_host, int32_t* idx_out_host, float* w_out_host, void* stream);
+FMOE_API fmoe_status fmoe_stack_forward_host(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer_end,
+                                             const void* h_in_host, int32_t T, void* h_out_host, void* stream);
+
+/*
  * Writes expert `expert` (-1: shared) of `layer` back in the canonical format
  * into dst_dev (fmoe_expert_bytes bytes).  Used to check the packed layout
  * round trip.

@@ -19,7 +19,7 @@ __all__ = [
     "FMOE_ERR_OOM", "FMOE_ERR_TIMEOUT", "FMOE_FLAG_FORCE_PER_TOKEN", "FMOE_FLAG_FORCE_GROUPED", "FMOE_FLAG_STACK_PER_LAYER",
     "FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE", "Config", "LayerDesc", "FmoeError", "lib", "fmoe_expert_bytes",
     "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward", "fmoe_layer_forward", "fmoe_stack_forward",
-    "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error", "EXPORTED_SYMBOLS",
+    "fmoe_layer_forward_host", "fmoe_stack_forward_host", "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error", "EXPORTED_SYMBOLS",
 ]
 
 FMOE_OK, FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED, FMOE_ERR_ALIGNMENT = 0, 1, 2, 3
@@ -30,7 +30,8 @@ FMOE_FLAG_STACK_PER_LAYER = 0x4
 FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE = 0x100
 
 EXPORTED_SYMBOLS = ["fmoe_expert_bytes", "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward",
-                    "fmoe_layer_forward", "fmoe_stack_forward", "fmoe_unpack_expert", "fmoe_requant_4to2", "fmoe_set_gemm_events",
+                    "fmoe_layer_forward", "fmoe_stack_forward", "fmoe_layer_forward_host", "fmoe_stack_forward_host",
+                    "fmoe_unpack_expert", "fmoe_requant_4to2", "fmoe_set_gemm_events",
                     "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error"]
 
 
@@ -76,6 +77,8 @@ def lib():
             L.fmoe_expert_forward.argtypes = [P, i32, i32, P, i32, P, P]
             L.fmoe_layer_forward.argtypes = [P, i32, P, i32, P, P, P, P]
             L.fmoe_stack_forward.argtypes = [P, i32, i32, P, i32, P, P]
+            L.fmoe_layer_forward_host.argtypes = [P, i32, P, i32, P, P, P, P]
+            L.fmoe_stack_forward_host.argtypes = [P, i32, i32, P, i32, P, P]
             L.fmoe_unpack_expert.argtypes = [P, i32, i32, P, P]
             L.fmoe_poll_status.argtypes = [P, P, ctypes.POINTER(u32)]
             L.fmoe_set_gemm_events.argtypes = [P, P]
@@ -84,7 +87,8 @@ def lib():
             L.fmoe_last_error.argtypes = [P]
             L.fmoe_last_error.restype = ctypes.c_char_p
             for name in ("fmoe_create", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
-                         "fmoe_stack_forward", "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy"):
+                         "fmoe_stack_forward", "fmoe_layer_forward_host", "fmoe_stack_forward_host",
+                         "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -143,6 +147,21 @@ def fmoe_layer_forward(ctx, layer, h_in_dev, T, h_out_dev, idx_out_dev=None, w_o
 
 def fmoe_stack_forward(ctx, layer_begin, layer_end, h_in_dev, T, h_out_dev, stream=0, *, check=True) -> int:
     st = lib().fmoe_stack_forward(_vp(ctx), layer_begin, layer_end, _vp(h_in_dev), T, _vp(h_out_dev), _vp(stream))
+    return _check(ctx, st) if check else st
+
+
+def fmoe_layer_forward_host(ctx, layer, h_in_host, T, h_out_host, idx_out_host=None, w_out_host=None, stream=0, *,
+                            check=True) -> int:
+    """fmoe_layer_forward on host buffers (addresses of page-locked memory)."""
+    st = lib().fmoe_layer_forward_host(_vp(ctx), layer, _vp(h_in_host), T, _vp(h_out_host), _vp(idx_out_host),
+                                       _vp(w_out_host), _vp(stream))
+    return _check(ctx, st) if check else st
+
+
+def fmoe_stack_forward_host(ctx, layer_begin, layer_end, h_in_host, T, h_out_host, stream=0, *, check=True) -> int:
+    """fmoe_stack_forward on host buffers (addresses of page-locked memory)."""
+    st = lib().fmoe_stack_forward_host(_vp(ctx), layer_begin, layer_end, _vp(h_in_host), T, _vp(h_out_host),
+                                       _vp(stream))
     return _check(ctx, st) if check else st
 
 

@@ -31,6 +31,10 @@ struct fmoe_ctx {
   uint16_t* stack_buf[2] = {nullptr, nullptr};  // ping-pong activations, [max_tokens][H] bf16
   LayerDev* layer_dev = nullptr;                // device [n_layers]: weights of every layer (multi-layer launches)
   uint64_t* hwords = nullptr;                   // device [H] tagged: a multi-layer launch's intermediate outputs
+  uint16_t* io_in = nullptr;                    // device staging of the *_host calls: [max_tokens][H] bf16 in,
+  uint16_t* io_out = nullptr;                   //   [max_tokens][H] bf16 out,
+  int32_t* io_idx = nullptr;                    //   [max_tokens][K] expert indices,
+  float* io_w = nullptr;                        //   [max_tokens][K] weights
   void* bws_mem = nullptr;  // batched-path workspace (max_tokens > 1)
   BatchWs bws{};
   std::vector<TmaDesc> tc_maps;  // per layer: tensor maps of the packed gate/up and down matrices
@@ -353,7 +357,7 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   }
 
   // workspace: header | logits [E] | activations [kMaxSlots][I] | task lists | 2 x [max_tokens][H] bf16 |
-  // per-layer weight table | tagged layer outputs [H]
+  // per-layer weight table | tagged layer outputs [H] | staging of the host-buffer calls
   size_t off = 256;
   size_t off_logits = off;
   off += ((size_t)c.n_experts * 8 + 255) / 256 * 256;
@@ -370,6 +374,15 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   off += ((size_t)c.n_layers * sizeof(LayerDev) + 255) / 256 * 256;
   size_t off_hwords = off;
   off += ((size_t)c.hidden * 8 + 255) / 256 * 256;
+  const size_t io_rows = (size_t)std::max(c.max_tokens, 1);
+  size_t off_io_in = off;
+  off += (io_rows * c.hidden * 2 + 255) / 256 * 256;
+  size_t off_io_out = off;
+  off += (io_rows * c.hidden * 2 + 255) / 256 * 256;
+  size_t off_io_idx = off;
+  off += (io_rows * c.top_k * 4 + 255) / 256 * 256;
+  size_t off_io_w = off;
+  off += (io_rows * c.top_k * 4 + 255) / 256 * 256;
   ctx->ws_bytes = off;
   e = cudaMalloc(&ctx->ws, ctx->ws_bytes);
   if (e != cudaSuccess) {
@@ -387,6 +400,10 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   ctx->stack_buf[1] = reinterpret_cast<uint16_t*>(base + off_stack + stack_bytes);
   ctx->layer_dev = reinterpret_cast<LayerDev*>(base + off_layers);
   ctx->hwords = reinterpret_cast<uint64_t*>(base + off_hwords);
+  ctx->io_in = reinterpret_cast<uint16_t*>(base + off_io_in);
+  ctx->io_out = reinterpret_cast<uint16_t*>(base + off_io_out);
+  ctx->io_idx = reinterpret_cast<int32_t*>(base + off_io_idx);
+  ctx->io_w = reinterpret_cast<float*>(base + off_io_w);
   // batched path: sized for max_tokens, only when more than one token is allowed
   const bool grouped_ok = c.n_experts <= kBatchMaxExperts && c.max_tokens <= kBatchMaxTokens;
   if ((c.flags & FMOE_FLAG_FORCE_GROUPED) && !grouped_ok)
@@ -645,18 +662,9 @@ fmoe_status fmoe_layer_forward(fmoe_ctx* ctx, int32_t layer, const void* h_in_de
                       idx_out_dev, w_out_dev, stream);
 }
 
-fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer_end, const void* h_in_dev, int32_t T,
-                               void* h_out_dev, void* stream) {
-  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
-  if (layer_begin < 0 || layer_end > ctx->cfg.n_layers || layer_begin >= layer_end)
-    return fail(ctx, FMOE_ERR_INVALID_ARG, "layer range [%d, %d) invalid", layer_begin, layer_end);
-  fmoe_status s = check_ctx_layer(ctx, layer_begin, T);
-  if (s != FMOE_OK) return s;
-  if (T == 0) return FMOE_OK;
-  if (!h_in_dev || !h_out_dev) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL tensor");
-  if (misaligned(h_in_dev) || misaligned(h_out_dev)) return fail(ctx, FMOE_ERR_ALIGNMENT, "tensor not 16-byte aligned");
-  const size_t bytes = (size_t)T * ctx->cfg.hidden * 2;
-  if (overlaps(h_in_dev, bytes, h_out_dev, bytes)) return fail(ctx, FMOE_ERR_INVALID_ARG, "h_out overlaps h_in");
+static fmoe_status stack_tokens(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer_end, const void* h_in_dev,
+                                int32_t T, void* h_out_dev, void* stream) {
+  fmoe_status s = FMOE_OK;
   const int n_layers = layer_end - layer_begin;
   if (n_layers > 1 && !use_batched(ctx, T) && !(ctx->cfg.flags & FMOE_FLAG_STACK_PER_LAYER)) {
     // one launch per token runs every layer of the range
@@ -681,6 +689,71 @@ fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer
     cur = dst;
   }
   return FMOE_OK;
+}
+
+static fmoe_status check_stack_range(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer_end, int32_t T) {
+  if (layer_begin < 0 || layer_end > ctx->cfg.n_layers || layer_begin >= layer_end)
+    return fail(ctx, FMOE_ERR_INVALID_ARG, "layer range [%d, %d) invalid", layer_begin, layer_end);
+  return check_ctx_layer(ctx, layer_begin, T);
+}
+
+fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer_end, const void* h_in_dev, int32_t T,
+                               void* h_out_dev, void* stream) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  fmoe_status s = check_stack_range(ctx, layer_begin, layer_end, T);
+  if (s != FMOE_OK) return s;
+  if (T == 0) return FMOE_OK;
+  if (!h_in_dev || !h_out_dev) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL tensor");
+  if (misaligned(h_in_dev) || misaligned(h_out_dev)) return fail(ctx, FMOE_ERR_ALIGNMENT, "tensor not 16-byte aligned");
+  const size_t bytes = (size_t)T * ctx->cfg.hidden * 2;
+  if (overlaps(h_in_dev, bytes, h_out_dev, bytes)) return fail(ctx, FMOE_ERR_INVALID_ARG, "h_out overlaps h_in");
+  return stack_tokens(ctx, layer_begin, layer_end, h_in_dev, T, h_out_dev, stream);
+}
+
+// Host-buffer variants: the input is copied into the context's staging buffer,
+// the device path runs on it, and the results are copied back, all enqueued
+// on `stream` (plain cudaMemcpyAsync, one per buffer).
+static fmoe_status copy_async(fmoe_ctx* ctx, void* dst, const void* src, size_t bytes, cudaMemcpyKind kind,
+                              void* stream) {
+  if (bytes == 0) return FMOE_OK;
+  cudaError_t e = cudaMemcpyAsync(dst, src, bytes, kind, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(ctx, e, kind == cudaMemcpyHostToDevice ? "host-to-device copy" : "device-to-host copy");
+  }
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_layer_forward_host(fmoe_ctx* ctx, int32_t layer, const void* h_in_host, int32_t T, void* h_out_host,
+                                    int32_t* idx_out_host, float* w_out_host, void* stream) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  fmoe_status s = check_ctx_layer(ctx, layer, T);
+  if (s != FMOE_OK) return s;
+  if (T == 0) return FMOE_OK;
+  if (!h_in_host || !h_out_host) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL buffer");
+  const size_t bytes = (size_t)T * ctx->cfg.hidden * 2, kbytes = (size_t)T * ctx->cfg.top_k * 4;
+  s = copy_async(ctx, ctx->io_in, h_in_host, bytes, cudaMemcpyHostToDevice, stream);
+  if (s == FMOE_OK)
+    s = layer_tokens(ctx, layer, ctx->io_in, T, ctx->io_out, idx_out_host ? ctx->io_idx : nullptr,
+                     w_out_host ? ctx->io_w : nullptr, stream);
+  if (s == FMOE_OK) s = copy_async(ctx, h_out_host, ctx->io_out, bytes, cudaMemcpyDeviceToHost, stream);
+  if (s == FMOE_OK && idx_out_host) s = copy_async(ctx, idx_out_host, ctx->io_idx, kbytes, cudaMemcpyDeviceToHost, stream);
+  if (s == FMOE_OK && w_out_host) s = copy_async(ctx, w_out_host, ctx->io_w, kbytes, cudaMemcpyDeviceToHost, stream);
+  return s;
+}
+
+fmoe_status fmoe_stack_forward_host(fmoe_ctx* ctx, int32_t layer_begin, int32_t layer_end, const void* h_in_host,
+                                    int32_t T, void* h_out_host, void* stream) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  fmoe_status s = check_stack_range(ctx, layer_begin, layer_end, T);
+  if (s != FMOE_OK) return s;
+  if (T == 0) return FMOE_OK;
+  if (!h_in_host || !h_out_host) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL buffer");
+  const size_t bytes = (size_t)T * ctx->cfg.hidden * 2;
+  s = copy_async(ctx, ctx->io_in, h_in_host, bytes, cudaMemcpyHostToDevice, stream);
+  if (s == FMOE_OK) s = stack_tokens(ctx, layer_begin, layer_end, ctx->io_in, T, ctx->io_out, stream);
+  if (s == FMOE_OK) s = copy_async(ctx, h_out_host, ctx->io_out, bytes, cudaMemcpyDeviceToHost, stream);
+  return s;
 }
 
 fmoe_status fmoe_unpack_expert(fmoe_ctx* ctx, int32_t layer, int32_t expert, void* dst_dev, void* stream) {

@@ -101,6 +101,8 @@ def test_calls_on_invalid_context_fail_cleanly():
     assert fm.fmoe_route(bogus, 0, 0x1000, 1, 0x2000, 0x3000, check=False) == fm.FMOE_ERR_INVALID_ARG
     assert fm.fmoe_expert_forward(bogus, 0, 0, 0x1000, 1, 0x2000, check=False) == fm.FMOE_ERR_INVALID_ARG
     assert fm.fmoe_stack_forward(bogus, 0, 1, 0x1000, 1, 0x2000, check=False) == fm.FMOE_ERR_INVALID_ARG
+    assert fm.fmoe_layer_forward_host(bogus, 0, 0x1000, 1, 0x2000, check=False) == fm.FMOE_ERR_INVALID_ARG
+    assert fm.fmoe_stack_forward_host(bogus, 0, 1, 0x1000, 1, 0x2000, check=False) == fm.FMOE_ERR_INVALID_ARG
     assert fm.fmoe_unpack_expert(bogus, 0, 0, 0x1000, check=False) == fm.FMOE_ERR_INVALID_ARG
     assert fm.fmoe_poll_status(bogus)[0] == fm.FMOE_ERR_INVALID_ARG
     assert fm.fmoe_destroy(bogus) == fm.FMOE_ERR_INVALID_ARG
