@@ -538,10 +538,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // lane, each lane refilling only its own stages), in rounds of n_issuers
     // consecutive tasks.  Within a round, tasks that need no routing go first,
     // so a round holding this block's own router rows never waits on routing.
-    const int NI = P.n_issuers;
+    const int NI = P.n_issuers, per_lane = P.nstage / NI;
+    // this lane's next ring position (its copies of the block's router rows
+    // issued during set-up took the first one)
+    int ring_slot = 0, ring_fill = 0;
+    if (lane < pre_issued) ring_advance(per_lane, ring_slot, ring_fill);
     auto issue = [&](int i, uint32_t t) -> int {
       int s, fill;
-      task_stage_of(P.nstage, NI, n_tasks, n_down, i, s, fill, cur);
+      if (i < n_tasks - n_down) {
+        s = ring_slot * NI + lane;
+        fill = ring_fill;
+        ring_advance(per_lane, ring_slot, ring_fill);
+      } else {
+        s = P.nstage + (i - (n_tasks - n_down));
+        fill = cur;
+      }
       if (fill > 0 && !wait_mbar(bar_empty + 8u * s, (uint32_t)((fill - 1) & 1), limit, abort_flag)) {
         if (!*abort_flag) atomicOr(&P.ws->status, kStatusTimeoutTma);
         *abort_flag = 1;

@@ -195,6 +195,17 @@ inline __host__ __device__ void task_stage(int nstage, int n_issuers, int i, int
   fill = j / L;
 }
 
+// The same positions, followed one issue at a time by the producer lane that
+// owns them: its next ring task goes to stage slot * n_issuers + lane as fill
+// `fill`; ring_advance moves to the lane's next stage (nstage / n_issuers of
+// them, used round-robin).
+inline __host__ __device__ void ring_advance(int per_lane, int& slot, int& fill) {
+  if (++slot == per_lane) {
+    slot = 0;
+    ++fill;
+  }
+}
+
 // Stage and fill of task i of layer l (0 for a single-layer launch) of a block
 // whose last n_down tasks are its down jobs: those sit in dedicated stages after
 // the ring (one fill per layer), the other tasks cycle through the ring.  Layer

@@ -7,8 +7,10 @@ consumers wait for a stage's phase by parity, which is only unambiguous if
 every stage is refilled in order, by one lane, with fills 0, 1, 2, ... and
 no two tasks of a layer share a (stage, fill).  A small host program (built
 with nvcc, no GPU needed) walks the issue order of many plan shapes for
-several layers and checks exactly that, plus that down jobs keep their own
-stages (fill = layer) and that layer 0 maps like a single-layer launch.
+several layers and checks exactly that.  It also checks that down jobs keep
+their own stages (fill = layer), that layer 0 maps like a single-layer launch,
+and that the per-lane counters the producer keeps (ring_advance) give the same
+positions at every issue.
 """
 import os
 import shutil
@@ -34,14 +36,21 @@ int main() {
         for (int n_down = 0; n_down < n_tasks && n_down <= 32; n_down += (n_down < 12 ? 1 : 5)) {
           const int ring_end = n_tasks - n_down, n_layers = 5;
           std::vector<int> next_fill(nstage + n_down, 0), owner(nstage + n_down, -1);
+          // the producer's per-lane counters (ring_advance), one pair per lane
+          std::vector<int> lane_slot(ni, 0), lane_fill(ni, 0);
           for (int l = 0; l < n_layers; ++l) {
-            std::vector<int> seen((nstage + n_down) * (n_layers * 100 + 1), 0);
             // issue order: rounds of ni consecutive tasks, lanes in parallel;
             // per lane the order is its tasks in increasing index
             for (int lane = 0; lane < ni; ++lane)
               for (int i = lane; i < ring_end; i += ni) {
                 int s, f;
                 task_stage_of(nstage, ni, n_tasks, n_down, i, s, f, l);
+                if (lane_slot[lane] * ni + lane != s || lane_fill[lane] != f) {
+                  printf("FAIL counters disagree ni=%d nstage=%d tasks=%d down=%d l=%d i=%d\n", ni, nstage, n_tasks,
+                         n_down, l, i);
+                  return 1;
+                }
+                ring_advance(per, lane_slot[lane], lane_fill[lane]);
                 if (s < 0 || s >= nstage || s % ni != lane) {
                   printf("FAIL stage range/owner ni=%d nstage=%d tasks=%d down=%d l=%d i=%d s=%d\n", ni, nstage,
                          n_tasks, n_down, l, i, s);
