@@ -144,6 +144,17 @@ def test_topk_agrees_with_full_sort():
         assert abs(w.sum() - 1.0) < 1e-12
 
 
+def test_topk_signed_zeros_tie_by_index():
+    """-0 and +0 logits are equal, so they break by the lower index like any tie
+    (the reading both sides take; the kernels map -0 to +0 before ranking)."""
+    logits = np.array([-1.0, -0.0, 0.0, -0.0, 0.0, -2.0], dtype=np.float32)
+    idx, w, _ = oracle.topk(logits, 4)
+    assert list(idx) == [1, 2, 3, 4]
+    np.testing.assert_allclose(w, [0.25] * 4, rtol=0, atol=1e-15)
+    idx, _, _ = oracle.topk(-logits[::-1].copy(), 3)  # [2, -0, 0, -0, 0, 1]: 2, 1, then the lowest-index zero
+    assert list(idx) == [0, 5, 1]
+
+
 def test_topk_weights_full_softmax_when_k_equals_e():
     rng = np.random.default_rng(1)
     logits = (rng.standard_normal(32) * 3).astype(np.float32)
