@@ -168,8 +168,10 @@ FMOE_API fmoe_status fmoe_expert_forward(fmoe_ctx* ctx, int32_t layer, int32_t e
  * with z, idx, w as in fmoe_route, accumulated in fp32 and rounded once to bf16.
  *   h_in_dev, h_out_dev : bf16 [T][H], must not overlap;
  *   idx_out_dev (int32 [T][K]) and w_out_dev (fp32 [T][K]) may be NULL.
- * T == 1 runs the fused single-token kernel; T > 1 the grouped batched path
- * (see FMOE_FLAG_*).  T == 0 is a no-op.  Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ * T < 8 runs the fused single-token kernel once per token; T >= 8 the grouped
+ * batched path when the context has one (n_experts <= 1023, max_tokens <=
+ * 16320), else the single-token kernel per token (see FMOE_FLAG_*).  T == 0
+ * is a no-op.  Errors: INVALID_ARG, ALIGNMENT, CUDA.
  */
 FMOE_API fmoe_status fmoe_layer_forward(fmoe_ctx* ctx, int32_t layer, const void* h_in_dev, int32_t T, void* h_out_dev,
                                int32_t* idx_out_dev, float* w_out_dev, void* stream);
