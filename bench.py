@@ -7,7 +7,7 @@ affine codes with bf16 scale/bias, bf16 router N(0, 0.02) -- decoding 1000
 seeded tokens x ~ N(0, 1) one at a time.  One step = one token through the
 whole hot path (router GEMV, softmax, top-K, K+1 dequantising SwiGLU experts,
 combine) = one fused kernel launch.  The weights stay resident in HBM; L2 is
-flushed (a 256 MB write) before every timed step, so the router and shared
+flushed (a 256 MB write, then a 256 MB read) before every timed step, so the router and shared
 expert are read from HBM as they would be inside a multi-layer model; each
 step is timed with CUDA events on the launching stream and the flush is not.
 
@@ -126,6 +126,21 @@ class ClockSampler(threading.Thread):
                 "reasons": sorted(reasons), "samples": len(self.samples)}
 
 
+class Flush:
+    """Evicts L2 (126 MB on B200) between timed steps: a 256 MB write, then a
+    256 MB read of another buffer, so the timed kernel finds neither its own
+    weights in L2 nor the write's dirty lines (which a real decode step, whose
+    neighbours mostly read weights, would not leave behind either)."""
+
+    def __init__(self, torch):
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        self.r = torch.zeros(64 << 20, dtype=torch.int32, device="cuda")
+
+    def __call__(self, i):
+        self.w.fill_(i & 0xFF)
+        self.r.max()
+
+
 # ----------------------------------------------------------------------------- oracle (CPU)
 
 
@@ -215,7 +230,7 @@ def config_dict(wl, flushed, cpu=False):
             "layers": wl.n_layers, "tokens": wl.tokens * (wl.steps if batched else 1),
             "batch": wl.tokens if batched else 1, "norm": wl.norm,
             **({"router_bias": f"Zipf(s={wl.zipf}) over a seeded expert ranking"} if wl.zipf else {}),
-            "l2": "n/a (CPU oracle)" if cpu else ("flushed (256 MB write) before every timed step" if flushed else
+            "l2": "n/a (CPU oracle)" if cpu else ("flushed (256 MB write + 256 MB read) before every timed step" if flushed else
                                                   "per-step weight traffic far above L2 (no flush)"),
             "parallelism": "replicas"}
 
@@ -292,11 +307,11 @@ def run_gpu(args, wl, ws, rank, local):
                                   None, sp)
 
     # a batched step streams ~0.5 GB of expert weights, far above L2: no flush
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if not (stacked or batched) else None
+    flush = Flush(torch) if not (stacked or batched) else None
 
     def maybe_flush(i):
         if flush is not None:
-            flush.fill_(i & 0xFF)
+            flush(i)
 
     steps, warmup = args.steps, args.warmup
     for i in range(warmup):
@@ -451,6 +466,90 @@ def run_gpu(args, wl, ws, rank, local):
     return 0
 
 
+# phase timestamps the trace build records per block and layer (fmoe_set_trace)
+TRACE_POINTS = [(0, "start"), (1, "router copies issued"), (2, "input z ready"),
+                (7, "block's router rows published"), (14, "block's shared units published"),
+                (3, "every logit seen (producer)"), (4, "top-K done"), (5, "first routed copy issued"),
+                (6, "every gate/up copy issued"), (8, "first routed gate/up chunk started"),
+                (9, "block's last routed unit published"), (15, "first down job started"),
+                (10, "first activations current"), (11, "last down job done"), (12, "combine done"),
+                (13, "block exit")]
+
+
+def run_trace(args, wl):
+    """Per-phase timeline of the fused kernel from the trace build: for each
+    recorded point, the median over steps of its median and latest time over
+    blocks, in microseconds after the earliest block start of the launch."""
+    import numpy as np
+    import torch
+
+    import quantised_expert_ffn_router_b200 as fm
+    from synth.gpu import DeviceWeights, tokens
+    fm.use_trace_build()
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    weights = DeviceWeights(wl)
+    L = wl.n_layers
+    cfg = fm.Config(wl.hidden, wl.n_experts, wl.top_k, wl.inter, wl.bits, 64, L, 1, wl.rms_eps, 0, 0)
+    _, ctx = fm.fmoe_create(cfg, [fm.LayerDesc(**d) for d in weights.descs()], sp)
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    NP, NLt = fm.fmoe_trace_points(), fm.fmoe_trace_layers()
+    buf = torch.zeros((n_sm, NLt, NP), dtype=torch.int64, device="cuda")
+    fm.fmoe_set_trace(ctx, buf.data_ptr())
+    n_tok = min(wl.tokens, 64)
+    X = tokens(wl, range(n_tok))
+    OUT = torch.empty_like(X)
+    flush = Flush(torch) if L == 1 else None
+    steps, warmup = args.steps, args.warmup
+    recs = []
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    event_us = []
+    for i in range(warmup + steps):
+        if flush is not None:
+            flush(i)
+        buf.zero_()
+        ev0.record(stream)
+        if L > 1:
+            fm.fmoe_stack_forward(ctx, 0, L, X[i % n_tok].data_ptr(), 1, OUT[i % n_tok].data_ptr(), sp)
+        else:
+            fm.fmoe_layer_forward(ctx, 0, X[i % n_tok].data_ptr(), 1, OUT[i % n_tok].data_ptr(), None, None, sp)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if i >= warmup:
+            recs.append(buf.cpu().numpy().astype(np.float64))
+            event_us.append(1e3 * ev0.elapsed_time(ev1))
+    st, word = fm.fmoe_poll_status(ctx, sp)
+    fm.fmoe_destroy(ctx)
+    if st != 0:
+        raise RuntimeError(f"device status 0x{word:x}")
+    table = {}
+    for layer in range(min(L, NLt)):
+        rows = []
+        for k, name in TRACE_POINTS:
+            if k == 13 and layer > 0:
+                continue
+            med, late = [], []
+            for r in recs:
+                t0 = r[:, 0, 0][r[:, 0, 0] > 0].min()
+                v = r[:, layer if k != 13 else 0, k]
+                v = v[v > 0]
+                if v.size:
+                    med.append((np.median(v) - t0) / 1e3)
+                    late.append((v.max() - t0) / 1e3)
+            if med:
+                rows.append({"point": name, "median_us": round(float(np.median(med)), 3),
+                             "latest_us": round(float(np.median(late)), 3), "blocks": int(v.size)})
+        table[f"layer{layer}"] = rows
+    for layer, rows in table.items():
+        print(f"# {wl.name} {layer}: median over {steps} launches (event time {statistics.median(event_us):.2f} us)")
+        for r in rows:
+            print(f"#   {r['point']:<48s} median block {r['median_us']:8.3f} us   latest block {r['latest_us']:8.3f} us")
+    print(json.dumps({"trace": wl.name, "steps": steps, "event_us_median": statistics.median(event_us),
+                      "phases": table}), flush=True)
+    return 0
+
+
 # fp32/integer operations per weight of the requantisation kernel: code
 # extraction, int-to-float and fma in both passes, min/max, subtract, multiply,
 # round, clamp and packing
@@ -515,10 +614,15 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stack-per-layer", action="store_true",
                     help="stacks: one launch per layer instead of one per token (the multi-layer kernel)")
+    ap.add_argument("--trace", action="store_true",
+                    help="per-phase timeline of the fused kernel from the trace build (not a bench line)")
     args = ap.parse_args(argv)
     if args.workload == "requant":
         return run_requant(args)
     wl = synth.WORKLOADS[args.workload]
+    if args.trace:
+        args.steps = args.steps or 50
+        return run_trace(args, wl)
     if args.steps is None:
         args.steps = {"layer": 3000, "stack4": 256, "stack2": 256, "tiny": 1000, "batched": 100}[args.workload]
     args.warmup = max(args.warmup, 3)

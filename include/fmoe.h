@@ -262,6 +262,30 @@ FMOE_API fmoe_status fmoe_requant_4to2(const void* src_dev, int32_t n_blobs, int
  */
 FMOE_API fmoe_status fmoe_set_gemm_events(fmoe_ctx* ctx, void* const* events);
 
+/*
+ * Phase-timing hook of the fused single-token kernel, for profiling; no
+ * counterpart on the pages.  While set, a library built with FMOE_TRACE
+ * (build.py --trace) records %globaltimer stamps into trace_dev, an unsigned
+ * 64-bit device array [grid][fmoe_trace_layers()][fmoe_trace_points()] (grid =
+ * the device's SM count; the first fmoe_trace_layers() layers of a launch),
+ * owned by the caller and overwritten by every launch.  The product library
+ * compiles the recording out and ignores the pointer.  NULL clears the hook.
+ * Errors: INVALID_ARG (context), ALIGNMENT.
+ */
+FMOE_API fmoe_status fmoe_set_trace(fmoe_ctx* ctx, void* trace_dev);
+FMOE_API int32_t fmoe_trace_points(void);
+FMOE_API int32_t fmoe_trace_layers(void);
+
+/*
+ * Test hook: sets the context's launch epoch (the tag counter of its
+ * cross-block words) on `stream` and synchronises it.  A launch tags its words
+ * epoch + 1 .. epoch + layers; before those would pass 2^32 - 1 the library
+ * clears the tagged words and restarts the count at 0, so setting the epoch
+ * just below 2^32 exercises that wrap in a few launches.  No counterpart on the
+ * pages.  Errors: INVALID_ARG (context), CUDA.
+ */
+FMOE_API fmoe_status fmoe_debug_set_epoch(fmoe_ctx* ctx, uint32_t epoch, void* stream);
+
 /* Releases the workspace; the context pointer is invalid afterwards (later
  * calls with it return FMOE_ERR_INVALID_ARG).  Does not free caller memory. */
 FMOE_API fmoe_status fmoe_destroy(fmoe_ctx* ctx);

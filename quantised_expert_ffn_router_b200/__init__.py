@@ -20,6 +20,7 @@ __all__ = [
     "FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE", "Config", "LayerDesc", "FmoeError", "lib", "fmoe_expert_bytes",
     "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward", "fmoe_layer_forward", "fmoe_stack_forward",
     "fmoe_layer_forward_host", "fmoe_stack_forward_host", "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error", "EXPORTED_SYMBOLS",
+    "fmoe_set_trace", "fmoe_trace_points", "fmoe_trace_layers", "fmoe_debug_set_epoch", "use_trace_build",
 ]
 
 FMOE_OK, FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED, FMOE_ERR_ALIGNMENT = 0, 1, 2, 3
@@ -31,7 +32,8 @@ FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE = 0x100
 
 EXPORTED_SYMBOLS = ["fmoe_expert_bytes", "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward",
                     "fmoe_layer_forward", "fmoe_stack_forward", "fmoe_layer_forward_host", "fmoe_stack_forward_host",
-                    "fmoe_unpack_expert", "fmoe_requant_4to2", "fmoe_set_gemm_events",
+                    "fmoe_unpack_expert", "fmoe_requant_4to2", "fmoe_set_gemm_events", "fmoe_set_trace",
+                    "fmoe_trace_points", "fmoe_trace_layers", "fmoe_debug_set_epoch",
                     "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error"]
 
 
@@ -55,6 +57,18 @@ class FmoeError(RuntimeError):
 
 _lock = threading.Lock()
 _lib = None
+_trace = False
+
+
+def use_trace_build() -> None:
+    """Loads libfmoe_trace.so (the same sources built with FMOE_TRACE, which
+    records phase timestamps through fmoe_set_trace) instead of libfmoe.so.
+    Must be called before the first library call of the process."""
+    global _trace
+    with _lock:
+        if _lib is not None and not _trace:
+            raise RuntimeError("the product library is already loaded")
+        _trace = True
 
 
 def lib():
@@ -62,9 +76,9 @@ def lib():
     global _lib
     with _lock:
         if _lib is None:
-            path = _build.LIB
-            if _build.stale():
-                path = _build.build()
+            path = _build.LIB_TRACE if _trace else _build.LIB
+            if _build.stale(trace=_trace):
+                path = _build.build(trace=_trace)
             if not os.path.exists(path):
                 raise ImportError(f"libfmoe.so not found at {path}")
             L = ctypes.CDLL(path)
@@ -83,12 +97,17 @@ def lib():
             L.fmoe_poll_status.argtypes = [P, P, ctypes.POINTER(u32)]
             L.fmoe_set_gemm_events.argtypes = [P, P]
             L.fmoe_requant_4to2.argtypes = [P, i32, i32, i32, P, P]
+            L.fmoe_set_trace.argtypes = [P, P]
+            L.fmoe_trace_points.argtypes = []
+            L.fmoe_trace_layers.argtypes = []
+            L.fmoe_debug_set_epoch.argtypes = [P, u32, P]
             L.fmoe_destroy.argtypes = [P]
             L.fmoe_last_error.argtypes = [P]
             L.fmoe_last_error.restype = ctypes.c_char_p
             for name in ("fmoe_create", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
                          "fmoe_stack_forward", "fmoe_layer_forward_host", "fmoe_stack_forward_host",
-                         "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy"):
+                         "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy", "fmoe_set_trace",
+                         "fmoe_trace_points", "fmoe_trace_layers", "fmoe_debug_set_epoch"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -182,6 +201,26 @@ def fmoe_set_gemm_events(ctx, handles=None) -> int:
         return lib().fmoe_set_gemm_events(_vp(ctx), None)
     arr = (ctypes.c_void_p * 4)(*[int(h) for h in handles])
     return lib().fmoe_set_gemm_events(_vp(ctx), arr)
+
+
+def fmoe_set_trace(ctx, trace_dev=None) -> int:
+    """Phase timestamps of later fused-kernel launches into a uint64 device
+    buffer [n_sm][fmoe_trace_layers()][fmoe_trace_points()] (trace build only);
+    None clears the hook."""
+    return _check(ctx, lib().fmoe_set_trace(_vp(ctx), _vp(trace_dev)))
+
+
+def fmoe_trace_points() -> int:
+    return lib().fmoe_trace_points()
+
+
+def fmoe_trace_layers() -> int:
+    return lib().fmoe_trace_layers()
+
+
+def fmoe_debug_set_epoch(ctx, epoch: int, stream=0) -> int:
+    """Test hook: sets the context's tag epoch (synchronises `stream`)."""
+    return _check(ctx, lib().fmoe_debug_set_epoch(_vp(ctx), ctypes.c_uint32(epoch), _vp(stream)))
 
 
 def fmoe_poll_status(ctx, stream=0):

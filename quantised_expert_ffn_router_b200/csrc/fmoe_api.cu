@@ -26,6 +26,9 @@ struct fmoe_ctx {
   WsHeader* hdr = nullptr;
   uint64_t* logits = nullptr;  // tagged
   uint64_t* act = nullptr;     // tagged
+  size_t tagged_bytes = 0;     // logits, activations and layer outputs: the tagged words after the header
+  uint64_t tags_used = 0;      // mirrors the device epoch: tags handed out since the last clear
+  unsigned long long* trace = nullptr;  // caller's timestamp buffer (FMOE_TRACE builds), or null
   uint32_t* tasks = nullptr;   // device [3 modes][grid][kMaxTasks]
   int32_t* ntasks = nullptr;   // device [3 modes][grid]
   uint16_t* stack_buf[2] = {nullptr, nullptr};  // ping-pong activations, [max_tokens][H] bf16
@@ -227,11 +230,26 @@ DecodePlan bind(const fmoe_ctx* ctx, int mode, int layer) {
   P.tasks = ctx->tasks + (size_t)mode * ctx->n_sm * kMaxTasks;
   P.n_tasks = ctx->ntasks + (size_t)mode * ctx->n_sm;
   P.flags = ctx->cfg.flags;
+  P.trace = ctx->trace;
   P.timeout_ns = (uint64_t)(ctx->cfg.wait_timeout_us ? ctx->cfg.wait_timeout_us : 1000000u) * 1000ull;
   return P;
 }
 
 fmoe_status launch(fmoe_ctx* ctx, const DecodePlan& P, void* stream) {
+  // A launch tags its words epoch + 1 .. epoch + layers.  Before the tags would
+  // pass 2^32 - 1, the tagged words and the epoch are cleared (stream-ordered),
+  // so a tag never wraps to a value that stale words still carry.
+  const uint64_t n_tags = (uint64_t)std::max(P.n_layers, 1);
+  if (ctx->tags_used + n_tags > 0xFFFFFFFFull) {
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(&ctx->hdr->epoch, 0, sizeof(uint32_t), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->logits, 0, ctx->tagged_bytes, st);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_fail(ctx, e, "tag reset");
+    }
+    ctx->tags_used = 0;
+  }
   int rc = launch_decode(P, stream, true, ctx->pdl_ok);
   if (rc != 0 && ctx->pdl_ok) {
     cudaGetLastError();
@@ -242,6 +260,7 @@ fmoe_status launch(fmoe_ctx* ctx, const DecodePlan& P, void* stream) {
     cudaGetLastError();
     return cuda_fail(ctx, (cudaError_t)rc, "decode launch");
   }
+  ctx->tags_used += n_tags;
   return FMOE_OK;
 }
 
@@ -356,13 +375,16 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
     if (blocks < 1) return bail(fail(ctx, FMOE_ERR_UNSUPPORTED, "fused kernel cannot be resident"));
   }
 
-  // workspace: header | logits [E] | activations [kMaxSlots][I] | task lists | 2 x [max_tokens][H] bf16 |
-  // per-layer weight table | tagged layer outputs [H] | staging of the host-buffer calls
+  // workspace: header | tagged words: logits [E], activations [kMaxSlots][I], layer outputs [H] |
+  // task lists | 2 x [max_tokens][H] bf16 | per-layer weight table | staging of the host-buffer calls
   size_t off = 256;
   size_t off_logits = off;
   off += ((size_t)c.n_experts * 8 + 255) / 256 * 256;
   size_t off_act = off;
   off += ((size_t)kMaxSlots * c.inter * 8 + 255) / 256 * 256;
+  size_t off_hwords = off;
+  off += ((size_t)c.hidden * 8 + 255) / 256 * 256;
+  ctx->tagged_bytes = off - off_logits;
   size_t off_tasks = off;
   off += ((size_t)3 * ctx->n_sm * kMaxTasks * 4 + 255) / 256 * 256;
   size_t off_ntasks = off;
@@ -372,8 +394,6 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   off += 2 * stack_bytes;
   size_t off_layers = off;
   off += ((size_t)c.n_layers * sizeof(LayerDev) + 255) / 256 * 256;
-  size_t off_hwords = off;
-  off += ((size_t)c.hidden * 8 + 255) / 256 * 256;
   const size_t io_rows = (size_t)std::max(c.max_tokens, 1);
   size_t off_io_in = off;
   off += (io_rows * c.hidden * 2 + 255) / 256 * 256;
@@ -808,6 +828,26 @@ fmoe_status fmoe_set_gemm_events(fmoe_ctx* ctx, void* const* events) {
   for (int k = 0; k < 4; ++k)
     if (events[k] == nullptr) return fail(ctx, FMOE_ERR_INVALID_ARG, "event %d is NULL", k);
   for (int k = 0; k < 4; ++k) ctx->gemm_events[k] = events[k];
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_set_trace(fmoe_ctx* ctx, void* trace_dev) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  if (misaligned(trace_dev)) return fail(ctx, FMOE_ERR_ALIGNMENT, "trace buffer not 16-byte aligned");
+  ctx->trace = static_cast<unsigned long long*>(trace_dev);
+  return FMOE_OK;
+}
+
+int32_t fmoe_trace_points(void) { return kTracePoints; }
+int32_t fmoe_trace_layers(void) { return kTraceLayers; }
+
+fmoe_status fmoe_debug_set_epoch(fmoe_ctx* ctx, uint32_t epoch, void* stream) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(&ctx->hdr->epoch, &epoch, sizeof epoch, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "epoch write");
+  ctx->tags_used = epoch;
   return FMOE_OK;
 }
 

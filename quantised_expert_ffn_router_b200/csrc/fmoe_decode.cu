@@ -379,6 +379,25 @@ __device__ __forceinline__ LayerDev layer_of(const DecodePlan& P, int l) {
   return LayerDev{P.experts, P.router_w, P.router_bias, P.norm_w};
 }
 
+#ifdef FMOE_TRACE
+// Phase timestamps (%globaltimer) of this block for the first kTraceLayers
+// layers: SET once by one thread, FIRST by the first of several threads
+// (slot starts at 0), LAST by the latest.
+__device__ __forceinline__ unsigned long long* trace_slot(const DecodePlan& P, int l, int k) {
+  return P.trace + ((size_t)blockIdx.x * kTraceLayers + l) * kTracePoints + k;
+}
+#define FMOE_TRACE_SET(l, k) \
+  do { if (P.trace && (l) < kTraceLayers) *trace_slot(P, l, k) = gtimer(); } while (0)
+#define FMOE_TRACE_FIRST(l, k) \
+  do { if (P.trace && (l) < kTraceLayers) atomicCAS(trace_slot(P, l, k), 0ull, (unsigned long long)gtimer()); } while (0)
+#define FMOE_TRACE_LAST(l, k) \
+  do { if (P.trace && (l) < kTraceLayers) atomicMax(trace_slot(P, l, k), (unsigned long long)gtimer()); } while (0)
+#else
+#define FMOE_TRACE_SET(l, k) do {} while (0)
+#define FMOE_TRACE_FIRST(l, k) do {} while (0)
+#define FMOE_TRACE_LAST(l, k) do {} while (0)
+#endif
+
 // MULTI: one launch runs layers 0..n_layers-1 of a stack for one token.  The
 // producer streams on into layer l+1 (its router rows, then the shared
 // expert's chunks, which need no routing) while the consumers finish layer l;
@@ -413,6 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int my_rrows = (has_router && cta < P.E) ? (P.E - cta + G - 1) / G : 0;
   const int n_down = P.n_down_max > 0 ? my_rb * P.n_slots * P.dn_chunks : 0;
   float h_res = 0.f;  // residual input of the row this thread combines
+  if (tid == 0) FMOE_TRACE_SET(0, 0);
 
   // ---------------------------------------------------------------- set-up
   // The producer initialises the ring and, before the block barrier, already
@@ -437,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         reinterpret_cast<volatile int*>(misc->last_task)[s] = lane;
       }
     }
+    if (lane == 0) FMOE_TRACE_SET(0, 1);
   } else if (warp == 1) {
     misc->aflag[lane] = 0;
     if (lane < 16) {
@@ -504,7 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
           }
         }
-        if (__all_sync(0xffffffffu, mine)) break;
+        if (__all_sync(0xffffffffu, mine)) {
+          if (lane == 0) FMOE_TRACE_SET(cur, 3);
+          break;
+        }
         __nanosleep(32);
         if (__any_sync(0xffffffffu, *abort_flag != 0 || gtimer() - t0 > limit)) {
           if (lane == 0) {
@@ -531,6 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (cta == 0 && P.w_out) P.w_out[lane] = w;
       }
       __syncwarp();
+      if (lane == 0) FMOE_TRACE_SET(cur, 4);
       return true;
     };
 
@@ -627,8 +652,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           if (!downs_issued && !issue_downs()) break;
           if (needs_route) ok = issue(i, t);
           if (!__all_sync(0xffffffffu, ok)) break;
+          if (lane == 0) FMOE_TRACE_SET(cur, 5);
         }
       }
+      if (lane == 0) FMOE_TRACE_SET(cur, 6);
       // a block whose own list needed no routing still owes its down jobs
       if (!downs_issued && !__any_sync(0xffffffffu, *abort_flag)) {
         if (P.mode == kModeLayer && !routed) routed = do_routing();
@@ -775,6 +802,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
       }
 
+      if (tid == 0) FMOE_TRACE_SET(cur, 2);
       // The producer selects the routed experts once per launch, late; running
       // the same selection code here on whatever the logit buffer holds (it
       // writes nothing) brings that code into the instruction cache meanwhile.
@@ -848,9 +876,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
               st_tagged(P.ws_logits + e, l, (P.flags & FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE) ? tag - 1u : tag);
               red_relaxed_add(&P.ws->router_cnt, 1u);
             atomicAdd(&misc->rdone, 1);
+            FMOE_TRACE_LAST(cur, 7);
             }
           }
         } else if (ty == kTaskGateUp) {
+          if (lane == 0 && slot > 0) FMOE_TRACE_FIRST(cur, 8);
           const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
           const float2 acc = chunk_dot<BITS>(stage, n, zfrag, zinfo, (int)c * kChunkTiles, lane);
           float acc0 = acc.x, acc1 = acc.y;
@@ -885,11 +915,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const float av = writer ? acc0 / (1.0f + expf(-acc0)) * acc1 : 0.f;
             if (writer) st_tagged(P.ws_a + (int64_t)slot * P.I + rb * 8 + row, av, tag);
             if (lane == 0) red_relaxed_add(&P.ws->h_cnt[slot], 1u);
+            if (lane == 0) {
+              if (slot > 0) FMOE_TRACE_LAST(cur, 9);
+              else FMOE_TRACE_LAST(cur, 14);
+            }
           }
         } else {
           // activations of this slot as fragments, built once per block in two
           // halves of the slot's groups: the block's two down jobs of a slot
           // usually run on two warps, which then fetch and build a half each.
+          if (lane == 0) FMOE_TRACE_FIRST(cur, 15);
           uint32_t* af = reinterpret_cast<uint32_t*>(smem + P.off_afrag + slot * P.afrag_bytes);
           float2* ai = reinterpret_cast<float2*>(smem + P.off_ainfo + slot * P.ainfo_bytes);
           const uint64_t* act = P.ws_a + (int64_t)slot * P.I;
@@ -933,6 +968,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 if (attempt > 0) __nanosleep(256);
               }
               if (!good) break;
+              if (lane == 0) FMOE_TRACE_FIRST(cur, 10);
               float lo[kFetchGroups], hi[kFetchGroups];
 #pragma unroll
               for (int k = 0; k < kFetchGroups; ++k) {
@@ -991,7 +1027,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_empty + 8u * s);
+        if (lane == 0) {
+          mbar_arrive(bar_empty + 8u * s);
+          if (ty == kTaskDown) FMOE_TRACE_LAST(cur, 11);
+        }
       }
       if (MULTI) {
         // all consumer warps are done with this layer's tasks
@@ -1007,6 +1046,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           else
             st_tagged(P.ws_h + out_row, h_res, tag);
         }
+        if (tid == 0) FMOE_TRACE_SET(cur, 12);
         if (warp == 1) {
           misc->aflag[lane] = 0;
           misc->unit_cnt[lane] = 0;
@@ -1035,6 +1075,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
   }
 
+  if (tid == 0) FMOE_TRACE_SET(0, 12);
   // ---------------------------------------------------------------- drain + reset
   if (tid == kConsumerWarps * 32) {
     // After an abort the latest copy into every stage must land before the
@@ -1051,6 +1092,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           break;
         }
     }
+    FMOE_TRACE_SET(0, 13);
     // the last block out advances the epoch for the next launch
     uint32_t old;
     asm volatile("atom.release.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&P.ws->exit_count) : "memory");

@@ -45,6 +45,8 @@ constexpr int kStaticRouteMaxTokens = 4096;  // tokens per fmoe_route_static cal
 constexpr int kMaxDevices = 64;          // devices fmoe_route_static caches a scratch address for
 constexpr int kMinRingStages = 20;       // ring stages kept when down jobs get stages of their own
 constexpr int kFetchGroups = 8;          // activation groups a warp fetches per round trip
+constexpr int kTracePoints = 32;         // FMOE_TRACE builds: %globaltimer stamps per block and layer
+constexpr int kTraceLayers = 4;          // ... for the first layers of a launch
 
 inline __host__ __device__ int tile_code_bytes(int bits) { return 16 * kGroup * bits / 8; }
 inline __host__ __device__ int tile_bytes(int bits) { return tile_code_bytes(bits) + 64; }
@@ -59,11 +61,15 @@ inline __host__ __device__ int64_t packed_gu_bytes(int H, int I, int bits) {
   return (int64_t)(I / 8) * (H / kGroup) * tile_bytes(bits);
 }
 
-// Device workspace header, followed by the tagged logits and activations.
-// Cross-block results are published as 64-bit words {float bits, tag} with
-// tag = epoch + 1, so a reader knows a value is from the current launch
-// without any counter, fence or atomic on the critical path.  The last block
-// to finish a launch advances the epoch (exit_count protocol).
+// Device workspace header, followed by the tagged logits, activations and
+// layer outputs.  Cross-block results are published as 64-bit words
+// {float bits, tag} with tag = epoch + 1 (+ layer in a multi-layer launch), so
+// a reader knows a value is from the current launch without any counter, fence
+// or atomic on the critical path.  The last block to finish a launch advances
+// the epoch by the launch's layer count (exit_count protocol).  The host never
+// lets a tag pass 2^32 - 1: before a launch whose tags would, it clears the
+// tagged words and the epoch, so tag 0 -- the value of every cleared word --
+// is never current.
 struct WsHeader {
   uint32_t epoch;           // launches completed on this workspace
   uint32_t exit_count;      // blocks finished in the current launch
@@ -184,6 +190,7 @@ struct DecodePlan {
   int n_layers;
   const LayerDev* layer_dev;
   uint64_t* ws_h;          // [H] tagged
+  unsigned long long* trace;  // FMOE_TRACE builds: [grid][kTraceLayers][kTracePoints] stamps, or null
 };
 
 // Ring position of task i: issued by producer lane i % n_issuers into that

@@ -15,7 +15,7 @@ import pytest
 
 import oracle
 import synth
-from moe_cases import REL_L2_TOL, Model, OracleLayer, bf16_tensor_bits, rel_l2, tie_free_subseeds
+from moe_cases import REL_L2_TOL, W_TOL, Model, OracleLayer, bf16_tensor_bits, rel_l2, tie_free_subseeds
 
 pytestmark = pytest.mark.gpu
 
@@ -142,3 +142,44 @@ def test_multi_layer_bounded_wait_reports_timeout(torch):
         b = bf16_tensor_bits(_chained(torch, m, x, 0, wl.n_layers))
         _ok(m)
     assert np.array_equal(a, b)
+
+
+def test_tags_survive_the_wrap_past_two_to_the_32(torch):
+    """A launch tags its cross-block words epoch + 1 .. epoch + layers.  With
+    the epoch set just below 2^32, single- and multi-layer launches run across
+    the point where the host clears the tagged words and restarts the count:
+    the outputs equal those of a fresh context bit for bit, and the
+    single-layer results (indices, weights, output) match the oracle."""
+    wl = STACK7
+    T = 2  # below the grouped path's threshold: one launch per token
+    x = _x(wl, T, start=40)
+
+    def run(m):
+        out = torch.empty_like(x)
+        idx = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+        m.fm.fmoe_layer_forward(m.ctx, 0, x.data_ptr(), T, out.data_ptr(), idx.data_ptr(), w.data_ptr(), m.stream)
+        stack = _stack(torch, m, x, 0, wl.n_layers)
+        return (bf16_tensor_bits(out), idx.cpu().numpy(), w.cpu().numpy(), bf16_tensor_bits(stack))
+
+    with Model(wl) as m:
+        fresh = run(m)
+        _ok(m)
+    top = 0xFFFFFFFF
+    with Model(wl) as m:
+        # per run(): 2 single-layer launches (1 tag each), then 2 stack launches (7 tags each)
+        for epoch in (top - 20, top - 9, top - 2, top - 1, top):
+            m.fm.fmoe_debug_set_epoch(m.ctx, epoch, m.stream)
+            for _ in range(2):
+                got = run(m)
+                _ok(m)
+                for a, b in zip(got, fresh):
+                    assert np.array_equal(a, b), hex(epoch)
+    ol = OracleLayer(wl, 0)
+    xb = bf16_tensor_bits(x)
+    out, gi, gw, _ = fresh
+    for t in range(T):
+        r = ol.forward(xb[t])
+        assert list(gi[t]) == list(r["idx"]), t
+        assert np.max(np.abs(gw[t] - r["w"])) <= W_TOL, t
+        assert rel_l2(oracle.bf16_to_f64(out[t]), oracle.bf16_to_f64(r["out"])) <= REL_L2_TOL, t
