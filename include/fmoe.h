@@ -115,17 +115,33 @@ FMOE_API size_t fmoe_expert_bytes(int32_t hidden, int32_t inter, int32_t bits);
  * descriptors (copied; the weights they point to are borrowed), allocates the
  * device workspace, and repacks every layer's experts_dev in place from the
  * canonical to the packed layout on `stream` (then synchronises it).
+ * When the context may take the grouped batched path (max_tokens > 1 and not
+ * FMOE_FLAG_FORCE_PER_TOKEN, or FMOE_FLAG_FORCE_GROUPED), every scale and bias
+ * is first checked against that path's fp16 dequantisation: every scale must
+ * be 0 or of magnitude in [2^-14, 65504], every bias at most 65504 in
+ * magnitude, and |scale| * (2^bits - 1) + |bias| <= 65504 (NaN and inf fail).
+ * Weights outside fail the call with UNSUPPORTED before anything is rewritten;
+ * the batch-1 kernel applies scale and bias in fp32 and takes any finite value.
  * Errors: INVALID_ARG (NULL, bad shapes, K > E, bits not 2/4, group != 64),
- * UNSUPPORTED (H or I above 4096 or a shape whose shared-memory plan does not
- * fit), ALIGNMENT, OOM, CUDA.  On error *out is NULL.
+ * UNSUPPORTED (H or I above 4096, a shape whose shared-memory plan does not
+ * fit, or scales/biases outside the grouped path's range), ALIGNMENT, OOM,
+ * CUDA.  On error *out is NULL.
  */
 FMOE_API fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, void* stream, fmoe_ctx** out);
 
 /*
+ * Passage: the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on
+ * a Laptop", section "How the SSD expert streaming pipeline works": the second
+ * command buffer normalises the layer input and computes the routing logits,
+ * then the host takes a softmax and the top K; the themata summary of the same
+ * title (Key Takeaways) gives 512 experts per layer with K = 4.
  * Router step of layer `layer` for T tokens: z = RMSNorm(x) when the layer has
  * a norm weight (else z = x), logits = W_r z (+ bias) in fp32, softmax, the K
  * largest probabilities in descending order (equal values: lower expert index
- * first) and their renormalised weights w_k = p_k / sum_j p_j.
+ * first) and their renormalised weights w_k = p_k / sum_j p_j.  A NaN logit
+ * counts as -inf; when the largest logit is infinite the softmax is taken as
+ * its limit, so the picks equal to it share the weight equally (each of K
+ * picks gets 1/K when every logit is -inf).
  *   x_dev   : bf16 [T][H];  idx_dev : int32 [T][K];  w_dev : fp32 [T][K].
  * T == 0 is a no-op.  Errors: INVALID_ARG (layer or T out of range, NULL),
  * ALIGNMENT, CUDA.
@@ -141,9 +157,13 @@ FMOE_API fmoe_status fmoe_route(fmoe_ctx* ctx, int32_t layer, const void* x_dev,
  * call -- a loop whose device memory is held entirely by its own pool
  * allocator, or one that cannot take cudaFree's device-wide synchronisation.
  * Limits: T * E <= 32768 and T <= 4096; larger calls return UNSUPPORTED
- * before any GPU work.  The first call on a device looks up the array's
- * address (cudaGetSymbolAddress); make it before any stream capture.  Calls
- * that overlap in time share the array and race: order them on one stream.
+ * before any GPU work.  fmoe_create looks up the array's address on its
+ * device (cudaGetSymbolAddress), so calls on a context never do, and may be
+ * captured into a CUDA graph; a call on a device where no context was created
+ * made inside a stream capture returns UNSUPPORTED instead of looking it up.
+ * Calls that overlap in time share the array and race: order them on one
+ * stream.  Weights follow fmoe_route's rule, including its limit for an
+ * infinite largest logit.
  * Logits accumulate in a different order than fmoe_route's, so weights may
  * differ in the last bits; the indices agree except at near-ties.
  * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA.
@@ -152,6 +172,11 @@ FMOE_API fmoe_status fmoe_route_static(fmoe_ctx* ctx, int32_t layer, const void*
                                        int32_t* idx_dev, float* w_dev, void* stream);
 
 /*
+ * Passage: "Flash-MoE: Running a 400 Billion Parameter Model on a MacBook",
+ * section "The Architecture" (each active expert's weights dequantised inside
+ * fused multiply-adds, about 6.75 MB per expert at 4 bits), and the Hysen Labs
+ * page's section "How the SSD expert streaming pipeline works" (the third
+ * command buffer runs the expert forward pass).
  * One expert's SwiGLU feed-forward on the layer's (normed) input:
  * y = W_down (silu(W_gate z) * (W_up z)), z as in fmoe_route.
  *   expert  : 0..E-1 for a routed expert, -1 for the shared expert.
@@ -163,6 +188,12 @@ FMOE_API fmoe_status fmoe_expert_forward(fmoe_ctx* ctx, int32_t layer, int32_t e
                                 float* y_dev, void* stream);
 
 /*
+ * Passage: the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on
+ * a Laptop", section "How the SSD expert streaming pipeline works": one layer's
+ * mixture-of-experts part is normalisation, routing and the shared expert
+ * (second command buffer), softmax and top-K (host), then the K = 4 routed
+ * experts' forward pass and their combine (third command buffer).  Here all of
+ * it is one launch (batch-1) or one stream of launches (grouped path).
  * One full mixture-of-experts layer:
  *   h_out = h_in + sum_k w_k * E_{idx_k}(z) + E_shared(z)
  * with z, idx, w as in fmoe_route, accumulated in fp32 and rounded once to bf16.
@@ -177,6 +208,11 @@ FMOE_API fmoe_status fmoe_layer_forward(fmoe_ctx* ctx, int32_t layer, const void
                                int32_t* idx_out_dev, float* w_out_dev, void* stream);
 
 /*
+ * Passage: the Hysen Labs page's section "How the SSD expert streaming
+ * pipeline works": 60 layers each run the same per-layer sequence, and the
+ * previous layer's expert command buffer is still in flight when the next
+ * layer starts; the wiki page "Flash-MoE" (Performance Results) quotes the
+ * resulting decode rates for the 4-bit and 2-bit expert sets.
  * Layers layer_begin .. layer_end-1 in sequence (a mixture-of-experts-only
  * stack: each layer's output is the next layer's input), equivalent to
  * chaining fmoe_layer_forward bit for bit; intermediate activations live in

@@ -119,13 +119,17 @@ void orc_router_logits(const uint16_t* wr, const float* bias, const uint16_t* z,
   }
 }
 
-typedef struct { double p; int e; } prob_entry;
+typedef struct { double p; double l; int e; } prob_entry;
 
+/* larger probability first; equal probabilities (exact ties, or both rounded
+ * to 0) by larger logit, then lower expert index */
 static int by_prob_desc(const void* a, const void* b) {
   const prob_entry* x = (const prob_entry*)a;
   const prob_entry* y = (const prob_entry*)b;
   if (x->p > y->p) return -1;
   if (x->p < y->p) return 1;
+  if (x->l > y->l) return -1;
+  if (x->l < y->l) return 1;
   return (x->e > y->e) - (x->e < y->e);
 }
 
@@ -133,15 +137,25 @@ static int by_prob_desc(const void* a, const void* b) {
  * section "How the SSD expert streaming pipeline works":
  * the host takes the softmax and picks the top K; the themata summary "Flash-MoE: Running a 397B Parameter Model on a Laptop",
  * Key Takeaways: K = 4).
- * Renormalising the K selected probabilities is a reading taken where the pages are silent. */
+ * Renormalising the K selected probabilities is a reading taken where the pages are silent.
+ * Non-finite logits, where the pages are silent too: a NaN logit counts as
+ * -inf, and when the largest logit is infinite the softmax is its limit, the
+ * whole mass shared equally by the experts whose logit equals the largest
+ * (all of them when every logit is -inf). */
 void orc_topk(const float* logits, int n_experts, int top_k, int32_t* idx, double* w, double* p) {
-  double mx = -INFINITY;
-  for (int e = 0; e < n_experts; ++e) mx = fmax(mx, (double)logits[e]);
   prob_entry* ent = (prob_entry*)malloc(sizeof(prob_entry) * (size_t)n_experts);
+  double mx = -INFINITY;
+  for (int e = 0; e < n_experts; ++e) {
+    ent[e].l = isnan(logits[e]) ? -INFINITY : (double)logits[e];
+    ent[e].e = e;
+    mx = fmax(mx, ent[e].l);
+  }
   double denom = 0.0;
   for (int e = 0; e < n_experts; ++e) {
-    ent[e].p = exp((double)logits[e] - mx);
-    ent[e].e = e;
+    if (isinf(mx))
+      ent[e].p = ent[e].l == mx ? 1.0 : 0.0;
+    else
+      ent[e].p = exp(ent[e].l - mx);
     denom += ent[e].p;
   }
   for (int e = 0; e < n_experts; ++e) {

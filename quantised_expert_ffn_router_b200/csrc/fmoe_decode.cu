@@ -542,9 +542,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       const TopPick pick = topk_select(lg, P.E, P.K, lane);
       const float my_top = pick.logit;
       const int my_sel = pick.expert;
-      // renormalised weights over the K selected: p_k / sum_j p_j = e^(l_k - l_0) / sum_j e^(l_j - l_0)
+      // renormalised weights over the K selected: p_k / sum_j p_j = e^(l_k - l_0) / sum_j e^(l_j - l_0);
+      // an infinite largest logit takes the softmax's limit (equal shares for the picks equal to it)
       const float top0 = __shfl_sync(0xffffffffu, my_top, 0);
-      const float ex = lane < P.K ? expf(my_top - top0) : 0.f;
+      const float ex = lane >= P.K ? 0.f : fabsf(top0) != INFINITY ? expf(my_top - top0) : (my_top == top0 ? 1.f : 0.f);
       float den = ex;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);

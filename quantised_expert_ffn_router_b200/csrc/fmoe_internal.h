@@ -336,10 +336,16 @@ int launch_repack(const uint8_t* src, uint8_t* dst, int n_experts, int H, int I,
 int launch_decode(const DecodePlan& plan, void* stream, bool cooperative, bool pdl);
 // Router step with its scratch in a fixed device array (fmoe_static.cu); returns
 // a cudaError_t value.
+int route_static_prepare();  // 0 or a cudaError_t
+bool route_static_ready();
 int launch_route_static(const uint16_t* wr, const float* bias, const uint16_t* norm_w, float eps,
                         const uint16_t* x, int T, int H, int E, int K, int32_t* idx_out, float* w_out, void* stream);
 // 4-bit -> 2-bit requantisation of n canonical blobs (fmoe_requant.cu).
 int launch_requant(const uint8_t* src, uint8_t* dst, int n_blobs, int H, int I, int n_sm, void* stream);
+// Bits of launch_check_affine's flag word.
+constexpr uint32_t kAffineNonFinite = 1u, kAffineScaleRange = 2u, kAffineBiasRange = 4u, kAffineWeightRange = 8u;
+int launch_check_affine(const uint8_t* blobs, int n_blobs, int H, int I, int bits, uint32_t* flags_dev,
+                        void* stream);
 int decode_max_smem_optin(int device);
 int decode_occupancy(int bits, bool multi, int smem_bytes, int* blocks_per_sm);
 int zero_workspace(void* ws, size_t bytes, void* stream);

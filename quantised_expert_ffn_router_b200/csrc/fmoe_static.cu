@@ -135,9 +135,10 @@ __global__ void __launch_bounds__(kWarps * 32) static_topk_kernel(const float* _
       my_idx = (int)~(uint32_t)prev;
     }
   }
-  // renormalised weights over the K picks: exp(l_k - l_0) / sum_j exp(l_j - l_0)
+  // renormalised weights over the K picks: exp(l_k - l_0) / sum_j exp(l_j - l_0); an infinite
+  // largest logit takes the softmax's limit (equal shares for the picks equal to it)
   const float top0 = __shfl_sync(0xffffffffu, my_logit, 0);
-  const float ex = lane < K ? expf(my_logit - top0) : 0.f;
+  const float ex = lane >= K ? 0.f : fabsf(top0) != INFINITY ? expf(my_logit - top0) : (my_logit == top0 ? 1.f : 0.f);
   float den = ex;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
@@ -158,21 +159,42 @@ int launch_topk_rows(const float* logits, int T, int E, int K, int32_t* idx_out,
   return (int)cudaGetLastError();
 }
 
+// Looks up the fixed scratch's address on the current device (once per
+// device).  fmoe_create calls it, so no later call has to, which matters
+// inside a stream capture, where the lookup may load the module.
+int route_static_prepare() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return (int)e;
+  if (dev < 0 || dev >= kMaxDevices) return (int)cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> g(g_symbol_mu);
+  if (g_symbol_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_logits);
+    if (e != cudaSuccess) return (int)e;
+    g_symbol_addr[dev] = static_cast<float*>(p);
+  }
+  return 0;
+}
+
+bool route_static_ready() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> g(g_symbol_mu);
+  return g_symbol_addr[dev] != nullptr;
+}
+
 int launch_route_static(const uint16_t* wr, const float* bias, const uint16_t* norm_w, float eps,
                         const uint16_t* x, int T, int H, int E, int K, int32_t* idx_out, float* w_out, void* stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return (int)e;
   if (dev < 0 || dev >= kMaxDevices) return (int)cudaErrorInvalidDevice;
+  const int rc = route_static_prepare();
+  if (rc != 0) return rc;
   float* scratch = nullptr;
   {
     std::lock_guard<std::mutex> g(g_symbol_mu);
-    if (g_symbol_addr[dev] == nullptr) {
-      void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_route_logits);
-      if (e != cudaSuccess) return (int)e;
-      g_symbol_addr[dev] = static_cast<float*>(p);
-    }
     scratch = g_symbol_addr[dev];
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -148,18 +148,20 @@ def test_grouped_path_is_deterministic(torch):
 
 
 @pytest.mark.slow
-def test_full_batched_step_sampled_tokens(torch):
+def test_full_batched_step_every_token(torch):
     """The batched workload at full size: 256 tokens per step through the
     grouped path (H 4096, 512 experts with a Zipf(1.1) router skew, top-4 +
-    shared, I 1024, 4-bit).  Routing is checked for every token, the layer
-    output for a sample of 8 tokens."""
+    shared, I 1024, 4-bit).  Routing and the layer output are checked for
+    every token.  The oracle runs expert by expert (one blob in host memory at
+    a time); the routing must give segments of every size class the grouped
+    path treats differently (1, 2-15, 16-63 and >= 64 tokens per expert)."""
     wl = synth.WORKLOADS["batched"]
-    T = wl.tokens
+    T, K, E = wl.tokens, wl.top_k, wl.n_experts
     x = _tokens(wl, T)
     with Model(wl) as m:
         out = torch.empty_like(x)
-        idx = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
-        w = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+        idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, K), dtype=torch.float32, device="cuda")
         m.fm.fmoe_layer_forward(m.ctx, 0, x.data_ptr(), T, out.data_ptr(), idx.data_ptr(), w.data_ptr(), m.stream)
         torch.cuda.synchronize()
         st, word = m.fm.fmoe_poll_status(m.ctx, m.stream)
@@ -169,12 +171,27 @@ def test_full_batched_step_sampled_tokens(torch):
     torch.cuda.empty_cache()
     ol = OracleLayer(wl, 0)
     xb = bf16_tensor_bits(x)
+    ri = np.empty((T, K), np.int64)
+    rw = np.empty((T, K))
     for t in range(T):
-        logits = oracle.router_logits(ol.router, ol.bias, xb[t])
-        ri, rw, _ = oracle.topk(logits, wl.top_k)
-        assert list(gi[t]) == list(ri), t
-        assert np.max(np.abs(gw[t] - rw)) <= W_TOL, t
-    for t in np.random.default_rng(1).choice(T, size=8, replace=False):
-        r = ol.forward(xb[t])
-        err = rel_l2(oracle.bf16_to_f64(got[t]), oracle.bf16_to_f64(r["out"]))
-        assert err <= REL_L2_TOL, (int(t), err)
+        i, wt, _ = oracle.topk(oracle.router_logits(ol.router, ol.bias, xb[t]), K)
+        ri[t], rw[t] = i, wt
+        assert list(gi[t]) == list(i), t
+        assert np.max(np.abs(gw[t] - wt)) <= W_TOL, t
+    seg = np.bincount(ri.ravel(), minlength=E)
+    used = seg[seg > 0]
+    for lo, hi in ((1, 1), (2, 15), (16, 63), (64, T)):
+        assert np.any((used >= lo) & (used <= hi)), (lo, hi)
+    y = np.zeros((T, K, wl.hidden))
+    for e in np.unique(ri):  # no norm in this workload: z = x
+        blob = synth.expert_blob(wl, 0, int(e))
+        for t, k in zip(*np.nonzero(ri == e)):
+            y[t, k] = oracle.expert(blob, wl.hidden, wl.inter, wl.bits, xb[t])[0]
+    shared = synth.expert_blob(wl, 0, E)
+    worst = 0.0
+    for t in range(T):
+        y_sh = oracle.expert(shared, wl.hidden, wl.inter, wl.bits, xb[t])[0]
+        _, want = oracle.combine(xb[t], rw[t], y[t], y_sh)
+        err = rel_l2(oracle.bf16_to_f64(got[t]), oracle.bf16_to_f64(want))
+        worst = max(worst, err)
+        assert err <= REL_L2_TOL, (t, int(seg[ri[t]].min()), err)

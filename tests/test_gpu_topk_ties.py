@@ -6,13 +6,16 @@ bias.  The selection must then be the first K entries of the experts sorted
 by (larger logit, lower index): the fused kernel's route and layer modes, the
 grouped path (T >= 8) and the allocation-free router step all have to agree
 with that order exactly, and the renormalised weights with the softmax of
-the picked logits.
+the picked logits.  Non-finite biases are included: NaN ranks as -inf, and an
+infinite largest logit gives the softmax's limit (equal weights for the picks
+equal to it), the rule the oracle takes.
 """
 import dataclasses
 
 import numpy as np
 import pytest
 
+import oracle
 import synth
 from moe_cases import Model
 
@@ -51,12 +54,27 @@ def _patterns(E):
     top_last = np.full(E, -2.0, np.float32)
     top_last[-3:] = np.float32(1.5)
     yield "ties at the end", top_last
+    plus_inf = np.full(E, -1.0, np.float32)
+    plus_inf[[1, E // 2, E - 1]] = np.inf
+    yield "+inf ties", plus_inf
+    yield "all -inf", np.full(E, -np.inf, np.float32)
+    nan_mix = np.full(E, np.nan, np.float32)
+    nan_mix[::4] = -np.inf
+    nan_mix[E // 3] = np.float32(0.5)
+    yield "NaN and -inf", nan_mix
 
 
 def _expected(bias, K):
-    order = sorted(range(len(bias)), key=lambda e: (-float(bias[e]), e))[:K]
-    logits = np.array([float(bias[e]) for e in order])
-    w = np.exp(logits - logits[0])
+    """Order (larger logit, lower index; NaN as -inf) and renormalised weights;
+    an infinite largest logit gives the softmax's limit, equal shares for the
+    picks equal to it."""
+    lg = np.where(np.isnan(bias), -np.inf, bias).astype(np.float64)
+    order = sorted(range(len(lg)), key=lambda e: (-lg[e], e))[:K]
+    logits = lg[order]
+    if np.isinf(logits[0]):
+        w = (logits == logits[0]).astype(np.float64)
+    else:
+        w = np.exp(logits - logits[0])
     return np.array(order, np.int32), w / w.sum()
 
 
@@ -73,6 +91,8 @@ def test_topk_exact_ties(torch, wl):
         for name, bias in _patterns(E):
             layer.bias.copy_(torch.from_numpy(bias))
             want_idx, want_w = _expected(bias, K)
+            o_idx, o_w, _ = oracle.topk(bias, K)  # the oracle takes the same rule
+            assert np.array_equal(o_idx, want_idx) and np.allclose(o_w, want_w, rtol=0, atol=1e-15), name
             got = {}
             idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
             w = torch.empty((T, K), dtype=torch.float32, device="cuda")

@@ -173,6 +173,44 @@ def test_topk_is_stable_for_huge_logits():
     np.testing.assert_allclose(w, [1 / (1 + math.exp(-1)), 1 / (1 + math.exp(1))], rtol=1e-14)
 
 
+def test_topk_underflowed_probabilities_rank_by_logit():
+    """Probabilities that underflow to 0 in double still rank by their logits:
+    selecting the K largest probabilities is selecting the K largest logits."""
+    logits = np.array([0.0, -1000.0, -800.0, -900.0, -800.0], dtype=np.float32)
+    idx, w, p = oracle.topk(logits, 4)
+    assert p[1] == 0.0 and p[2] == 0.0  # exp(-800) underflows
+    assert list(idx) == [0, 2, 4, 3]
+    np.testing.assert_allclose(w, [1.0, 0.0, 0.0, 0.0], rtol=0, atol=0)
+
+
+def test_topk_infinite_logits_take_the_softmax_limit():
+    """+inf logits share the mass equally (the limit of the softmax as those
+    logits grow together); the picks after them rank by logit."""
+    inf = np.float32(np.inf)
+    logits = np.array([1.0, inf, -3.0, inf, 2.0, inf], dtype=np.float32)
+    idx, w, p = oracle.topk(logits, 5)
+    assert list(idx) == [1, 3, 5, 4, 0]
+    np.testing.assert_allclose(w, [1 / 3, 1 / 3, 1 / 3, 0, 0], rtol=1e-15, atol=0)
+    np.testing.assert_allclose(p, [0, 1 / 3, 0, 1 / 3, 0, 1 / 3], rtol=1e-15, atol=0)
+    idx, w, _ = oracle.topk(logits, 2)
+    assert list(idx) == [1, 3]
+    np.testing.assert_allclose(w, [0.5, 0.5], rtol=1e-15, atol=0)
+
+
+def test_topk_all_minus_inf_or_nan_is_uniform():
+    """Every logit -inf (NaN counts as -inf): all experts tie, so the lowest
+    indices are picked with equal weights; a single finite logit takes all."""
+    logits = np.array([np.nan, -np.inf, np.nan, -np.inf, -np.inf], dtype=np.float32)
+    idx, w, p = oracle.topk(logits, 3)
+    assert list(idx) == [0, 1, 2]
+    np.testing.assert_allclose(w, [1 / 3] * 3, rtol=1e-15, atol=0)
+    np.testing.assert_allclose(p, [0.2] * 5, rtol=1e-15, atol=0)
+    logits[3] = -7.0
+    idx, w, _ = oracle.topk(logits, 3)
+    assert list(idx) == [3, 0, 1]
+    np.testing.assert_allclose(w, [1.0, 0.0, 0.0], rtol=0, atol=0)
+
+
 def test_router_bias_shift_and_expert_permutation():
     wl = synth.WORKLOADS["tiny"]
     wr = synth.router_weight(wl, 0)

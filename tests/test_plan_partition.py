@@ -39,6 +39,9 @@ int launch_decode(const DecodePlan&, void*, bool, bool) { return 1; }
 int launch_route_static(const uint16_t*, const float*, const uint16_t*, float, const uint16_t*, int, int, int, int,
                         int32_t*, float*, void*) { return 1; }
 int launch_requant(const uint8_t*, uint8_t*, int, int, int, int, void*) { return 1; }
+int launch_check_affine(const uint8_t*, int, int, int, int, uint32_t*, void*) { return 1; }
+int route_static_prepare() { return 0; }
+bool route_static_ready() { return true; }
 int decode_max_smem_optin(int) { return 232448; }
 int decode_occupancy(int, bool, int, int* b) { *b = 1; return 0; }
 int zero_workspace(void*, size_t, void*) { return 1; }
