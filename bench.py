@@ -433,7 +433,7 @@ def run_gpu(args, wl, ws, rank, local):
     line = {
         "metric": metric_name(wl), "value": tps, "unit": "tokens/s", "n_gpus": ws, "steps": steps,
         "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": ("fp16 dequantised weights x fp16 inputs on tcgen05, fp32 accumulate (bf16 I/O)"
+        "vs_baseline": None, "dtype": ("exact integer codes x fp16 inputs on tcgen05, fp32 accumulate + fp32 scale/bias (bf16 I/O)"
                                        if batched else "fp16 tensor-core MAC of exact integer codes, fp32 accumulate (bf16 I/O)"),
         "data": "synthetic (seeded, shaped like the pages' model; random weights)",
         "config": {**config_dict(wl, flushed=not stacked),

@@ -115,17 +115,11 @@ FMOE_API size_t fmoe_expert_bytes(int32_t hidden, int32_t inter, int32_t bits);
  * descriptors (copied; the weights they point to are borrowed), allocates the
  * device workspace, and repacks every layer's experts_dev in place from the
  * canonical to the packed layout on `stream` (then synchronises it).
- * When the context may take the grouped batched path (max_tokens > 1 and not
- * FMOE_FLAG_FORCE_PER_TOKEN, or FMOE_FLAG_FORCE_GROUPED), every scale and bias
- * is first checked against that path's fp16 dequantisation: every scale must
- * be 0 or of magnitude in [2^-14, 65504], every bias at most 65504 in
- * magnitude, and |scale| * (2^bits - 1) + |bias| <= 65504 (NaN and inf fail).
- * Weights outside fail the call with UNSUPPORTED before anything is rewritten;
- * the batch-1 kernel applies scale and bias in fp32 and takes any finite value.
+ * Both paths apply the bf16 scale and bias in fp32 to exact integer codes, so
+ * any bf16 value is taken as it is.
  * Errors: INVALID_ARG (NULL, bad shapes, K > E, bits not 2/4, group != 64),
- * UNSUPPORTED (H or I above 4096, a shape whose shared-memory plan does not
- * fit, or scales/biases outside the grouped path's range), ALIGNMENT, OOM,
- * CUDA.  On error *out is NULL.
+ * UNSUPPORTED (H or I above 4096 or a shape whose shared-memory plan does not
+ * fit), ALIGNMENT, OOM, CUDA.  On error *out is NULL.
  */
 FMOE_API fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, void* stream, fmoe_ctx** out);
 

@@ -492,34 +492,6 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
     cudaGetLastError();
     return bail(fail(ctx, FMOE_ERR_OOM, "repack staging allocation failed"));
   }
-  // The grouped path dequantises in fp16: before anything is rewritten, every
-  // scale and bias must lie where that is exact (see launch_check_affine).
-  const bool grouped_used = ctx->bws_mem != nullptr &&
-                            ((c.flags & FMOE_FLAG_FORCE_GROUPED) || !(c.flags & FMOE_FLAG_FORCE_PER_TOKEN));
-  if (grouped_used) {
-    uint32_t* flag = static_cast<uint32_t*>(tmp);
-    uint32_t bad = 0;
-    e = cudaMemsetAsync(flag, 0, sizeof(uint32_t), st);
-    for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
-      const int rc = launch_check_affine(static_cast<const uint8_t*>(ctx->layers[l].experts_dev), per_layer,
-                                         c.hidden, c.inter, c.bits, flag, stream);
-      if (rc != 0) e = (cudaError_t)rc;
-    }
-    if (e == cudaSuccess) e = cudaMemcpyAsync(&bad, flag, sizeof bad, cudaMemcpyDeviceToHost, st);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    if (e != cudaSuccess) {
-      cudaFree(tmp);
-      return bail(cuda_fail(ctx, e, "scale/bias range check"));
-    }
-    if (bad) {
-      cudaFree(tmp);
-      return bail(fail(ctx, FMOE_ERR_UNSUPPORTED,
-                       "expert scales/biases outside the grouped path's fp16 range (%s%s%s%s); weights left "
-                       "unchanged -- create with FMOE_FLAG_FORCE_PER_TOKEN or max_tokens=1 to use the batch-1 kernel",
-                       (bad & kAffineNonFinite) ? " non-finite" : "", (bad & kAffineScaleRange) ? " scale" : "",
-                       (bad & kAffineBiasRange) ? " bias" : "", (bad & kAffineWeightRange) ? " |w|>65504" : ""));
-    }
-  }
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
     uint8_t* ex = static_cast<uint8_t*>(ctx->layers[l].experts_dev);
     for (int e0 = 0; e0 < per_layer; e0 += chunk) {

@@ -116,9 +116,12 @@ __device__ __forceinline__ void load16(const float* src, float (&v)[16]) {
 // with sh putting the row's largest magnitude in [2^14, 2^15) (any finite row
 // fits fp16; bf16 inputs convert exactly unless they are 2^28 times smaller
 // than the row's largest), and scale[p] = 2^-sh.  row(p) = rowmap[p], or p.
+// sums[(g / 2) * pcap + p][g % 2] = the fp32 sum of the fp16 values of 64-column
+// group g of dst[p] (the grouped GEMM's bias term).
 template <typename Src>
 __global__ void bt_prep_kernel(const Src* __restrict__ src, const int32_t* __restrict__ rowmap, int P, int K,
-                               uint16_t* __restrict__ dst, float* __restrict__ scale) {
+                               uint16_t* __restrict__ dst, float* __restrict__ scale, float* __restrict__ sums,
+                               int pcap) {
   const int lane = threadIdx.x & 31, nb = K / 16;
   for (int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x / 32)) {
     const Src* row = src + (size_t)(rowmap ? rowmap[p] : p) * K;
@@ -135,17 +138,31 @@ __global__ void bt_prep_kernel(const Src* __restrict__ src, const int32_t* __res
     const float mul = pow2(sh);
     if (lane == 0) scale[p] = pow2(-sh);
     uint16_t* drow = dst + (size_t)p * K;
-    for (int b = lane; b < nb; b += 32) {
-      float v[16];
-      load16(row + 16 * b, v);
-      uint32_t o[8];
+    // K is a multiple of 64, so the four 16-column blocks of a group are four
+    // consecutive lanes of one pass
+    for (int b0 = 0; b0 < nb; b0 += 32) {
+      const int b = b0 + lane;
+      float gsum = 0.f;
+      if (b < nb) {
+        float v[16];
+        load16(row + 16 * b, v);
+        uint32_t o[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const __half2 h = __floats2half2_rn(v[k_perm(2 * k)] * mul, v[k_perm(2 * k + 1)] * mul);
-        o[k] = *reinterpret_cast<const uint32_t*>(&h);
+        for (int k = 0; k < 8; ++k) {
+          const __half2 h = __floats2half2_rn(v[k_perm(2 * k)] * mul, v[k_perm(2 * k + 1)] * mul);
+          o[k] = *reinterpret_cast<const uint32_t*>(&h);
+          const float2 f = __half22float2(h);
+          gsum += f.x + f.y;
+        }
+        reinterpret_cast<uint4*>(drow + 16 * b)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        reinterpret_cast<uint4*>(drow + 16 * b)[1] = make_uint4(o[4], o[5], o[6], o[7]);
       }
-      reinterpret_cast<uint4*>(drow + 16 * b)[0] = make_uint4(o[0], o[1], o[2], o[3]);
-      reinterpret_cast<uint4*>(drow + 16 * b)[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      gsum += __shfl_xor_sync(0xffffffffu, gsum, 1);
+      gsum += __shfl_xor_sync(0xffffffffu, gsum, 2);
+      if (b < nb && (b & 3) == 0) {
+        const int g = b >> 2;
+        sums[((size_t)(g >> 1) * pcap + p) * 4 + (g & 1)] = gsum;
+      }
     }
   }
 }
@@ -443,11 +460,13 @@ size_t carve(uintptr_t base, int H, int E, int K, int I, int T, BatchWs& ws) {
   const int rbg = (2 * I + kGemmRows - 1) / kGemmRows, rbd = (H + kGemmRows - 1) / kGemmRows;
   // token blocks: at most P/64 full ones plus one partial per segment
   const int max_tb = (int)((P + kGemmTokens - 1) / kGemmTokens) + (E + 1);
+  ws.pcap = (int)P;
   ws.max_items_gu = rbg * max_tb;
   ws.max_items_dn = rbd * max_tb;
   ws.z = reinterpret_cast<uint16_t*>(take((size_t)T * H * 2));
   ws.zp = reinterpret_cast<uint16_t*>(take(P * H * 2));
   ws.zsc = reinterpret_cast<float*>(take(P * 4));
+  ws.zsum = reinterpret_cast<float*>(take((size_t)((H + 127) / 128) * P * 16));
   ws.logits = reinterpret_cast<float*>(take((size_t)T * E * 4));
   ws.logit_part = reinterpret_cast<float*>(take((size_t)kRtSplit * T * E * 4));
   ws.idx = reinterpret_cast<int32_t*>(take((size_t)T * K * 4));
@@ -462,6 +481,7 @@ size_t carve(uintptr_t base, int H, int E, int K, int I, int T, BatchWs& ws) {
   ws.a = reinterpret_cast<float*>(take(P * I * 4));
   ws.ap = reinterpret_cast<uint16_t*>(take(P * I * 2));
   ws.asc = reinterpret_cast<float*>(take(P * 4));
+  ws.asum = reinterpret_cast<float*>(take((size_t)((I + 127) / 128) * P * 16));
   ws.y = reinterpret_cast<float*>(take(P * H * 4));
   return off;
 }
@@ -475,8 +495,11 @@ size_t batch_ws_bytes(int H, int E, int K, int I, int T) {
 int batch_ws_carve(uint8_t* base, int H, int E, int K, int I, int T, BatchWs& ws) {
   carve(reinterpret_cast<uintptr_t>(base), H, E, K, I, T, ws);
   const int P = T * (K + 1);
-  const int rc = tc_encode_token_maps(ws.zp, H, P, ws.zmap);
-  return rc != 0 ? rc : tc_encode_token_maps(ws.ap, I, P, ws.amap);
+  int rc = tc_encode_token_maps(ws.zp, H, P, ws.zmap);
+  if (rc == 0) rc = tc_encode_token_maps(ws.ap, I, P, ws.amap);
+  if (rc == 0) rc = tc_encode_sum_maps(ws.zsum, (H + 127) / 128, P, ws.zsmap);
+  if (rc == 0) rc = tc_encode_sum_maps(ws.asum, (I + 127) / 128, P, ws.asmap);
+  return rc;
 }
 
 int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream) {
@@ -518,8 +541,9 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
   // gate/up: B = each position's token input
+  const int pcap = ws.pcap;
   bt_prep_kernel<uint16_t><<<grid_of(positions, 8, 8 * n_sm), 256, 0, st>>>(ws.z, ws.pos_tok, positions, a.H, ws.zp,
-                                                                           ws.zsc);
+                                                                           ws.zsc, ws.zsum, pcap);
   TcArgs g{};
   g.seg = ws.seg;
   g.S = a.E + 1;
@@ -535,11 +559,12 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
     if (a.gemm_events[k]) cudaEventRecord(static_cast<cudaEvent_t>(a.gemm_events[k]), st);
   };
   mark(0);
-  int rc = launch_tc_gemm(a.bits, true, *a.wmap_gu, ws.zmap, g, n_sm, stream);
+  int rc = launch_tc_gemm(a.bits, true, *a.wmap_gu, ws.zmap, ws.zsmap, g, n_sm, stream);
   if (rc != 0) return rc;
   mark(1);
   // down: B = the position's activation
-  bt_prep_kernel<float><<<grid_of(positions, 8, 8 * n_sm), 256, 0, st>>>(ws.a, nullptr, positions, a.I, ws.ap, ws.asc);
+  bt_prep_kernel<float><<<grid_of(positions, 8, 8 * n_sm), 256, 0, st>>>(ws.a, nullptr, positions, a.I, ws.ap, ws.asc,
+                                                                        ws.asum, pcap);
   g.items = ws.items_dn;
   g.n_items = ws.n_items + 1;
   g.k_chunks = (a.I + 127) / 128;
@@ -548,7 +573,7 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   g.bscale = ws.asc;
   g.out = layer ? ws.y : a.y_out;
   mark(2);
-  rc = launch_tc_gemm(a.bits, false, *a.wmap_dn, ws.amap, g, n_sm, stream);
+  rc = launch_tc_gemm(a.bits, false, *a.wmap_dn, ws.amap, ws.asmap, g, n_sm, stream);
   if (rc != 0) return rc;
   mark(3);
   if (layer) {

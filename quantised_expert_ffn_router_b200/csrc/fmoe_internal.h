@@ -255,6 +255,7 @@ struct BatchWs {              // device buffers, sized for max_tokens at create
   uint16_t* z;                // bf16 [T][H]   (normalised input)
   uint16_t* zp;               // fp16 [T*(K+1)][H] GEMM input of each position (scaled, k-permuted)
   float* zsc;                 // [T*(K+1)] 2^sh that undoes the scaling of zp
+  float* zsum;                // [H/128][T*(K+1)][4] sums of zp's 64-column groups (fp32)
   float* logits;              // [T][E]
   float* logit_part;          // [4][T][E] partial router logits (K split)
   int32_t* idx;               // [T][K]
@@ -269,9 +270,12 @@ struct BatchWs {              // device buffers, sized for max_tokens at create
   float* a;                   // [T*(K+1)][I] activations
   uint16_t* ap;               // fp16 [T*(K+1)][I] down-GEMM input (scaled, k-permuted)
   float* asc;                 // [T*(K+1)]
+  float* asum;                // [I/128][T*(K+1)][4] sums of ap's 64-column groups
   float* y;                   // [T*(K+1)][H] expert outputs
   int max_items_gu, max_items_dn;
+  int pcap;                   // positions the buffers hold: max_tokens * (K + 1)
   TmaDesc zmap[4], amap[4];   // zp / ap boxes of 16, 32, 48, 64 rows x 2 x 64 columns, 128-byte swizzle
+  TmaDesc zsmap[4], asmap[4]; // zsum / asum boxes of 16, 32, 48, 64 rows x 4 floats
 };
 
 struct BatchArgs {
@@ -320,8 +324,12 @@ int tc_encode_weight_map(const uint8_t* matrix0, int64_t blob_bytes, int n_blobs
 // Four tensor maps over an fp16 [rows][cols] matrix seen as (64 columns, rows,
 // cols/64 blocks): boxes of 16, 32, 48, 64 rows x 2 blocks, 128-byte swizzle.
 int tc_encode_token_maps(const uint16_t* base, int cols, int rows, TmaDesc* out);
-int launch_tc_gemm(int bits, bool gate_up, const TmaDesc& wmap, const TmaDesc* xmaps, const TcArgs& a, int n_sm,
-                   void* stream);
+// Four tensor maps over fp32 group sums laid out [chunks][rows][4] (per
+// 128-column chunk and row: the sums of its two 64-column groups, two unused):
+// boxes of 16, 32, 48, 64 rows x 4 floats of one chunk.
+int tc_encode_sum_maps(const float* base, int chunks, int rows, TmaDesc* out);
+int launch_tc_gemm(int bits, bool gate_up, const TmaDesc& wmap, const TmaDesc* xmaps, const TmaDesc* smaps,
+                   const TcArgs& a, int n_sm, void* stream);
 int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream);
 
 // Top-K and renormalised weights of T rows of fp32 logits (one warp per row).
@@ -342,10 +350,6 @@ int launch_route_static(const uint16_t* wr, const float* bias, const uint16_t* n
                         const uint16_t* x, int T, int H, int E, int K, int32_t* idx_out, float* w_out, void* stream);
 // 4-bit -> 2-bit requantisation of n canonical blobs (fmoe_requant.cu).
 int launch_requant(const uint8_t* src, uint8_t* dst, int n_blobs, int H, int I, int n_sm, void* stream);
-// Bits of launch_check_affine's flag word.
-constexpr uint32_t kAffineNonFinite = 1u, kAffineScaleRange = 2u, kAffineBiasRange = 4u, kAffineWeightRange = 8u;
-int launch_check_affine(const uint8_t* blobs, int n_blobs, int H, int I, int bits, uint32_t* flags_dev,
-                        void* stream);
 int decode_max_smem_optin(int device);
 int decode_occupancy(int bits, bool multi, int smem_bytes, int* blocks_per_sm);
 int zero_workspace(void* ws, size_t bytes, void* stream);

@@ -220,69 +220,7 @@ __global__ void pack_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict
   }
 }
 
-// Range check of the canonical scales and biases for the grouped path, which
-// dequantises w = q*scale + bias in fp16 (one fma.rn.f16x2 on fp16 copies of
-// the bf16 scale and bias).  A pair passes when both are finite; the scale is
-// 0 or of magnitude in [2^-14, 65504] (fp16's normal range, where every bf16
-// value converts exactly, so the weights of a group are spaced at least 2^-14
-// apart); the bias is at most 65504 in magnitude (its fp16 copy is exact from
-// 2^-17 up, and below that off by at most 2^-25, the absolute error fp16
-// rounding puts on every dequantised weight anyway); and
-// |scale|*(2^bits - 1) + |bias| <= 65504, so no weight overflows.  ORs
-// kAffine* bits into *flags.
-__global__ void check_affine_kernel(const uint8_t* __restrict__ blobs, int n_blobs, Geo g,
-                                    uint32_t* __restrict__ flags) {
-  const int64_t per_mat = (int64_t)g.H * g.I / kGroup;  // (scale, bias) pairs of one matrix
-  const int64_t total = (int64_t)n_blobs * 3 * per_mat;
-  const float qmax = (float)((1 << g.bits) - 1);
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int64_t end = (total + stride - 1) / stride * stride;  // every lane of a warp runs the same trips
-  uint32_t bad = 0;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < end; i += stride) {
-    if (i < total) {
-      const int64_t e = i / (3 * per_mat), rest = i % (3 * per_mat);
-      const int m = (int)(rest / per_mat);
-      const int64_t k = rest % per_mat;
-      // canonical matrix m: codes (R*C*bits/8 bytes), scales [R*C/64], biases [R*C/64]
-      const uint8_t* sb = blobs + e * g.blob + canon_mat_base(g, m) + (int64_t)g.H * g.I * g.bits / 8;
-      const uint32_t su = *reinterpret_cast<const uint16_t*>(sb + 2 * k);
-      const uint32_t bu = *reinterpret_cast<const uint16_t*>(sb + 2 * per_mat + 2 * k);
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const uint32_t u = j ? bu : su;
-        const uint32_t ex = (u >> 7) & 0xFFu;  // bf16 biased exponent
-        if (ex == 0xFFu) bad |= kAffineNonFinite;
-        else if (ex > 127u + 15u) bad |= j ? kAffineBiasRange : kAffineScaleRange;
-        else if (j == 0 && (u & 0x7FFFu) != 0 && ex < 127u - 14u) bad |= kAffineScaleRange;
-      }
-      const float sv = __uint_as_float(su << 16), bv = __uint_as_float(bu << 16);
-      if (fabsf(sv) * qmax + fabsf(bv) > 65504.f) bad |= kAffineWeightRange;
-    }
-    const uint32_t any = __reduce_or_sync(0xffffffffu, bad);
-    if (any && (threadIdx.x & 31) == 0) atomicOr(flags, any);
-    bad = 0;
-  }
-}
-
 }  // namespace
-
-int launch_check_affine(const uint8_t* blobs, int n_blobs, int H, int I, int bits, uint32_t* flags_dev,
-                        void* stream) {
-  Geo g;
-  g.H = H;
-  g.I = I;
-  g.bits = bits;
-  g.blob = expert_bytes(H, I, bits);
-  g.gate_bytes = canonical_matrix_bytes(I, H, bits);
-  g.gu_packed = packed_gu_bytes(H, I, bits);
-  g.tb = tile_bytes(bits);
-  g.cb = tile_code_bytes(bits);
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  check_affine_kernel<<<sms * 8, 256, 0, (cudaStream_t)stream>>>(blobs, n_blobs, g, flags_dev);
-  return (int)cudaGetLastError();
-}
 
 int launch_repack(const uint8_t* src, uint8_t* dst, int n_experts, int H, int I, int bits, int to_packed,
                   void* stream) {

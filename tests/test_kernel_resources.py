@@ -1,7 +1,9 @@
 """Build health of the CUDA sources for sm_100a, checked on the CPU: every
 kernel and device function compiles without register spills, and the fused
 decode kernel (512 threads, one block per SM) stays within 128 registers per
-thread with no stack frame.  A spill in these kernels costs far more than any
+thread with no stack frame, as does the grouped tensor-core kernel (480
+threads: four warps share a sub-partition's 16,384 registers, so a launch with
+more than 128 a thread fails).  A spill in these kernels costs far more than any
 tuning gains, so it should fail here rather than show up as a slowdown.
 (Only ptxas's resource summary is read.)"""
 import concurrent.futures
@@ -55,6 +57,9 @@ def test_no_spills_and_decode_register_budget(tmp_path):
     for src, rep in reports.items():
         for name, regs, stack, st, ld in _functions(rep):
             assert st == 0 and ld == 0, f"{os.path.basename(src)}: {name} spills ({st} B stored, {ld} B loaded)"
+            if "bt_tc_gemm_kernel" in name and regs is not None:
+                # 15 warps: an SM sub-partition holds four of them in its 16,384 registers
+                assert regs <= 128, f"{name}: {regs} registers (4 warps x 32 x 128 per sub-partition)"
             if "decode_kernel" in name and regs is not None:
                 decode_entries += 1
                 assert regs <= 128, f"{name}: {regs} registers (512 threads x 128 fill the SM)"

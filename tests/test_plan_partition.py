@@ -31,7 +31,7 @@ size_t batch_ws_bytes(int, int, int, int, int) { return 0; }
 int batch_ws_carve(uint8_t*, int, int, int, int, int, BatchWs&) { return 1; }
 int tc_encode_weight_map(const uint8_t*, int64_t, int, int, int, int, TmaDesc*) { return 1; }
 int tc_encode_token_maps(const uint16_t*, int, int, TmaDesc*) { return 1; }
-int launch_tc_gemm(int, bool, const TmaDesc&, const TmaDesc*, const TcArgs&, int, void*) { return 1; }
+int launch_tc_gemm(int, bool, const TmaDesc&, const TmaDesc*, const TmaDesc*, const TcArgs&, int, void*) { return 1; }
 int launch_batched(const BatchArgs&, const BatchWs&, int, void*) { return 1; }
 int launch_topk_rows(const float*, int, int, int, int32_t*, float*, void*) { return 1; }
 int launch_repack(const uint8_t*, uint8_t*, int, int, int, int, int, void*) { return 1; }
@@ -39,7 +39,6 @@ int launch_decode(const DecodePlan&, void*, bool, bool) { return 1; }
 int launch_route_static(const uint16_t*, const float*, const uint16_t*, float, const uint16_t*, int, int, int, int,
                         int32_t*, float*, void*) { return 1; }
 int launch_requant(const uint8_t*, uint8_t*, int, int, int, int, void*) { return 1; }
-int launch_check_affine(const uint8_t*, int, int, int, int, uint32_t*, void*) { return 1; }
 int route_static_prepare() { return 0; }
 bool route_static_ready() { return true; }
 int decode_max_smem_optin(int) { return 232448; }
