@@ -273,6 +273,34 @@ def job_throughput(ws: int, units_per_rank: int, max_ms: float) -> float:
 
 
 def run_gpu(args, wl, ws, rank, local):
+    line = measure_gpu(args, wl, ws, rank, local, args.steps, args.warmup, args.e2e_steps,
+                       cpu_baseline=ws == 1 and not args.no_cpu_baseline)
+    if line is None:
+        return 0
+    if wl.name == "layer" and ws == 1 and not args.no_workloads:
+        # the other full-size workloads, each on its own weights (freed before the next)
+        line["workloads"] = {}
+        for name, steps in (("stack4", 64), ("stack2", 32), ("batched", 30)):
+            import torch
+            torch.cuda.empty_cache()
+            w = measure_gpu(args, synth.WORKLOADS[name], ws, rank, local, steps, 3, min(steps, 16), cpu_baseline=False)
+            line["workloads"][name] = workload_summary(w)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_summary(w: dict) -> dict:
+    """The fields of a workload's bench line kept in the headline's `workloads` object."""
+    keep = ("value", "unit", "steps", "warmup", "ms_per_step", "us_per_layer", "hbm_gbs", "hbm_frac", "roofline",
+            "e2e", "gpu_launches", "clocks", "dtype", "config", "step_us_p10_p50_p90")
+    out = {k: w[k] for k in keep if k in w}
+    if "batched" in w:
+        out["batched"] = w["batched"]
+    return out
+
+
+def measure_gpu(args, wl, ws, rank, local, steps, warmup, e2e_steps, cpu_baseline):
+    """One workload's bench line (rank 0; None on other ranks)."""
     import torch
 
     import quantised_expert_ffn_router_b200 as fm
@@ -313,7 +341,6 @@ def run_gpu(args, wl, ws, rank, local):
         if flush is not None:
             flush(i)
 
-    steps, warmup = args.steps, args.warmup
     for i in range(warmup):
         maybe_flush(i)
         step(i)
@@ -367,7 +394,7 @@ def run_gpu(args, wl, ws, rank, local):
         warm_us = 1e3 * a.elapsed_time(b) / steps
 
     # end to end through the public API with host buffers (pinned), copies timed
-    e2e_steps = min(steps, args.e2e_steps)
+    e2e_steps = min(steps, e2e_steps)
     # one library call per step on page-locked host buffers: it enqueues the
     # input copy, the layer (or stack) and the output copy on the stream
     x_host = X[:min(n_batches, e2e_steps)].cpu().pin_memory()
@@ -387,9 +414,10 @@ def run_gpu(args, wl, ws, rank, local):
         e2e_ms.append(a.elapsed_time(b))
     e2e_total = max_over_ranks(ws, sum(e2e_ms))
     fm.fmoe_destroy(ctx)
+    del weights, X, OUT, x_host, out_host
 
     if rank != 0:
-        return 0
+        return None
     ms_per_step = total_ms / steps
     tps = job_throughput(ws, steps * B, total_ms)
     us_layer = 1e3 * ms_per_step / L
@@ -399,6 +427,7 @@ def run_gpu(args, wl, ws, rank, local):
         # per step: router + every distinct selected expert + the shared one, tokens in and out
         idx_h = IDX.cpu().numpy()
         uniq = [len(set(idx_h[i % n_batches].ravel().tolist())) for i in range(steps)]
+        del IDX
         bytes_launch = (wl.n_experts * wl.hidden * 2 + (statistics.mean(uniq) + 1) * wl.blob_bytes
                         + 2 * B * wl.hidden * 2)
         flops = 2 * B * (wl.top_k + 1) * 3 * wl.hidden * wl.inter + 2 * B * wl.hidden * wl.n_experts
@@ -457,13 +486,12 @@ def run_gpu(args, wl, ws, rank, local):
     }
     if tensor is not None:
         line["batched"] = tensor
-    if ws == 1 and not args.no_cpu_baseline:
+    if cpu_baseline:
         tps_cpu, done, threads, dt = oracle_tokens_per_s(wl, 400, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tps_cpu, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                 "sample": f"{done} tokens of workload '{wl.name}' ({L} layer(s) each), "
                                           f"{dt:.1f} s"}
-    print(json.dumps(line), flush=True)
-    return 0
+    return line
 
 
 # phase timestamps the trace build records per block and layer (fmoe_set_trace)
@@ -614,6 +642,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stack-per-layer", action="store_true",
                     help="stacks: one launch per layer instead of one per token (the multi-layer kernel)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="layer workload: skip the stack4 / stack2 / batched entries of the `workloads` object")
     ap.add_argument("--trace", action="store_true",
                     help="per-phase timeline of the fused kernel from the trace build (not a bench line)")
     args = ap.parse_args(argv)

@@ -125,6 +125,39 @@ FMOE_API fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* 
 
 /*
  * Passage: the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on
+ * a Laptop", section "How the SSD expert streaming pipeline works": only the
+ * K = 4 selected experts of a layer are read from storage, and the operating
+ * system's page cache (standard LRU, about 35 GB) serves roughly 71% of them.
+ * Here host memory plays the storage and an HBM pool of expert slots the page
+ * cache.
+ * As fmoe_create, except that every layers[l].experts_dev is a HOST pointer to
+ * page-locked memory (cudaHostAlloc, or cudaHostRegister with mapping)
+ * holding the layer's E + 1 canonical blobs; it is repacked in place (it must
+ * stay allocated and unmodified until destroy).  The shared experts are copied
+ * into HBM; the routed experts stay in host memory behind a cache of
+ * `cache_slots` expert slots in HBM (2 * top_k <= cache_slots; more than
+ * n_layers * n_experts are not used), shared by all layers.  The fused kernel
+ * consults the cache after routing: a hit is read from its slot; a miss is
+ * read from host memory over the host link and, as its tiles arrive, written
+ * into a slot chosen by CLOCK replacement (second chance, the textbook
+ * approximation of LRU), all in the same launch, so no host round trip is
+ * involved.  Results are bit-identical to a resident context's.  Such a
+ * context runs every call on the batch-1 kernel, one launch per layer and
+ * token; fmoe_expert_forward returns UNSUPPORTED.  Calls on one cached context
+ * must be ordered on one stream (the cache state is part of the context).
+ * Errors: as fmoe_create; INVALID_ARG also for cache_slots < 2 * top_k or
+ * experts that are not page-locked host memory.
+ */
+FMOE_API fmoe_status fmoe_create_cached(const fmoe_config* cfg, const fmoe_layer_desc* layers, int64_t cache_slots,
+                                        void* stream, fmoe_ctx** out);
+
+/* Synchronises `stream` and returns the expert-cache hit and miss counts of a
+ * cached context since create (each routed pick of each launch counts once).
+ * Errors: INVALID_ARG (no cache), CUDA. */
+FMOE_API fmoe_status fmoe_cache_stats(fmoe_ctx* ctx, void* stream, uint64_t* hits, uint64_t* misses);
+
+/*
+ * Passage: the Hysen Labs page "Flash-MoE: Running a 397B Parameter Model on
  * a Laptop", section "How the SSD expert streaming pipeline works": the second
  * command buffer normalises the layer input and computes the routing logits,
  * then the host takes a softmax and the top K; the themata summary of the same

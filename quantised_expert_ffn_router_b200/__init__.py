@@ -21,6 +21,7 @@ __all__ = [
     "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward", "fmoe_layer_forward", "fmoe_stack_forward",
     "fmoe_layer_forward_host", "fmoe_stack_forward_host", "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy", "fmoe_last_error", "EXPORTED_SYMBOLS",
     "fmoe_set_trace", "fmoe_trace_points", "fmoe_trace_layers", "fmoe_debug_set_epoch", "use_trace_build",
+    "fmoe_create_cached", "fmoe_cache_stats",
 ]
 
 FMOE_OK, FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED, FMOE_ERR_ALIGNMENT = 0, 1, 2, 3
@@ -30,7 +31,7 @@ FMOE_FLAG_FORCE_GROUPED = 0x2
 FMOE_FLAG_STACK_PER_LAYER = 0x4
 FMOE_FLAG_DEBUG_SKIP_ROUTER_RELEASE = 0x100
 
-EXPORTED_SYMBOLS = ["fmoe_expert_bytes", "fmoe_create", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward",
+EXPORTED_SYMBOLS = ["fmoe_expert_bytes", "fmoe_create", "fmoe_create_cached", "fmoe_cache_stats", "fmoe_route", "fmoe_route_static", "fmoe_expert_forward",
                     "fmoe_layer_forward", "fmoe_stack_forward", "fmoe_layer_forward_host", "fmoe_stack_forward_host",
                     "fmoe_unpack_expert", "fmoe_requant_4to2", "fmoe_set_gemm_events", "fmoe_set_trace",
                     "fmoe_trace_points", "fmoe_trace_layers", "fmoe_debug_set_epoch",
@@ -86,6 +87,9 @@ def lib():
             L.fmoe_expert_bytes.argtypes = [i32, i32, i32]
             L.fmoe_expert_bytes.restype = ctypes.c_size_t
             L.fmoe_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerDesc), P, ctypes.POINTER(P)]
+            L.fmoe_create_cached.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerDesc), ctypes.c_int64, P,
+                                             ctypes.POINTER(P)]
+            L.fmoe_cache_stats.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)]
             L.fmoe_route.argtypes = [P, i32, P, i32, P, P, P]
             L.fmoe_route_static.argtypes = [P, i32, P, i32, P, P, P]
             L.fmoe_expert_forward.argtypes = [P, i32, i32, P, i32, P, P]
@@ -104,7 +108,7 @@ def lib():
             L.fmoe_destroy.argtypes = [P]
             L.fmoe_last_error.argtypes = [P]
             L.fmoe_last_error.restype = ctypes.c_char_p
-            for name in ("fmoe_create", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
+            for name in ("fmoe_create", "fmoe_create_cached", "fmoe_cache_stats", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
                          "fmoe_stack_forward", "fmoe_layer_forward_host", "fmoe_stack_forward_host",
                          "fmoe_unpack_expert", "fmoe_poll_status", "fmoe_destroy", "fmoe_set_trace",
                          "fmoe_trace_points", "fmoe_trace_layers", "fmoe_debug_set_epoch"):
@@ -140,6 +144,25 @@ def fmoe_create(cfg: Config, layers, stream: int = 0, *, check: bool = True):
     if check:
         _check(None, st)
     return st, out.value
+
+
+def fmoe_create_cached(cfg: Config, layers, cache_slots: int, stream: int = 0, *, check: bool = True):
+    """Context whose routed experts stay in page-locked host memory (each
+    layer's experts_dev a host pointer) behind an HBM cache of `cache_slots`
+    expert slots.  Returns (status, ctx handle as int or None)."""
+    arr = (LayerDesc * len(layers))(*layers)
+    out = ctypes.c_void_p()
+    st = lib().fmoe_create_cached(ctypes.byref(cfg), arr, ctypes.c_int64(cache_slots), _vp(stream), ctypes.byref(out))
+    if check:
+        _check(None, st)
+    return st, out.value
+
+
+def fmoe_cache_stats(ctx, stream=0):
+    """(hits, misses) of a cached context's expert cache (synchronises `stream`)."""
+    h, m = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    _check(ctx, lib().fmoe_cache_stats(_vp(ctx), _vp(stream), ctypes.byref(h), ctypes.byref(m)))
+    return int(h.value), int(m.value)
 
 
 def fmoe_route(ctx, layer, x_dev, T, idx_dev, w_dev, stream=0, *, check=True) -> int:

@@ -43,6 +43,18 @@ struct fmoe_ctx {
   std::vector<TmaDesc> tc_maps;  // per layer: tensor maps of the packed gate/up and down matrices
   void* gemm_events[4] = {nullptr, nullptr, nullptr, nullptr};  // caller's timing events (fmoe_set_gemm_events)
   DecodePlan plan[3];  // per mode: layer, expert, route (pointers filled per call)
+  // host-resident routed experts (fmoe_create_cached)
+  bool cached = false;
+  int n_cache_slots = 0;
+  std::vector<const uint8_t*> host_dev;  // per layer: device address of the page-locked expert blobs
+  uint8_t* shared_dev = nullptr;         // [n_layers] packed shared experts in HBM
+  uint8_t* cache_slots = nullptr;        // [n_cache_slots] blobs in HBM
+  void* cache_state = nullptr;           // slot_of | owner | ref | hand | stats
+  int32_t* slot_of = nullptr;
+  int32_t* owner = nullptr;
+  uint8_t* ref = nullptr;
+  uint32_t* hand = nullptr;
+  unsigned long long* stats = nullptr;
   std::string err;
 };
 
@@ -232,6 +244,24 @@ DecodePlan bind(const fmoe_ctx* ctx, int mode, int layer) {
   P.flags = ctx->cfg.flags;
   P.trace = ctx->trace;
   P.timeout_ns = (uint64_t)(ctx->cfg.wait_timeout_us ? ctx->cfg.wait_timeout_us : 1000000u) * 1000ull;
+  P.cache = CacheArgs{};
+  if (ctx->cached) {
+    P.experts = ctx->host_dev[layer];
+    if (mode == kModeLayer) {
+      CacheArgs& C = P.cache;
+      C.on = 1;
+      C.n_slots = ctx->n_cache_slots;
+      C.key0 = layer * ctx->cfg.n_experts;
+      C.host = ctx->host_dev[layer];
+      C.shared = ctx->shared_dev + (size_t)layer * P.blob_bytes;
+      C.slots = ctx->cache_slots;
+      C.slot_of = ctx->slot_of;
+      C.owner = ctx->owner;
+      C.ref = ctx->ref;
+      C.hand = ctx->hand;
+      C.stats = ctx->stats;
+    }
+  }
   return P;
 }
 
@@ -319,11 +349,29 @@ const char* fmoe_last_error(const fmoe_ctx* ctx) {
   return ctx->err.c_str();
 }
 
-fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, void* stream, fmoe_ctx** out) {
+namespace {
+// fmoe_create and fmoe_create_cached: cache_slots > 0 makes a context whose
+// routed experts stay in page-locked host memory (layers[l].experts_dev is a
+// host pointer) behind an HBM cache of that many expert slots.
+fmoe_status create_impl(const fmoe_config* cfg, const fmoe_layer_desc* layers, int64_t cache_slots, void* stream,
+                        fmoe_ctx** out) {
   if (out) *out = nullptr;
   if (!cfg || !layers || !out) return fail(nullptr, FMOE_ERR_INVALID_ARG, "NULL argument");
   fmoe_config c = *cfg;
   if (c.max_tokens == 0) c.max_tokens = 256;
+  const bool cached = cache_slots > 0;
+  if (cached) {
+    // one launch per layer and token on the batch-1 kernel: the cache is
+    // consulted per launch, and the grouped path needs resident weights
+    c.flags = (c.flags | FMOE_FLAG_FORCE_PER_TOKEN | FMOE_FLAG_STACK_PER_LAYER) & ~FMOE_FLAG_FORCE_GROUPED;
+    if (cfg->flags & FMOE_FLAG_FORCE_GROUPED)
+      return fail(nullptr, FMOE_ERR_UNSUPPORTED, "host-resident experts run on the batch-1 kernel only");
+    if (cache_slots < 2 * (int64_t)c.top_k)
+      return fail(nullptr, FMOE_ERR_INVALID_ARG, "cache_slots=%lld below 2 * top_k", (long long)cache_slots);
+    if (c.n_layers > 0 && c.n_experts > 0 && (int64_t)c.n_layers * c.n_experts > INT32_MAX)
+      return fail(nullptr, FMOE_ERR_UNSUPPORTED, "n_layers * n_experts above 2^31");
+    if (cache_slots > (int64_t)c.n_layers * std::max(c.n_experts, 1)) cache_slots = (int64_t)c.n_layers * c.n_experts;
+  }
   if (c.hidden <= 0 || c.hidden % kGroup)
     return fail(nullptr, FMOE_ERR_INVALID_ARG, "hidden=%d must be a positive multiple of 64", c.hidden);
   if (c.inter <= 0 || c.inter % kGroup)
@@ -356,9 +404,26 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
     g_create_err = ctx->err;
     if (ctx->ws) cudaFree(ctx->ws);
     if (ctx->bws_mem) cudaFree(ctx->bws_mem);
+    if (ctx->shared_dev) cudaFree(ctx->shared_dev);
+    if (ctx->cache_slots) cudaFree(ctx->cache_slots);
+    if (ctx->cache_state) cudaFree(ctx->cache_state);
     delete ctx;
     return st;
   };
+  if (cached) {
+    ctx->cached = true;
+    ctx->n_cache_slots = (int)std::min<int64_t>(cache_slots, INT32_MAX);
+    for (int l = 0; l < c.n_layers; ++l) {
+      cudaPointerAttributes at{};
+      cudaError_t pe = cudaPointerGetAttributes(&at, layers[l].experts_dev);
+      if (pe != cudaSuccess || at.type != cudaMemoryTypeHost || at.devicePointer == nullptr) {
+        cudaGetLastError();
+        return bail(fail(ctx, FMOE_ERR_INVALID_ARG,
+                         "layer %d: experts must be page-locked host memory (cudaHostAlloc / cudaHostRegister)", l));
+      }
+      ctx->host_dev.push_back(static_cast<const uint8_t*>(at.devicePointer));
+    }
+  }
   cudaError_t e = cudaGetDevice(&ctx->device);
   if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "cudaGetDevice"));
   cudaDeviceGetAttribute(&ctx->n_sm, cudaDevAttrMultiProcessorCount, ctx->device);
@@ -433,7 +498,7 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
   if ((c.flags & FMOE_FLAG_FORCE_GROUPED) && !grouped_ok)
     return bail(fail(ctx, FMOE_ERR_UNSUPPORTED, "grouped path: n_experts=%d (max %d), max_tokens=%d (max %d)",
                      c.n_experts, kBatchMaxExperts, c.max_tokens, kBatchMaxTokens));
-  if ((c.max_tokens > 1 || (c.flags & FMOE_FLAG_FORCE_GROUPED)) && grouped_ok) {
+  if (!cached && (c.max_tokens > 1 || (c.flags & FMOE_FLAG_FORCE_GROUPED)) && grouped_ok) {
     const size_t bb = batch_ws_bytes(c.hidden, c.n_experts, c.top_k, c.inter, std::max(c.max_tokens, 1));
     e = cudaMalloc(&ctx->bws_mem, bb);
     if (e != cudaSuccess) {
@@ -482,29 +547,74 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
     if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "task table upload"));
   }
 
-  // In-place repack, canonical -> packed, through a bounded staging buffer.
+  // In-place repack, canonical -> packed, through a bounded staging buffer
+  // (host-resident experts: through two, the packed blobs copied back; the
+  // shared expert also kept in HBM).
   const size_t blob = (size_t)expert_bytes(c.hidden, c.inter, c.bits);
   const int per_layer = c.n_experts + 1;
   int chunk = (int)std::max<size_t>(1, std::min<size_t>((size_t)per_layer, (size_t)(256u << 20) / blob));
+  if (cached) {
+    const size_t state = ((size_t)c.n_layers * c.n_experts * 4 + 255) / 256 * 256 +
+                         ((size_t)ctx->n_cache_slots * 4 + 255) / 256 * 256 + ((size_t)ctx->n_cache_slots + 255) / 256 * 256 +
+                         256 + 256;
+    e = cudaMalloc(&ctx->shared_dev, (size_t)c.n_layers * blob);
+    if (e == cudaSuccess) e = cudaMalloc(&ctx->cache_slots, (size_t)ctx->n_cache_slots * blob);
+    if (e == cudaSuccess) e = cudaMalloc(&ctx->cache_state, state);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return bail(fail(ctx, FMOE_ERR_OOM, "expert cache allocation (%d slots of %zu bytes) failed",
+                       ctx->n_cache_slots, blob));
+    }
+    uint8_t* cs = static_cast<uint8_t*>(ctx->cache_state);
+    size_t o = 0;
+    ctx->slot_of = reinterpret_cast<int32_t*>(cs + o);
+    o += ((size_t)c.n_layers * c.n_experts * 4 + 255) / 256 * 256;
+    ctx->owner = reinterpret_cast<int32_t*>(cs + o);
+    o += ((size_t)ctx->n_cache_slots * 4 + 255) / 256 * 256;
+    ctx->ref = cs + o;
+    o += ((size_t)ctx->n_cache_slots + 255) / 256 * 256;
+    ctx->hand = reinterpret_cast<uint32_t*>(cs + o);
+    o += 256;
+    ctx->stats = reinterpret_cast<unsigned long long*>(cs + o);
+    // empty cache: no key has a slot, no slot a key, no reference bits, hand at 0
+    e = cudaMemsetAsync(ctx->slot_of, 0xFF, (size_t)c.n_layers * c.n_experts * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->owner, 0xFF, (size_t)ctx->n_cache_slots * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->ref, 0, (size_t)ctx->n_cache_slots, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->hand, 0, 512, st);
+    if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "expert cache clear"));
+  }
   void* tmp = nullptr;
+  void* tmp2 = nullptr;
   e = cudaMalloc(&tmp, (size_t)chunk * blob);
+  if (e == cudaSuccess && cached) e = cudaMalloc(&tmp2, (size_t)chunk * blob);
   if (e != cudaSuccess) {
     cudaGetLastError();
+    if (tmp) cudaFree(tmp);
     return bail(fail(ctx, FMOE_ERR_OOM, "repack staging allocation failed"));
   }
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
     uint8_t* ex = static_cast<uint8_t*>(ctx->layers[l].experts_dev);
     for (int e0 = 0; e0 < per_layer; e0 += chunk) {
       int n = std::min(chunk, per_layer - e0);
-      e = cudaMemcpyAsync(tmp, ex + (size_t)e0 * blob, (size_t)n * blob, cudaMemcpyDeviceToDevice, st);
+      uint8_t* dst = cached ? static_cast<uint8_t*>(tmp2) : ex + (size_t)e0 * blob;
+      e = cudaMemcpyAsync(tmp, ex + (size_t)e0 * blob, (size_t)n * blob, cudaMemcpyDefault, st);
       if (e != cudaSuccess) break;
-      int rc = launch_repack(static_cast<const uint8_t*>(tmp), ex + (size_t)e0 * blob, n, c.hidden, c.inter, c.bits,
-                             1, stream);
+      int rc = launch_repack(static_cast<const uint8_t*>(tmp), dst, n, c.hidden, c.inter, c.bits, 1, stream);
       if (rc != 0) { e = (cudaError_t)rc; break; }
+      if (cached) {
+        e = cudaMemcpyAsync(ex + (size_t)e0 * blob, dst, (size_t)n * blob, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess && e0 + n == per_layer)  // the chunk ends with the shared expert
+          e = cudaMemcpyAsync(ctx->shared_dev + (size_t)l * blob, dst + (size_t)(n - 1) * blob, blob,
+                              cudaMemcpyDeviceToDevice, st);
+        // the staging buffers are reused by the next chunk
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) break;
+      }
     }
   }
   cudaError_t e2 = cudaStreamSynchronize(st);
   cudaFree(tmp);
+  if (tmp2) cudaFree(tmp2);
   if (e != cudaSuccess) return bail(cuda_fail(ctx, e, "expert repack"));
   if (e2 != cudaSuccess) return bail(cuda_fail(ctx, e2, "expert repack (sync)"));
   {
@@ -512,6 +622,33 @@ fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, v
     g_live.insert(ctx);
   }
   *out = ctx;
+  return FMOE_OK;
+}
+}  // namespace
+
+fmoe_status fmoe_create(const fmoe_config* cfg, const fmoe_layer_desc* layers, void* stream, fmoe_ctx** out) {
+  return create_impl(cfg, layers, 0, stream, out);
+}
+
+fmoe_status fmoe_create_cached(const fmoe_config* cfg, const fmoe_layer_desc* layers, int64_t cache_slots,
+                               void* stream, fmoe_ctx** out) {
+  if (cache_slots <= 0) {
+    if (out) *out = nullptr;
+    return fail(nullptr, FMOE_ERR_INVALID_ARG, "cache_slots=%lld must be positive", (long long)cache_slots);
+  }
+  return create_impl(cfg, layers, cache_slots, stream, out);
+}
+
+fmoe_status fmoe_cache_stats(fmoe_ctx* ctx, void* stream, uint64_t* hits, uint64_t* misses) {
+  if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
+  if (!ctx->cached) return fail(ctx, FMOE_ERR_INVALID_ARG, "context has no expert cache");
+  unsigned long long v[2] = {0, 0};
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(v, ctx->stats, sizeof v, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "cache statistics");
+  if (hits) *hits = v[0];
+  if (misses) *misses = v[1];
   return FMOE_OK;
 }
 
@@ -525,6 +662,9 @@ fmoe_status fmoe_destroy(fmoe_ctx* ctx) {
   }
   if (ctx->ws) cudaFree(ctx->ws);
   if (ctx->bws_mem) cudaFree(ctx->bws_mem);
+  if (ctx->shared_dev) cudaFree(ctx->shared_dev);
+  if (ctx->cache_slots) cudaFree(ctx->cache_slots);
+  if (ctx->cache_state) cudaFree(ctx->cache_state);
   delete ctx;
   return FMOE_OK;
 }
@@ -634,6 +774,8 @@ fmoe_status fmoe_expert_forward(fmoe_ctx* ctx, int32_t layer, int32_t expert, co
   if (s != FMOE_OK) return s;
   if (expert < -1 || expert >= ctx->cfg.n_experts)
     return fail(ctx, FMOE_ERR_INVALID_ARG, "expert %d outside [-1, %d)", expert, ctx->cfg.n_experts);
+  if (ctx->cached)
+    return fail(ctx, FMOE_ERR_UNSUPPORTED, "host-resident experts: single-expert calls are not supported");
   if (T == 0) return FMOE_OK;
   if (!x_dev || !y_dev) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL tensor");
   if (misaligned(x_dev) || misaligned(y_dev)) return fail(ctx, FMOE_ERR_ALIGNMENT, "tensor not 16-byte aligned");
@@ -797,7 +939,9 @@ fmoe_status fmoe_unpack_expert(fmoe_ctx* ctx, int32_t layer, int32_t expert, voi
   if (misaligned(dst_dev)) return fail(ctx, FMOE_ERR_ALIGNMENT, "destination not 16-byte aligned");
   const size_t blob = (size_t)expert_bytes(ctx->cfg.hidden, ctx->cfg.inter, ctx->cfg.bits);
   const int e = expert < 0 ? ctx->cfg.n_experts : expert;
-  const uint8_t* src = static_cast<const uint8_t*>(ctx->layers[layer].experts_dev) + (size_t)e * blob;
+  const uint8_t* src = ctx->cached ? (e == ctx->cfg.n_experts ? ctx->shared_dev + (size_t)layer * blob
+                                                                : ctx->host_dev[layer] + (size_t)e * blob)
+                                   : static_cast<const uint8_t*>(ctx->layers[layer].experts_dev) + (size_t)e * blob;
   int rc = launch_repack(src, static_cast<uint8_t*>(dst_dev), 1, ctx->cfg.hidden, ctx->cfg.inter, ctx->cfg.bits, 0,
                          stream);
   if (rc != 0) return cuda_fail(ctx, (cudaError_t)rc, "unpack");

@@ -67,6 +67,17 @@ __device__ __forceinline__ void tma_load(uint32_t dst, const void* src, uint32_t
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
 }
+// smem -> global bulk copy (one bulk group per call), and waits for the
+// issuing thread's groups: until their sources are read / until complete.
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("fence.proxy.async.shared::cta;\n"
+               "cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n"
+               "cp.async.bulk.commit_group;" ::"l"(dst),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ uint64_t gtimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -379,6 +390,101 @@ __device__ __forceinline__ LayerDev layer_of(const DecodePlan& P, int l) {
   return LayerDev{P.experts, P.router_w, P.router_bias, P.norm_w};
 }
 
+// Expert cache decision for one launch, in the producer warp after top-K
+// (lane k < K holds pick k in `sel`).  Every block computes the same result
+// from the state the launch started with: a pick whose key has a slot is a
+// hit and is read from that slot; the misses are read from host memory and
+// take the CLOCK victims among the kCacheWindow slots from the hand (a slot
+// holding a hit is never one): first the unreferenced slots in sweep order,
+// then, when those run out, the referenced ones (the sweep has cleared them).
+__device__ __noinline__ void cache_assign(const DecodePlan& P, Misc* misc, int sel, int lane) {
+  const CacheArgs& C = P.cache;
+  const int K = P.K, n = C.n_slots;
+  const bool pick = lane < K;
+  const int have = pick ? C.slot_of[C.key0 + sel] : -1;
+  const bool hit = pick && have >= 0;
+  const uint32_t hits = __ballot_sync(0xffffffffu, hit), misses = __ballot_sync(0xffffffffu, pick && !hit);
+  const uint32_t hand = *C.hand;
+  const int W = min(kCacheWindow, n);
+  const int ws = (int)((hand + (uint32_t)lane) % (uint32_t)n);
+  const int wref = lane < W ? C.ref[ws] : 1;
+  bool held = false;  // window position holds one of this launch's hits
+  for (int k = 0; k < K; ++k) {
+    const int hs = __shfl_sync(0xffffffffu, have, k);
+    held = held || (((hits >> k) & 1u) && hs == ws);
+  }
+  const bool usable = lane < W && !held;
+  const uint32_t f0 = __ballot_sync(0xffffffffu, usable && wref == 0);
+  const uint32_t f1 = __ballot_sync(0xffffffffu, usable && wref != 0);
+  int vpos = -1;
+  if (pick && !hit) {
+    int r = __popc(misses & ((1u << lane) - 1u));
+    uint32_t m = f0;
+    if (r >= __popc(f0)) {
+      r -= __popc(f0);
+      m = f1;
+    }
+    for (int i = 0; i < r; ++i) m &= m - 1u;
+    vpos = __ffs(m) - 1;  // -1 only if fewer than 2K slots (the host refuses that)
+  }
+  const int victim = vpos >= 0 ? (int)((hand + (uint32_t)vpos) % (uint32_t)n) : -1;
+  const int walk = __reduce_max_sync(0xffffffffu, (uint32_t)(vpos + 1));
+  if (pick) {
+    const int slot = hit ? have : victim;
+    misc->cslot[1 + lane] = slot;
+    misc->chit[1 + lane] = hit ? 1 : 0;
+    misc->slot_src[1 + lane] = hit ? C.slots + (int64_t)slot * P.blob_bytes : C.host + (int64_t)sel * P.blob_bytes;
+    misc->slot_dst[1 + lane] = (hit || slot < 0) ? nullptr : C.slots + (int64_t)slot * P.blob_bytes;
+  }
+  if (lane == 0) {
+    misc->chand = (int)hand;
+    misc->cwalk = walk;
+  }
+}
+
+// Applies a launch's cache decision (the last block out, one thread).  After
+// an aborted launch the victims' contents are incomplete, so they are dropped
+// from the cache instead.
+__device__ void cache_update(const DecodePlan& P, const Misc* misc, bool aborted) {
+  const CacheArgs& C = P.cache;
+  const int K = P.K, n = C.n_slots;
+  if (aborted) {
+    for (int k = 1; k <= K; ++k) {
+      const int v = misc->cslot[k];
+      if (misc->chit[k] || v < 0 || v >= n) continue;
+      const int old = C.owner[v];
+      if (old >= 0) C.slot_of[old] = -1;
+      C.owner[v] = -1;
+      C.ref[v] = 0;
+    }
+    return;
+  }
+  for (int w = 0; w < misc->cwalk; ++w) {  // the sweep clears what it passed
+    const int sl = (int)(((uint32_t)misc->chand + (uint32_t)w) % (uint32_t)n);
+    bool mine = false;
+    for (int k = 1; k <= K; ++k) mine = mine || misc->cslot[k] == sl;
+    if (!mine) C.ref[sl] = 0;
+  }
+  unsigned long long h = 0, m = 0;
+  for (int k = 1; k <= K; ++k) {
+    const int v = misc->cslot[k], key = C.key0 + misc->slot_e[k];
+    if (v < 0 || v >= n) continue;  // no decision recorded (cannot happen after routing)
+    if (misc->chit[k]) {
+      ++h;
+    } else {
+      const int old = C.owner[v];
+      if (old >= 0) C.slot_of[old] = -1;
+      C.owner[v] = key;
+      C.slot_of[key] = v;
+      ++m;
+    }
+    C.ref[v] = 1;
+  }
+  *C.hand = (uint32_t)(((uint32_t)misc->chand + (uint32_t)misc->cwalk) % (uint32_t)n);
+  C.stats[0] += h;
+  C.stats[1] += m;
+}
+
 #ifdef FMOE_TRACE
 // Phase timestamps (%globaltimer) of this block for the first kTraceLayers
 // layers: SET once by one thread, FIRST by the first of several threads
@@ -464,6 +570,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       misc->rcnt[lane] = 0;
       misc->slot_e[lane] = (lane == 0) ? (P.mode == kModeExpert ? P.expert_id : P.E) : 0;
       misc->slot_w[lane] = (lane == 0) ? 1.f : 0.f;
+      misc->slot_src[lane] = (lane == 0) ? P.cache.shared : nullptr;  // cached contexts: the shared expert
+      misc->slot_dst[lane] = nullptr;
+      misc->cslot[lane] = -1;
+      misc->chit[lane] = 1;
     }
     misc->unit_cnt[lane] = 0;
     misc->dn_cnt[lane] = 0;
@@ -556,6 +666,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (cta == 0 && P.w_out) P.w_out[lane] = w;
       }
       __syncwarp();
+      if (P.cache.on && P.mode == kModeLayer) {
+        cache_assign(P, misc, my_sel, lane);
+        __syncwarp();
+      }
       if (lane == 0) FMOE_TRACE_SET(cur, 4);
       return true;
     };
@@ -592,17 +706,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const int c0 = (int)c * P.router_part_cols;
         src = Ld.router_w + (int64_t)(cta + (int)idx * G) * P.H + c0;
         bytes = (uint32_t)min(P.router_part_cols, P.H - c0) * 2;
-      } else if (ty == kTaskGateUp) {
-        const int u = cta + (int)idx * G, rb = u % P.units_per_slot;
-        const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
-        src = Ld.experts + (int64_t)misc->slot_e[slot] * P.blob_bytes + ((int64_t)rb * P.gu_tiles + c * kChunkTiles) * TB;
-        bytes = (uint32_t)(n * TB);
       } else {
-        const int rbg = first_rb + (int)idx * G;
-        const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
-        src = Ld.experts + (int64_t)misc->slot_e[slot] * P.blob_bytes + packed_gu_bytes(P.H, P.I, BITS) +
-              ((int64_t)rbg * P.dn_tiles + c * kChunkTiles) * TB;
-        bytes = (uint32_t)(n * TB);
+        // the expert's blob: resident, or (cached contexts) its cache slot or host copy
+        const uint8_t* blob =
+            P.cache.on ? misc->slot_src[slot] : Ld.experts + (int64_t)misc->slot_e[slot] * P.blob_bytes;
+        if (ty == kTaskGateUp) {
+          const int u = cta + (int)idx * G, rb = u % P.units_per_slot;
+          const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
+          src = blob + ((int64_t)rb * P.gu_tiles + c * kChunkTiles) * TB;
+          bytes = (uint32_t)(n * TB);
+        } else {
+          const int rbg = first_rb + (int)idx * G;
+          const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
+          src = blob + packed_gu_bytes(P.H, P.I, BITS) + ((int64_t)rbg * P.dn_tiles + c * kChunkTiles) * TB;
+          bytes = (uint32_t)(n * TB);
+        }
       }
       mbar_expect_tx(bar_full + 8u * s, bytes);
       tma_load(dst, src, bytes, bar_full + 8u * s);
@@ -662,9 +780,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (P.mode == kModeLayer && !routed) routed = do_routing();
         if (routed || P.mode != kModeLayer) issue_downs();
       }
-      // routing still owed for the output indices
-      if (!__any_sync(0xffffffffu, *abort_flag) && !routed && has_router && cta == 0 && (P.idx_out || P.w_out))
-        do_routing();
+      // routing still owed for the output indices, and (cached contexts) by
+      // every block, since the last one out records the cache decision
+      if (!__any_sync(0xffffffffu, *abort_flag) && !routed && has_router &&
+          ((cta == 0 && (P.idx_out || P.w_out)) || (P.cache.on && P.mode == kModeLayer)))
+        routed = do_routing();
     }
   } else {
     // ============================================================ consumer warps
@@ -831,6 +951,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const uint8_t* stage = smem + P.off_ring + (uint32_t)s * P.stage_bytes;
         const uint32_t t = tasks[i];
         const uint32_t ty = task_type(t), idx = task_idx(t), slot = task_slot(t), c = task_chunk(t);
+        // cached contexts: a routed expert read from host memory is also
+        // written into its victim slot, tile range by tile range, as it lands
+        if (P.cache.on && ty != kTaskRouter && lane == 0 && misc->slot_dst[slot] != nullptr) {
+          int64_t off;
+          int n;
+          if (ty == kTaskGateUp) {
+            const int rb = (cta + (int)idx * G) % P.units_per_slot;
+            n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
+            off = ((int64_t)rb * P.gu_tiles + c * kChunkTiles) * TB;
+          } else {
+            n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
+            off = packed_gu_bytes(P.H, P.I, BITS) + ((int64_t)(first_rb + (int)idx * G) * P.dn_tiles + c * kChunkTiles) * TB;
+          }
+          bulk_store(misc->slot_dst[slot] + off, smem_u32(stage), (uint32_t)(n * TB));
+        }
         // The shared expert's chunks arrive with the router rows (or before
         // them, past a launch's first layer): they wait until this block's
         // router rows are published, so that the router rows have the SM to
@@ -1029,6 +1164,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         __syncwarp();
         if (lane == 0) {
+          if (P.cache.on) bulk_wait_read();  // a cache fill from this stage has read it
           mbar_arrive(bar_empty + 8u * s);
           if (ty == kTaskDown) FMOE_TRACE_LAST(cur, 11);
         }
@@ -1057,6 +1193,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
       }
     }
+    if (P.cache.on && lane == 0) bulk_wait_all();  // cache fills complete before the block reports out
   }
   __syncthreads();
 
@@ -1096,12 +1233,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     FMOE_TRACE_SET(0, 13);
     // the last block out advances the epoch for the next launch
     uint32_t old;
-    asm volatile("atom.release.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&P.ws->exit_count) : "memory");
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&P.ws->exit_count) : "memory");
     if (old == (uint32_t)G - 1) {
       P.ws->exit_count = 0;
       P.ws->router_cnt = 0;
       for (int k = 0; k < 16; ++k) P.ws->h_cnt[k] = 0;
       P.ws->epoch = misc->tag;
+      if (P.cache.on && P.mode == kModeLayer)
+        cache_update(P, misc, aborted || *reinterpret_cast<volatile uint32_t*>(&P.ws->status) != 0u);
     }
   }
 }

@@ -109,6 +109,16 @@ struct Misc {
   int n_tasks;          // length of this block's task list
   int rdone;            // router rows of this block published in the current layer
   int pad[12];
+  // expert cache (contexts with host-resident experts): per slot the blob base
+  // the copies read, the cache slot a miss fills (null on a hit) and the slot
+  // index / hit flag the last block out records; the CLOCK hand advance
+  const uint8_t* slot_src[16];
+  uint8_t* slot_dst[16];
+  int cslot[16];
+  int chit[16];
+  int cwalk;
+  int chand;
+  int cpad[14];
   int aflag[32];        // per (slot, half) activation fragments: 0 none, 1 building, 2 ready
   int rcnt[16];         // parts finished per router row of this block
   float rpart[16][4];   // partial logits per router row and part
@@ -116,6 +126,28 @@ struct Misc {
   int dn_cnt[32];       // K-chunks finished per (row block, slot) down job
   int last_task[64];    // last task issued into each ring stage (-1: none)
   float red[16];        // RMSNorm scratch
+};
+
+// Host-resident routed experts with an HBM cache (fmoe_create_cached), as
+// the fused kernel sees them for one layer.  Slots are shared by all layers
+// (key = layer * E + expert) and replaced by CLOCK (second chance): the hand
+// sweeps the slots, a slot whose reference bit is set loses the bit and is
+// skipped, the first unreferenced one is the victim; a hit or a fill sets the
+// bit.  Every block derives the same decision from the state the launch
+// starts with; the last block out applies it.
+constexpr int kCacheWindow = 32;  // slots from the hand a launch may sweep
+struct CacheArgs {
+  int on;
+  int n_slots;
+  int key0;                  // layer * E
+  const uint8_t* host;       // the layer's packed routed blobs, device-mapped page-locked host memory
+  const uint8_t* shared;     // the layer's packed shared expert in HBM
+  uint8_t* slots;            // [n_slots] blobs in HBM
+  int32_t* slot_of;          // [n_layers * E]: cache slot of a key, or -1
+  int32_t* owner;            // [n_slots]: key held, or -1
+  uint8_t* ref;              // [n_slots]: reference bits
+  uint32_t* hand;            // CLOCK hand
+  unsigned long long* stats; // [2]: hits, misses
 };
 
 // Per-layer weights of a multi-layer launch (device array, one entry per layer).
@@ -191,6 +223,7 @@ struct DecodePlan {
   const LayerDev* layer_dev;
   uint64_t* ws_h;          // [H] tagged
   unsigned long long* trace;  // FMOE_TRACE builds: [grid][kTraceLayers][kTracePoints] stamps, or null
+  CacheArgs cache;         // host-resident experts (single-layer launches, layer mode)
 };
 
 // Ring position of task i: issued by producer lane i % n_issuers into that
