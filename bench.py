@@ -285,8 +285,92 @@ def run_gpu(args, wl, ws, rank, local):
             torch.cuda.empty_cache()
             w = measure_gpu(args, synth.WORKLOADS[name], ws, rank, local, steps, 3, min(steps, 16), cpu_baseline=False)
             line["workloads"][name] = workload_summary(w)
+        import torch
+        torch.cuda.empty_cache()
+        line["workloads"]["cached"] = measure_cached()
     print(json.dumps(line), flush=True)
     return 0
+
+
+def measure_cached(steps: int = 200) -> dict:
+    """Host-resident experts behind the HBM expert cache (fmoe_create_cached),
+    on the single-layer shape: us/layer and hit rate with a cold cache (2K
+    slots, uniform routing), with a Zipf(1.1)-skewed router and 64 slots, and
+    with every expert cached; the host->HBM rate the misses stream at, next to
+    a plain pinned host->device copy of the same link."""
+    import ctypes
+    import dataclasses
+
+    import torch
+
+    import quantised_expert_ffn_router_b200 as fm
+    from synth.gpu import DeviceLayer, tokens
+
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    out = {}
+    # the link: one pinned 256 MB host->device copy, timed on the stream
+    hb = torch.empty(256 << 20, dtype=torch.uint8, pin_memory=True)
+    db = torch.empty_like(hb, device="cuda")
+    for _ in range(3):
+        db.copy_(hb, non_blocking=True)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(5):
+        db.copy_(hb, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    out["link_h2d_gbs"] = 5 * hb.numel() / (a.elapsed_time(b) * 1e-3) / 1e9
+    del hb, db
+    base = synth.WORKLOADS["layer"]
+    cases = (("cold", base, 2 * base.top_k), ("zipf", dataclasses.replace(base, name="layer_zipf", zipf=1.1), 64),
+             ("warm", base, base.n_experts))
+    for name, wl, n_slots in cases:
+        E, K = wl.n_experts, wl.top_k
+        blob = wl.blob_bytes
+        host = torch.empty((E + 1) * blob, dtype=torch.uint8, pin_memory=True)
+        p = wl.params(0)
+        synth.host().synth_gen_experts(ctypes.byref(p), 0, E + 1, ctypes.c_void_p(host.data_ptr()))
+        dl = DeviceLayer(wl, 0, sp)
+        d = dl.desc()
+        d["experts_dev"] = host.data_ptr()
+        del dl.experts  # routed experts are read from host memory only
+        cfg = fm.Config(wl.hidden, E, K, wl.inter, wl.bits, 64, 1, 1, wl.rms_eps, 0, 0)
+        _, ctx = fm.fmoe_create_cached(cfg, [fm.LayerDesc(**d)], n_slots, sp)
+        X = tokens(wl, range(steps))
+        Y = torch.empty_like(X)
+        n_warm = steps if name == "warm" else 8  # warm: every token once, so every expert it picks is cached
+        for i in range(n_warm):
+            fm.fmoe_layer_forward(ctx, 0, X[i].data_ptr(), 1, Y[i].data_ptr(), None, None, sp)
+        h0, m0 = fm.fmoe_cache_stats(ctx, sp)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(steps):
+            fm.fmoe_layer_forward(ctx, 0, X[i].data_ptr(), 1, Y[i].data_ptr(), None, None, sp)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        h1, m1 = fm.fmoe_cache_stats(ctx, sp)
+        st, word = fm.fmoe_poll_status(ctx, sp)
+        if st != 0:
+            raise RuntimeError(f"device status 0x{word:x} (cached {name})")
+        fm.fmoe_destroy(ctx)
+        hits, misses = h1 - h0, m1 - m0
+        out[name] = {"cache_slots": n_slots, "router": "Zipf(s=1.1)" if wl.zipf else "uniform",
+                     "us_per_layer": 1e3 * ms / steps, "tokens_per_s": steps / (ms * 1e-3),
+                     "hit_rate": hits / max(hits + misses, 1), "hits": hits, "misses": misses,
+                     "host_gbs": misses * blob / (ms * 1e-3) / 1e9}
+        del host, dl, X, Y
+        torch.cuda.empty_cache()
+    cold, warm = out["cold"], out["warm"]
+    if cold["misses"] > 0:
+        # what a missed expert adds to a layer, and the rate that implies
+        per_miss_us = (cold["us_per_layer"] - warm["us_per_layer"]) / (cold["misses"] / steps)
+        out["us_per_missed_expert"] = per_miss_us
+        out["missed_expert_gbs"] = base.blob_bytes / (per_miss_us * 1e-6) / 1e9
+    out["shape"] = "H4096 E512 top4+1shared I1024 4-bit g64, batch 1, one layer"
+    out["steps"] = steps
+    return out
 
 
 def workload_summary(w: dict) -> dict:
@@ -413,6 +497,25 @@ def measure_gpu(args, wl, ws, rank, local, steps, warmup, e2e_steps, cpu_baselin
         stream.synchronize()
         e2e_ms.append(a.elapsed_time(b))
     e2e_total = max_over_ranks(ws, sum(e2e_ms))
+    # where the end-to-end time goes: the same step as three separately timed
+    # parts (copy in, device call, copy out) with the stream's own copies
+    parts = []
+    xd, od = torch.empty_like(X[0]), torch.empty_like(OUT[0])
+    for i in range(min(e2e_steps, 50)):
+        maybe_flush(i)
+        j = i % len(x_host)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        xd.copy_(x_host[j], non_blocking=True)
+        ev[1].record(stream)
+        step(i, xd.data_ptr(), od.data_ptr())
+        ev[2].record(stream)
+        out_host[j].copy_(od, non_blocking=True)
+        ev[3].record(stream)
+        stream.synchronize()
+        parts.append([ev[k].elapsed_time(ev[k + 1]) for k in range(3)])
+    e2e_parts_us = [1e3 * statistics.mean(p[k] for p in parts) for k in range(3)]
+    del xd, od
     fm.fmoe_destroy(ctx)
     del weights, X, OUT, x_host, out_host
 
@@ -480,7 +583,13 @@ def measure_gpu(args, wl, ws, rank, local, steps, warmup, e2e_steps, cpu_baselin
         "step_us_p10_p50_p90": [1e3 * q for q in statistics.quantiles(step_ms, n=10)[0::4]] if steps >= 10 else None,
         "warm_l2_us_per_layer": warm_us,
         "e2e": {"value": job_throughput(ws, e2e_steps * B, e2e_total), "unit": "tokens/s",
-                "h2d_bytes_per_step": B * wl.hidden * 2, "d2h_bytes_per_step": B * wl.hidden * 2},
+                "h2d_bytes_per_step": B * wl.hidden * 2, "d2h_bytes_per_step": B * wl.hidden * 2,
+                "us_per_step": 1e3 * e2e_total / e2e_steps,
+                "path": ("page-locked buffers: input read over the link by a stage-in kernel, output written "
+                         "to host memory by the fused kernel" if not batched else
+                         "one copy-engine transfer each way around the grouped path"),
+                "breakdown_copy_engine_us": {"h2d": e2e_parts_us[0], "device": e2e_parts_us[1],
+                                             "d2h": e2e_parts_us[2]}},
         "gpu_launches": steps * (BATCHED_LAUNCHES if batched else (L if per_layer or not stacked else 1)),
         "clocks": clocks,
     }

@@ -255,15 +255,20 @@ FMOE_API fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int3
 
 /*
  * fmoe_layer_forward / fmoe_stack_forward on HOST buffers: h_in_host (bf16
- * [T][H]) is copied into the context's device staging buffer, the device path
- * runs on it, and h_out_host (bf16 [T][H]) and, when not NULL, idx_out_host
- * (int32 [T][K]) and w_out_host (fp32 [T][K]) are copied back.  Everything is
- * enqueued on `stream` with one cudaMemcpyAsync per buffer and the call
+ * [T][H]) is brought into the context's device staging buffer, the device
+ * path runs on it, and h_out_host (bf16 [T][H]) and, when not NULL,
+ * idx_out_host (int32 [T][K]) and w_out_host (fp32 [T][K]) receive the
+ * results.  When every buffer is page-locked and mapped into the device's
+ * address space (cudaHostAlloc, or cudaHostRegister with mapping; h_in_host
+ * 16-byte aligned) and the call runs on the batch-1 kernel, no copy engine is
+ * involved: a small kernel reads the input over the host link and the fused
+ * kernel writes the outputs straight into host memory.  Otherwise (pageable
+ * buffers, or the grouped path) each buffer is one cudaMemcpyAsync; pageable
+ * copies block the host.  Everything is enqueued on `stream` and the call
  * returns without synchronising; the caller synchronises `stream` before
- * reading the outputs and keeps the buffers alive until then.  Page-locked
- * buffers (cudaHostAlloc / cudaHostRegister) keep the copies asynchronous;
- * pageable ones work but their copies block the host.  The staging buffers
- * are per context, so h_in_host and h_out_host may be the same buffer.
+ * reading the outputs and keeps the buffers alive until then.  The input is
+ * staged per context before anything is written, so h_in_host and h_out_host
+ * may be the same buffer.
  * Results are bit-identical to the device-pointer calls.  Errors: as the
  * device-pointer calls (no alignment rule on host buffers), FMOE_ERR_CUDA when
  * a copy cannot be enqueued.

@@ -898,6 +898,38 @@ static fmoe_status copy_async(fmoe_ctx* ctx, void* dst, const void* src, size_t 
   return FMOE_OK;
 }
 
+namespace {
+// Device address of page-locked, device-mapped host memory, or null (pageable
+// memory, or a query that fails).
+void* mapped_host(const void* p) {
+  if (p == nullptr) return nullptr;
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
+// Reads `bytes` (a multiple of 16) from mapped host memory into device memory:
+// a few blocks of 16-byte loads over the host link, one round trip for an 8 KB
+// token instead of a copy-engine transfer.
+__global__ void stage_in_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n16) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = src[i];
+}
+
+// The input of a host-buffer call into the context's staging buffer.
+fmoe_status stage_in(fmoe_ctx* ctx, const void* src_mapped, size_t bytes, void* stream) {
+  const size_t n16 = bytes / 16;  // H is a multiple of 64: bf16 rows are multiples of 16 bytes
+  const int blocks = (int)std::min<size_t>((n16 + 255) / 256, (size_t)ctx->n_sm);
+  stage_in_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<const uint4*>(src_mapped),
+                                                                        reinterpret_cast<uint4*>(ctx->io_in), n16);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FMOE_OK : cuda_fail(ctx, e, "input stage-in launch");
+}
+}  // namespace
+
 fmoe_status fmoe_layer_forward_host(fmoe_ctx* ctx, int32_t layer, const void* h_in_host, int32_t T, void* h_out_host,
                                     int32_t* idx_out_host, float* w_out_host, void* stream) {
   if (!alive(ctx)) return fail(nullptr, FMOE_ERR_INVALID_ARG, "invalid or destroyed context");
@@ -906,6 +938,21 @@ fmoe_status fmoe_layer_forward_host(fmoe_ctx* ctx, int32_t layer, const void* h_
   if (T == 0) return FMOE_OK;
   if (!h_in_host || !h_out_host) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL buffer");
   const size_t bytes = (size_t)T * ctx->cfg.hidden * 2, kbytes = (size_t)T * ctx->cfg.top_k * 4;
+  if (!use_batched(ctx, T)) {
+    // page-locked buffers: the input is read over the link by a small kernel
+    // and the fused kernel writes its outputs straight into host memory
+    void* in = mapped_host(h_in_host);
+    void* out = mapped_host(h_out_host);
+    void* idx = mapped_host(idx_out_host);
+    void* w = mapped_host(w_out_host);
+    if (in && out && !misaligned(in) && (!idx_out_host || idx) && (!w_out_host || w)) {
+      s = stage_in(ctx, in, bytes, stream);
+      if (s == FMOE_OK)
+        s = layer_tokens(ctx, layer, ctx->io_in, T, static_cast<uint16_t*>(out), static_cast<int32_t*>(idx),
+                         static_cast<float*>(w), stream);
+      return s;
+    }
+  }
   s = copy_async(ctx, ctx->io_in, h_in_host, bytes, cudaMemcpyHostToDevice, stream);
   if (s == FMOE_OK)
     s = layer_tokens(ctx, layer, ctx->io_in, T, ctx->io_out, idx_out_host ? ctx->io_idx : nullptr,
@@ -924,6 +971,15 @@ fmoe_status fmoe_stack_forward_host(fmoe_ctx* ctx, int32_t layer_begin, int32_t 
   if (T == 0) return FMOE_OK;
   if (!h_in_host || !h_out_host) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL buffer");
   const size_t bytes = (size_t)T * ctx->cfg.hidden * 2;
+  if (!use_batched(ctx, T)) {  // page-locked buffers: as fmoe_layer_forward_host
+    void* in = mapped_host(h_in_host);
+    void* out = mapped_host(h_out_host);
+    if (in && out && !misaligned(in)) {
+      s = stage_in(ctx, in, bytes, stream);
+      if (s == FMOE_OK) s = stack_tokens(ctx, layer_begin, layer_end, ctx->io_in, T, out, stream);
+      return s;
+    }
+  }
   s = copy_async(ctx, ctx->io_in, h_in_host, bytes, cudaMemcpyHostToDevice, stream);
   if (s == FMOE_OK) s = stack_tokens(ctx, layer_begin, layer_end, ctx->io_in, T, ctx->io_out, stream);
   if (s == FMOE_OK) s = copy_async(ctx, h_out_host, ctx->io_out, bytes, cudaMemcpyDeviceToHost, stream);

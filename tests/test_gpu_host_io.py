@@ -1,8 +1,11 @@
 """The host-buffer entry points (fmoe_layer_forward_host,
-fmoe_stack_forward_host) against the device-pointer calls: the staging copies
-must leave results bit-identical, for one token, several tokens (token by
-token and on the grouped path) and a multi-layer stack, with the expert
-indices and weights, and with the input and output in one host buffer."""
+fmoe_stack_forward_host) against the device-pointer calls: results must be
+bit-identical, for one token, several tokens (token by token and on the
+grouped path) and a multi-layer stack, with the expert indices and weights,
+and with the input and output in one host buffer.  Page-locked buffers take
+the path without copy-engine transfers (input read over the link by a
+stage-in kernel, outputs written to host memory by the fused kernel);
+pageable buffers take the copies."""
 import dataclasses
 
 import numpy as np
@@ -59,6 +62,26 @@ def test_layer_host_equals_device(torch, T):
         m.fm.fmoe_layer_forward_host(m.ctx, 0, xh.data_ptr(), T, xh.data_ptr(), None, None, m.stream)
         torch.cuda.synchronize()
         assert torch.equal(xh.view(torch.int16), out.cpu().view(torch.int16))
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_layer_host_pageable_equals_device(torch, T):
+    wl = TINY
+    x = _x(wl, T, start=60)
+    with Model(wl) as m:
+        out = torch.empty_like(x)
+        idx = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+        m.fm.fmoe_layer_forward(m.ctx, 0, x.data_ptr(), T, out.data_ptr(), idx.data_ptr(), w.data_ptr(), m.stream)
+        xh = x.cpu()  # pageable
+        oh, ih, wh = torch.empty_like(xh), torch.empty_like(idx.cpu()), torch.empty_like(w.cpu())
+        m.fm.fmoe_layer_forward_host(m.ctx, 0, xh.data_ptr(), T, oh.data_ptr(), ih.data_ptr(), wh.data_ptr(),
+                                     m.stream)
+        torch.cuda.synchronize()
+        st, word = m.fm.fmoe_poll_status(m.ctx, m.stream)
+        assert st == 0, hex(word)
+        assert torch.equal(oh.view(torch.int16), out.cpu().view(torch.int16))
+        assert torch.equal(ih, idx.cpu()) and torch.equal(wh, w.cpu())
 
 
 def test_stack_host_equals_device(torch):
