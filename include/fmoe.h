@@ -260,8 +260,9 @@ FMOE_API fmoe_status fmoe_stack_forward(fmoe_ctx* ctx, int32_t layer_begin, int3
  * idx_out_host (int32 [T][K]) and w_out_host (fp32 [T][K]) receive the
  * results.  When every buffer is page-locked and mapped into the device's
  * address space (cudaHostAlloc, or cudaHostRegister with mapping; h_in_host
- * 16-byte aligned) and the call runs on the batch-1 kernel, no copy engine is
- * involved: a small kernel reads the input over the host link and the fused
+ * 16-byte aligned), lies inside one page-locked allocation (checked through the
+ * driver's pointer range) and the call runs on the batch-1 kernel, no copy
+ * engine is involved: a small kernel reads the input over the host link and the fused
  * kernel writes the outputs straight into host memory.  Otherwise (pageable
  * buffers, or the grouped path) each buffer is one cudaMemcpyAsync; pageable
  * copies block the host.  Everything is enqueued on `stream` and the call

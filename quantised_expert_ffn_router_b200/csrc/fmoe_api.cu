@@ -1,5 +1,6 @@
 // fmoe_api.cu -- C ABI (include/fmoe.h): contexts, argument validation,
 // shared-memory plans and kernel launches.  No compute happens on the host.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -899,16 +900,43 @@ static fmoe_status copy_async(fmoe_ctx* ctx, void* dst, const void* src, size_t 
 }
 
 namespace {
-// Device address of page-locked, device-mapped host memory, or null (pageable
-// memory, or a query that fails).
-void* mapped_host(const void* p) {
+using PointerAttrFn = CUresult (*)(void*, CUpointer_attribute, CUdeviceptr);
+PointerAttrFn pointer_attr_fn() {
+  static PointerAttrFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuPointerGetAttribute", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PointerAttrFn>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// Device address of `bytes` of page-locked, device-mapped host memory at p, or
+// null: for pageable memory, a failed query, or a buffer that does not lie
+// inside one page-locked allocation (a kernel reading or writing past its end
+// would fault; the copy path reports the error on the host instead).
+void* mapped_host(const void* p, size_t bytes) {
   if (p == nullptr) return nullptr;
   cudaPointerAttributes at{};
   if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
     cudaGetLastError();
     return nullptr;
   }
-  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+  if (at.type != cudaMemoryTypeHost || at.devicePointer == nullptr) return nullptr;
+  PointerAttrFn fn = pointer_attr_fn();
+  if (fn == nullptr) return nullptr;
+  CUdeviceptr start = 0;
+  size_t size = 0;
+  const CUdeviceptr addr = (CUdeviceptr)(uintptr_t)p;
+  if (fn(&start, CU_POINTER_ATTRIBUTE_RANGE_START_ADDR, addr) != CUDA_SUCCESS ||
+      fn(&size, CU_POINTER_ATTRIBUTE_RANGE_SIZE, addr) != CUDA_SUCCESS)
+    return nullptr;
+  if (addr < start || bytes > size || addr - start > size - bytes) return nullptr;
+  return at.devicePointer;
 }
 
 // Reads `bytes` (a multiple of 16) from mapped host memory into device memory:
@@ -941,10 +969,10 @@ fmoe_status fmoe_layer_forward_host(fmoe_ctx* ctx, int32_t layer, const void* h_
   if (!use_batched(ctx, T)) {
     // page-locked buffers: the input is read over the link by a small kernel
     // and the fused kernel writes its outputs straight into host memory
-    void* in = mapped_host(h_in_host);
-    void* out = mapped_host(h_out_host);
-    void* idx = mapped_host(idx_out_host);
-    void* w = mapped_host(w_out_host);
+    void* in = mapped_host(h_in_host, bytes);
+    void* out = mapped_host(h_out_host, bytes);
+    void* idx = mapped_host(idx_out_host, kbytes);
+    void* w = mapped_host(w_out_host, kbytes);
     if (in && out && !misaligned(in) && (!idx_out_host || idx) && (!w_out_host || w)) {
       s = stage_in(ctx, in, bytes, stream);
       if (s == FMOE_OK)
@@ -972,8 +1000,8 @@ fmoe_status fmoe_stack_forward_host(fmoe_ctx* ctx, int32_t layer_begin, int32_t 
   if (!h_in_host || !h_out_host) return fail(ctx, FMOE_ERR_INVALID_ARG, "NULL buffer");
   const size_t bytes = (size_t)T * ctx->cfg.hidden * 2;
   if (!use_batched(ctx, T)) {  // page-locked buffers: as fmoe_layer_forward_host
-    void* in = mapped_host(h_in_host);
-    void* out = mapped_host(h_out_host);
+    void* in = mapped_host(h_in_host, bytes);
+    void* out = mapped_host(h_out_host, bytes);
     if (in && out && !misaligned(in)) {
       s = stage_in(ctx, in, bytes, stream);
       if (s == FMOE_OK) s = stack_tokens(ctx, layer_begin, layer_end, ctx->io_in, T, out, stream);

@@ -58,6 +58,15 @@ def test_layer_host_equals_device(torch, T):
         assert torch.equal(oh.view(torch.int16), out.cpu().view(torch.int16))
         assert torch.equal(ih, idx.cpu())
         assert torch.equal(wh, w.cpu())
+        # buffers at an offset inside larger page-locked allocations
+        big_in = torch.empty((2 * T, wl.hidden), dtype=x.dtype, pin_memory=True)
+        big_out = torch.zeros((3 * T, wl.hidden), dtype=x.dtype, pin_memory=True)
+        big_in[T:].copy_(x.cpu())
+        m.fm.fmoe_layer_forward_host(m.ctx, 0, big_in[T:].data_ptr(), T, big_out[T:2 * T].data_ptr(), None, None,
+                                     m.stream)
+        torch.cuda.synchronize()
+        assert torch.equal(big_out[T:2 * T].view(torch.int16), out.cpu().view(torch.int16))
+        assert not big_out[:T].view(torch.int16).any() and not big_out[2 * T:].view(torch.int16).any()
         # input and output in one host buffer: the staging makes that safe
         m.fm.fmoe_layer_forward_host(m.ctx, 0, xh.data_ptr(), T, xh.data_ptr(), None, None, m.stream)
         torch.cuda.synchronize()
