@@ -49,12 +49,17 @@ FALLBACK_HBM_GBS = 6650.0
 BATCHED_LAUNCHES = 10
 
 
-def kernel_source_sha() -> str:
+# the sources each timed kernel is compiled from: a DRAM capture stays valid
+# (roofline.traffic) until one of them changes
+KERNEL_SOURCES = {"layer": ["fmoe_decode.cu", "fmoe_internal.h"],
+                  "batched": ["fmoe_grouped_tc.cu", "fmoe_batched.cu", "fmoe_internal.h"]}
+
+
+def kernel_source_sha(key: str) -> str:
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".h")):
-            h.update(name.encode())
-            h.update(open(os.path.join(CSRC, name), "rb").read())
+    for name in sorted(KERNEL_SOURCES[key]):
+        h.update(name.encode())
+        h.update(open(os.path.join(CSRC, name), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -558,7 +563,8 @@ def measure_gpu(args, wl, ws, rank, local, steps, warmup, e2e_steps, cpu_baselin
     try:
         tr = json.load(open(TRAFFIC_PATH))
         key = f"{wl.name}"
-        if tr.get("source_sha") == kernel_source_sha() and key in tr.get("bytes_per_launch", {}):
+        if key in KERNEL_SOURCES and tr.get("source_sha", {}).get(key) == kernel_source_sha(key) \
+                and key in tr.get("bytes_per_launch", {}):
             traffic = tr["bytes_per_launch"][key]
     except Exception:
         traffic = None
