@@ -45,8 +45,9 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 # kernels one batched layer step launches: norm, router, logit sum, top-K,
-# permute, input prep, gate/up GEMM, activation prep, down GEMM, combine
-BATCHED_LAUNCHES = 10
+# permute, input prep, GEMV fragments, gate/up GEMM (tcgen05), gate/up GEMV,
+# activation prep, GEMV fragments, down GEMM (tcgen05), down GEMV, combine
+BATCHED_LAUNCHES = 14
 
 
 # the sources each timed kernel is compiled from: a DRAM capture stays valid
@@ -551,10 +552,12 @@ def measure_gpu(args, wl, ws, rank, local, steps, warmup, e2e_steps, cpu_baselin
         gu_flops = 2 * P * 2 * wl.inter * wl.hidden
         tensor = {"flops_per_step": flops, "achieved_tflops": flops / (ms_per_step * 1e-3) / 1e12,
                   "unique_experts_per_step": statistics.mean(uniq),
-                  "gate_up_gemm": {"kernel": f"bt_tc_gemm_kernel<{wl.bits}, true>", "us": 1e3 * gemm_ms[0],
+                  "gate_up_gemm": {"kernel": f"gate/up phase: bt_gv_frag_kernel, bt_tc_gemm_kernel<{wl.bits}, true>, "
+                                             f"bt_gemv_kernel<{wl.bits}, true>", "us": 1e3 * gemm_ms[0],
                                    "algorithmic_bytes": gu_bytes, "gbs": gu_bytes / (gemm_ms[0] * 1e-3) / 1e9,
                                    "tflops": gu_flops / (gemm_ms[0] * 1e-3) / 1e12},
-                  "down_gemm": {"kernel": f"bt_tc_gemm_kernel<{wl.bits}, false>", "us": 1e3 * gemm_ms[1],
+                  "down_gemm": {"kernel": f"down phase: bt_gv_frag_kernel, bt_tc_gemm_kernel<{wl.bits}, false>, "
+                                          f"bt_gemv_kernel<{wl.bits}, false>", "us": 1e3 * gemm_ms[1],
                                 "algorithmic_bytes": dn_bytes, "gbs": dn_bytes / (gemm_ms[1] * 1e-3) / 1e9,
                                 "tflops": gu_flops / 2 / (gemm_ms[1] * 1e-3) / 1e12}}
     achieved = bytes_launch / (us_layer * 1e-6) / 1e9

@@ -20,6 +20,7 @@
 //   down     grouped tcgen05 GEMM, 128 output rows x up to 64 positions
 //   combine  out = h + y_shared + sum_k w_k y_k, fp32, one bf16 rounding
 #include <cuda_bf16.h>
+#include <algorithm>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -256,6 +257,8 @@ struct PermuteArgs {
   uint32_t* items_dn;
   int32_t* n_items;
   int max_items_gu, max_items_dn;
+  int32_t* small_seg;    // [E+1]
+  int bands_gu, bands_dn;  // 16-row bands of gate/up (2I/16) and down (H/16)
 };
 
 // Block-wide exclusive scan of three counters per thread (blockDim 1024);
@@ -329,19 +332,23 @@ __global__ void __launch_bounds__(1024) bt_permute_kernel(PermuteArgs p) {
   int32_t* seg_item = p.seg + 3 * S;  // first gate/up item of each segment
   const int rbg = (p.rows_gu + kGemmRows - 1) / kGemmRows, rbd = (p.rows_dn + kGemmRows - 1) / kGemmRows;
   if (p.single_expert >= 0) {
+    const bool small = p.T <= kGemvTokens;
     if (tid == 0) {
       seg_e[0] = p.single_expert;
       seg_start[0] = 0;
       seg_cnt[0] = p.T;
       p.seg[4 * S] = 1;
+      p.small_seg[0] = 0;
     }
     for (int t = tid; t < p.T; t += blockDim.x) p.pos_tok[t] = t;
-    const int ntb = (p.T + kGemmTokens - 1) / kGemmTokens;
+    const int ntb = small ? 0 : (p.T + kGemmTokens - 1) / kGemmTokens;
     for (int i = tid; i < rbg * ntb; i += blockDim.x) p.items_gu[i] = ((uint32_t)(i / ntb) << 8) | (i % ntb);
     for (int i = tid; i < rbd * ntb; i += blockDim.x) p.items_dn[i] = ((uint32_t)(i / ntb) << 8) | (i % ntb);
     if (tid == 0) {
       p.n_items[0] = rbg * ntb;
       p.n_items[1] = rbd * ntb;
+      p.n_items[2] = small ? p.bands_gu : 0;
+      p.n_items[3] = small ? p.bands_dn : 0;
     }
     return;
   }
@@ -358,23 +365,30 @@ __global__ void __launch_bounds__(1024) bt_permute_kernel(PermuteArgs p) {
   if (tid == 0) cnt[p.E] = p.T;
   __syncthreads();
   // per candidate: positions, a segment if non-empty, its token blocks
+  // segments of up to kGemvTokens positions go to the GEMV (no token blocks);
+  // the second counter packs segments (low 16 bits) and small ones (high)
   const int c = tid < S ? cnt[tid] : 0;
-  const int ntb = (c + kGemmTokens - 1) / kGemmTokens;
-  const int3 pre = block_scan3(make_int3(c, c > 0 ? 1 : 0, ntb), scratch, tot);
-  const int n_seg = tot[1], n_tb = tot[2];
+  const bool small = c > 0 && c <= kGemvTokens;
+  const int ntb = small ? 0 : (c + kGemmTokens - 1) / kGemmTokens;
+  const int3 pre = block_scan3(make_int3(c, (c > 0 ? 1 : 0) | (small ? 1 << 16 : 0), ntb), scratch, tot);
+  const int n_seg = tot[1] & 0xFFFF, n_small = tot[1] >> 16, n_tb = tot[2];
+  const int sidx = pre.y & 0xFFFF;
   if (tid < S) {
     cur[tid] = pre.x;
     if (c > 0) {
-      seg_e[pre.y] = tid;
-      seg_start[pre.y] = pre.x;
-      seg_cnt[pre.y] = c;
-      seg_item[pre.y] = rbg * pre.z;
+      seg_e[sidx] = tid;
+      seg_start[sidx] = pre.x;
+      seg_cnt[sidx] = c;
+      seg_item[sidx] = rbg * pre.z;
+      if (small) p.small_seg[pre.y >> 16] = sidx;
     }
   }
   if (tid == 0) {
     p.seg[4 * S] = n_seg;
     p.n_items[0] = min(rbg * n_tb, p.max_items_gu);
     p.n_items[1] = min(rbd * n_tb, p.max_items_dn);
+    p.n_items[2] = n_small * p.bands_gu;
+    p.n_items[3] = n_small * p.bands_dn;
   }
   __syncthreads();
   for (int base = tid - lane; base < n; base += blockDim.x) {
@@ -400,7 +414,7 @@ __global__ void __launch_bounds__(1024) bt_permute_kernel(PermuteArgs p) {
   // token block (token blocks of one row block run side by side and share the
   // weight tiles in L2)
   if (tid < S && c > 0) {
-    const int s = pre.y, ig0 = rbg * pre.z, id0 = rbd * pre.z;
+    const int s = sidx, ig0 = rbg * pre.z, id0 = rbd * pre.z;
     for (int rb = 0; rb < rbg; ++rb)
       for (int tb = 0; tb < ntb; ++tb) {
         const int i = ig0 + rb * ntb + tb;
@@ -411,6 +425,172 @@ __global__ void __launch_bounds__(1024) bt_permute_kernel(PermuteArgs p) {
         const int i = id0 + rb * ntb + tb;
         if (i < p.max_items_dn) p.items_dn[i] = ((uint32_t)s << 16) | ((uint32_t)rb << 8) | (uint32_t)tb;
       }
+  }
+}
+
+// ------------------------------------------------------------------ small segments: GEMV
+// Segments of at most kGemvTokens positions (most experts of a 256-token step)
+// are contracted by one warp per 16-row band with mma.sync m16n8k16: the
+// packed tile is the A fragment layout, so the exact codes come out of one
+// lop3 + sub per pair, and the 8 columns of B are the segment's positions.
+// Per 64-column group each position's input is scaled to fp16 by its own
+// power of two (exact for bf16), and the group's result is s*2^-sh*sum(q*x')
+// + b*sum(x) in fp32, as in the batch-1 kernel: scale and bias never pass
+// through fp16.
+
+__device__ __forceinline__ uint32_t gv_lop(uint32_t a, uint32_t mask, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t gv_code2(uint32_t w, uint32_t mask) {  // codes * 4^k, exact fp16 pair
+  constexpr uint32_t kMagic = 0x64006400u;  // (1024, 1024)
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(gv_lop(w, mask, kMagic)), "r"(kMagic));
+  return d;
+}
+__device__ __forceinline__ void gv_mma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                       uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ float gv_exp2i(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
+
+struct GemvArgs {
+  const int32_t* seg;        // segment table ([4][S] + n_seg)
+  int S;
+  const int32_t* small_seg;  // small segment -> segment index
+  const int32_t* n_items;    // device count of (small segment, band) items
+  const int32_t* pos_tok;    // position -> token (gate/up input rows)
+  const void* src;           // gate/up: z bf16 [T][H] by token; down: a fp32 [P][I] by position
+  int K;                     // contraction length (H or I)
+  int bits;
+  uint32_t* frag;            // [max_small][K/64][8][32]
+  float2* info;              // [max_small][K/64][8]
+  const uint8_t* experts;    // packed blobs of the layer
+  int64_t blob;
+  int64_t mat_off;           // byte offset of the matrix in a blob (0: gate/up, else down)
+  int bands;                 // 16-row bands of the matrix
+  float* out;                // gate/up: a [P][I]; down: y [P][H]
+  int ldo;
+};
+
+// B fragments of every small segment: one warp per (segment, group), the
+// group's 64 values of each of the segment's (up to 8) positions; lane l holds
+// values 2l, 2l+1.  Fragment word (position p, lane column t, slice s, half
+// `which`) sits at ((item * 8 + p) * 32) + (t * 4 + s) * 2 + which, laid out
+// as the batch-1 kernel's fragments; positions past the segment are zero.
+template <typename Src>
+__global__ void bt_gv_frag_kernel(GemvArgs g, int n_small_cap) {
+  const int lane = threadIdx.x & 31, G = g.K / kGroup;
+  const int n_small = *g.n_items / g.bands;  // the GEMV item count is small segments x bands
+  const int q = 2 * lane, sl = q / 16, qq = q % 16, which = qq / 8, t = (qq % 8) / 2;
+  const int fs = (g.bits == 4) ? (which ? 4 : 0) : ((sl & 1) ? 4 : 0) + (which ? 2 : 0);
+  const int total = min(n_small, n_small_cap) * G;
+  for (int it = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); it < total; it += gridDim.x * (blockDim.x / 32)) {
+    const int sr = it / G, gr = it % G;
+    const int sg = g.small_seg[sr];
+    const int pos0 = g.seg[g.S + sg], n = g.seg[2 * g.S + sg];
+#pragma unroll 1
+    for (int pj = 0; pj < kGemvTokens; ++pj) {
+      float lo = 0.f, hi = 0.f;
+      if (pj < n) {
+        const int c0 = gr * kGroup + 2 * lane;
+        if constexpr (sizeof(Src) == 2) {
+          const uint32_t v = *reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(g.src) +
+                                                                (size_t)g.pos_tok[pos0 + pj] * g.K + c0);
+          lo = bflo(v);
+          hi = bfhi(v);
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(static_cast<const float*>(g.src) + (size_t)(pos0 + pj) * g.K + c0);
+          lo = v.x;
+          hi = v.y;
+        }
+      }
+      const uint32_t m = __reduce_max_sync(0xffffffffu, max(__float_as_uint(fabsf(lo)), __float_as_uint(fabsf(hi))));
+      float sum = lo + hi;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      const int e = (int)((m >> 23) & 0xFF) - 127;
+      const int sh = m == 0 ? 0 : min(14 - max(e, -126), 126);
+      const __half2 h2 = __floats2half2_rn(lo * gv_exp2i(sh - fs), hi * gv_exp2i(sh - fs));
+      const size_t base = ((size_t)it * kGemvTokens + pj) * 32;
+      g.frag[base + (t * 4 + sl) * 2 + which] = *reinterpret_cast<const uint32_t*>(&h2);
+      if (lane == 0) g.info[(size_t)it * kGemvTokens + pj] = make_float2(gv_exp2i(-sh), sum);
+    }
+  }
+}
+
+// One warp per (small segment, 16-row band): all K/64 tiles of the band.
+// Lane 4r+t accumulates rows r and r+8 of the band for positions 2t and 2t+1.
+template <int BITS, bool GATE_UP>
+__global__ void __launch_bounds__(256) bt_gemv_kernel(GemvArgs g) {
+  constexpr int TB = 16 * kGroup * BITS / 8 + 64, CB = 16 * kGroup * BITS / 8;
+  const int lane = threadIdx.x & 31, r = lane >> 2, t = lane & 3;
+  const int G = g.K / kGroup, n_items = *g.n_items;
+  for (int it = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); it < n_items; it += gridDim.x * (blockDim.x / 32)) {
+    const int sr = it / g.bands, band = it % g.bands;
+    const int sg = g.small_seg[sr];
+    const int e = g.seg[sg], pos0 = g.seg[g.S + sg], n = g.seg[2 * g.S + sg];
+    const uint8_t* tiles = g.experts + (int64_t)e * g.blob + g.mat_off + (int64_t)band * G * TB;
+    const uint32_t* fr = g.frag + ((size_t)sr * G * kGemvTokens + r) * 32 + t * 8;
+    const float2* inf = g.info + (size_t)sr * G * kGemvTokens + 2 * t;
+    float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;  // (row r | r+8) x (position 2t | 2t+1)
+#pragma unroll 4
+    for (int gr = 0; gr < G; ++gr) {
+      const uint8_t* tile = tiles + (int64_t)gr * TB;
+      const uint4 f0 = *reinterpret_cast<const uint4*>(fr + (size_t)gr * kGemvTokens * 32);
+      const uint4 f1 = *reinterpret_cast<const uint4*>(fr + (size_t)gr * kGemvTokens * 32 + 4);
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (BITS == 4) {
+        const uint4 qv = *reinterpret_cast<const uint4*>(tile + lane * 16);
+        const uint32_t w4[4] = {qv.x, qv.y, qv.z, qv.w};
+        const uint32_t bb[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl) {
+          const uint32_t w = w4[sl], w8 = w >> 8;
+          gv_mma(c, gv_code2(w, 0x000F000Fu), gv_code2(w8, 0x000F000Fu), gv_code2(w, 0x00F000F0u),
+                 gv_code2(w8, 0x00F000F0u), bb[2 * sl], bb[2 * sl + 1]);
+        }
+      } else {
+        const uint2 qv = *reinterpret_cast<const uint2*>(tile + lane * 8);
+        const uint32_t w2[2] = {qv.x, qv.y};
+        const uint32_t bb[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+#pragma unroll
+        for (int wj = 0; wj < 2; ++wj) {
+          const uint32_t w = w2[wj], w8 = w >> 8;
+          gv_mma(c, gv_code2(w, 0x00030003u), gv_code2(w8, 0x00030003u), gv_code2(w, 0x000C000Cu),
+                 gv_code2(w8, 0x000C000Cu), bb[4 * wj], bb[4 * wj + 1]);
+          gv_mma(c, gv_code2(w, 0x00300030u), gv_code2(w8, 0x00300030u), gv_code2(w, 0x00C000C0u),
+                 gv_code2(w8, 0x00C000C0u), bb[4 * wj + 2], bb[4 * wj + 3]);
+        }
+      }
+      const uint2 sb = *reinterpret_cast<const uint2*>(tile + CB + r * 8);
+      const float4 iv = *reinterpret_cast<const float4*>(inf + (size_t)gr * kGemvTokens);  // positions 2t, 2t+1
+      const float s0 = bflo(sb.x), b0 = bfhi(sb.x), s8 = bflo(sb.y), b8 = bfhi(sb.y);
+      a00 = fmaf(s0 * iv.x, c[0], fmaf(b0, iv.y, a00));
+      a01 = fmaf(s0 * iv.z, c[1], fmaf(b0, iv.w, a01));
+      a10 = fmaf(s8 * iv.x, c[2], fmaf(b8, iv.y, a10));
+      a11 = fmaf(s8 * iv.z, c[3], fmaf(b8, iv.w, a11));
+    }
+    const int p0 = 2 * t, p1 = 2 * t + 1;
+    if constexpr (GATE_UP) {
+      // band rows r (gate) and r + 8 (up) are the same activation j
+      const int j = band * 8 + r;
+      if (p0 < n) g.out[(size_t)(pos0 + p0) * g.ldo + j] = a00 / (1.0f + expf(-a00)) * a10;
+      if (p1 < n) g.out[(size_t)(pos0 + p1) * g.ldo + j] = a01 / (1.0f + expf(-a01)) * a11;
+    } else {
+      const int row = band * 16 + r;
+      if (p0 < n) {
+        g.out[(size_t)(pos0 + p0) * g.ldo + row] = a00;
+        g.out[(size_t)(pos0 + p0) * g.ldo + row + 8] = a10;
+      }
+      if (p1 < n) {
+        g.out[(size_t)(pos0 + p1) * g.ldo + row] = a01;
+        g.out[(size_t)(pos0 + p1) * g.ldo + row + 8] = a11;
+      }
+    }
   }
 }
 
@@ -438,6 +618,18 @@ __global__ void bt_combine_kernel(const uint16_t* __restrict__ h, const float* _
     *reinterpret_cast<uint2*>(out + 4 * i) = make_uint2((uint32_t)to_bf16(a0) | ((uint32_t)to_bf16(a1) << 16),
                                                         (uint32_t)to_bf16(a2) | ((uint32_t)to_bf16(a3) << 16));
   }
+}
+
+int launch_gemv(int bits, bool gate_up, const GemvArgs& v, int n_sm, cudaStream_t st) {
+  const dim3 grid(4 * n_sm), block(256);
+  if (bits == 4) {
+    if (gate_up) bt_gemv_kernel<4, true><<<grid, block, 0, st>>>(v);
+    else bt_gemv_kernel<4, false><<<grid, block, 0, st>>>(v);
+  } else {
+    if (gate_up) bt_gemv_kernel<2, true><<<grid, block, 0, st>>>(v);
+    else bt_gemv_kernel<2, false><<<grid, block, 0, st>>>(v);
+  }
+  return (int)cudaGetLastError();
 }
 
 int grid_of(int64_t work, int per_block, int cap) {
@@ -477,7 +669,12 @@ size_t carve(uintptr_t base, int H, int E, int K, int I, int T, BatchWs& ws) {
   ws.pos_of = reinterpret_cast<int32_t*>(take(P * 4));
   ws.items_gu = reinterpret_cast<uint32_t*>(take((size_t)ws.max_items_gu * 4));
   ws.items_dn = reinterpret_cast<uint32_t*>(take((size_t)ws.max_items_dn * 4));
-  ws.n_items = reinterpret_cast<int32_t*>(take(2 * 4));
+  ws.n_items = reinterpret_cast<int32_t*>(take(4 * 4));
+  ws.max_small = (int)std::min<size_t>((size_t)E + 1, P);
+  ws.small_seg = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
+  const size_t gmax = (size_t)std::max(H, I) / kGroup;
+  ws.gv_frag = reinterpret_cast<uint32_t*>(take((size_t)ws.max_small * gmax * kGemvTokens * 32 * 4));
+  ws.gv_info = reinterpret_cast<float2*>(take((size_t)ws.max_small * gmax * kGemvTokens * 8));
   ws.a = reinterpret_cast<float*>(take(P * I * 4));
   ws.ap = reinterpret_cast<uint16_t*>(take(P * I * 2));
   ws.asc = reinterpret_cast<float*>(take(P * 4));
@@ -537,6 +734,9 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   pa.n_items = ws.n_items;
   pa.max_items_gu = ws.max_items_gu;
   pa.max_items_dn = ws.max_items_dn;
+  pa.small_seg = ws.small_seg;
+  pa.bands_gu = 2 * a.I / 16;
+  pa.bands_dn = a.H / 16;
   bt_permute_kernel<<<1, 1024, (size_t)(2 * (a.E + 1) + 96 + 3) * 4, st>>>(pa);
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
@@ -558,8 +758,29 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   auto mark = [&](int k) {
     if (a.gemm_events[k]) cudaEventRecord(static_cast<cudaEvent_t>(a.gemm_events[k]), st);
   };
+  // small segments: B fragments of their positions, then the GEMV
+  GemvArgs v{};
+  v.seg = ws.seg;
+  v.S = a.E + 1;
+  v.small_seg = ws.small_seg;
+  v.pos_tok = ws.pos_tok;
+  v.bits = a.bits;
+  v.frag = ws.gv_frag;
+  v.info = ws.gv_info;
+  v.experts = a.experts;
+  v.blob = a.blob_bytes;
   mark(0);
+  v.n_items = ws.n_items + 2;
+  v.src = ws.z;
+  v.K = a.H;
+  v.mat_off = 0;
+  v.bands = 2 * a.I / 16;
+  v.out = ws.a;
+  v.ldo = a.I;
+  bt_gv_frag_kernel<uint16_t><<<2 * n_sm, 256, 0, st>>>(v, ws.max_small);
   int rc = launch_tc_gemm(a.bits, true, *a.wmap_gu, ws.zmap, ws.zsmap, g, n_sm, stream);
+  if (rc != 0) return rc;
+  rc = launch_gemv(a.bits, true, v, n_sm, st);
   if (rc != 0) return rc;
   mark(1);
   // down: B = the position's activation
@@ -573,7 +794,17 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   g.bscale = ws.asc;
   g.out = layer ? ws.y : a.y_out;
   mark(2);
+  v.n_items = ws.n_items + 3;
+  v.src = ws.a;
+  v.K = a.I;
+  v.mat_off = packed_gu_bytes(a.H, a.I, a.bits);
+  v.bands = a.H / 16;
+  v.out = g.out;
+  v.ldo = a.H;
+  bt_gv_frag_kernel<float><<<2 * n_sm, 256, 0, st>>>(v, ws.max_small);
   rc = launch_tc_gemm(a.bits, false, *a.wmap_dn, ws.amap, ws.asmap, g, n_sm, stream);
+  if (rc != 0) return rc;
+  rc = launch_gemv(a.bits, false, v, n_sm, st);
   if (rc != 0) return rc;
   mark(3);
   if (layer) {

@@ -276,6 +276,7 @@ inline __host__ __device__ void task_stage_of(int nstage, int n_issuers, int n_t
 constexpr int kGemmRows = 128;       // rows per work item (8 packed bands of 16)
 constexpr int kGemmTokens = 64;      // tokens (positions) per work item
 constexpr int kGroupedMinTokens = 8; // fmoe_layer_forward uses the batched path from this T on
+constexpr int kGemvTokens = 8;       // segments up to this many positions take the mma.sync GEMV, not tcgen05
 constexpr int kBatchMaxExperts = 1023;  // batched permute: one thread per expert plus the shared one
 constexpr int kBatchMaxTokens = 255 * kGemmTokens;  // token blocks per segment fit 8 bits of a work item
 
@@ -299,7 +300,11 @@ struct BatchWs {              // device buffers, sized for max_tokens at create
   int32_t* pos_of;            // [T][K+1] position of (token, slot); slot K = shared
   uint32_t* items_gu;         // work items (seg, row block, token block)
   uint32_t* items_dn;
-  int32_t* n_items;           // [2]
+  int32_t* n_items;           // [4]: tcgen05 gate/up, down items; GEMV gate/up, down items
+  int32_t* small_seg;         // [E+1]: segments of <= kGemvTokens positions, in segment order
+  uint32_t* gv_frag;          // [small][H/64][8 positions][32] fp16 pairs: mma.sync B fragments (GEMV)
+  float2* gv_info;            // [small][H/64][8]: (2^-shift, group sum) per position and group
+  int max_small;              // segments the GEMV buffers hold
   float* a;                   // [T*(K+1)][I] activations
   uint16_t* ap;               // fp16 [T*(K+1)][I] down-GEMM input (scaled, k-permuted)
   float* asc;                 // [T*(K+1)]
