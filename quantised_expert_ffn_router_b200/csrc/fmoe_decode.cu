@@ -797,6 +797,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     for (int cur = 0; cur < NL; ++cur) {
       const uint32_t tag = tag0 + (uint32_t)cur;
       const LayerDev Ld = layer_of<MULTI>(P, cur);
+      // warps whose first task is a router row (the first tasks of the list)
+      const int n_early = (P.mode != kModeExpert && P.n_slots > 0 && my_rrows * P.router_parts <= kConsumerWarps / 2)
+                              ? my_rrows * P.router_parts
+                              : 0;
+      const bool early_router = warp < n_early;
       // thread tid holds columns 8*(tid + j*threads) .. +7, j < kPrepChunks
       constexpr int kCT = kConsumerWarps * 32;
       constexpr int kPrepChunks = (kMaxHidden + 8 * kCT - 1) / (8 * kCT);
@@ -906,10 +911,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           if (c0 < P.H) *reinterpret_cast<uint4*>(zs + c0) = hv[j];
         }
         asm volatile("bar.sync 1, %0;" ::"r"(kCT) : "memory");
-        if (P.n_slots > 0) {
-          // warp w builds groups 4w..4w+3, then 4(w+W).., so a batch is contiguous
-          const int ngz = P.H / kGroup;
-          for (int G0 = 4 * warp; G0 < ngz; G0 += 4 * kConsumerWarps) {
+        // The warps whose first task is a router row start it now (the rows
+        // need z only); the others build the fp16 fragments, which the gate/up
+        // chunks need, and every warp meets at barrier 2 before its first
+        // chunk.
+        if (P.n_slots > 0 && !early_router) {
+          // builder b builds groups 4b..4b+3, then 4(b+B).., so a batch is contiguous
+          const int ngz = P.H / kGroup, nb = kConsumerWarps - n_early, b = warp - n_early;
+          for (int G0 = 4 * b; G0 < ngz; G0 += 4 * nb) {
             float lo[4], hi[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -920,8 +929,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             frag_batch<4>(lo, hi, G0, ngz, BITS, zfrag, zinfo, lane);
           }
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
+        if (!early_router) asm volatile("bar.sync 2, %0;" ::"r"(kCT) : "memory");
       }
+      bool frags_seen = !early_router;
 
       if (tid == 0) FMOE_TRACE_SET(cur, 2);
       // The producer selects the routed experts once per launch, late; running
@@ -933,6 +943,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
       // ---- task loop: warp w takes tasks w, w+16, ...
       for (int i = warp; i < n_tasks; i += kConsumerWarps) {
+        if (!frags_seen && i != warp) {  // an early router warp's first chunk: fragments first
+          asm volatile("bar.sync 2, %0;" ::"r"(kCT) : "memory");
+          frags_seen = true;
+        }
         int s, fill;
         task_stage_of(P.nstage, P.n_issuers, n_tasks, n_down, i, s, fill, cur);
         // A stage's fills are consumed by different warps, so first make sure
@@ -1169,6 +1183,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           if (ty == kTaskDown) FMOE_TRACE_LAST(cur, 11);
         }
       }
+      if (!frags_seen) asm volatile("bar.sync 2, %0;" ::"r"(kCT) : "memory");  // an early router warp without chunks
       if (MULTI) {
         // all consumer warps are done with this layer's tasks
         if (consumers_any(*abort_flag != 0)) break;
