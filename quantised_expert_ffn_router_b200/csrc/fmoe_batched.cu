@@ -174,7 +174,7 @@ __global__ void bt_prep_kernel(const Src* __restrict__ src, const int32_t* __res
 // both operands are staged in shared memory by cp.async (3 stages, rows padded
 // to 36 words so fragment reads are conflict-free); warp (we, wt) owns experts
 // 16*we.. and tokens 32*wt.. (4 blocks of 8).
-constexpr int kRtRows = 64, kRtStages = 4, kRtRowWords = 36, kRtSplit = 4;
+constexpr int kRtRows = 64, kRtStages = 4, kRtRowWords = 36, kRtSplit = 8;
 constexpr int kRtStage = 2 * kRtRows * kRtRowWords * 4;
 __global__ void __launch_bounds__(256) bt_router_kernel(const uint16_t* __restrict__ wr, const uint16_t* __restrict__ z,
                                                         int T, int E, int H, float* __restrict__ part) {
