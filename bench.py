@@ -489,16 +489,18 @@ def measure_gpu(args, wl, ws, rank, local, steps, warmup, e2e_steps, cpu_baselin
     # input copy, the layer (or stack) and the output copy on the stream
     x_host = X[:min(n_batches, e2e_steps)].cpu().pin_memory()
     out_host = torch.empty_like(x_host).pin_memory()
-    e2e_ms = []
+    e2e_ms, call_us = [], []
     for i in range(e2e_steps):
         maybe_flush(i)
         j = i % len(x_host)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
+        c0 = time.perf_counter()
         if stacked:
             fm.fmoe_stack_forward_host(ctx, 0, L, x_host[j].data_ptr(), B, out_host[j].data_ptr(), sp)
         else:
             fm.fmoe_layer_forward_host(ctx, 0, x_host[j].data_ptr(), B, out_host[j].data_ptr(), None, None, sp)
+        call_us.append(1e6 * (time.perf_counter() - c0))
         b.record(stream)
         stream.synchronize()
         e2e_ms.append(a.elapsed_time(b))
@@ -597,6 +599,7 @@ def measure_gpu(args, wl, ws, rank, local, steps, warmup, e2e_steps, cpu_baselin
                 "path": ("page-locked buffers: input read over the link by a stage-in kernel, output written "
                          "to host memory by the fused kernel" if not batched else
                          "one copy-engine transfer each way around the grouped path"),
+                "host_call_us": statistics.median(call_us),
                 "breakdown_copy_engine_us": {"h2d": e2e_parts_us[0], "device": e2e_parts_us[1],
                                              "d2h": e2e_parts_us[2]}},
         "gpu_launches": steps * (BATCHED_LAUNCHES if batched else (L if per_layer or not stacked else 1)),

@@ -900,16 +900,16 @@ static fmoe_status copy_async(fmoe_ctx* ctx, void* dst, const void* src, size_t 
 }
 
 namespace {
-using PointerAttrFn = CUresult (*)(void*, CUpointer_attribute, CUdeviceptr);
-PointerAttrFn pointer_attr_fn() {
-  static PointerAttrFn fn = nullptr;
+using PointerAttrsFn = CUresult (*)(unsigned int, CUpointer_attribute*, void**, CUdeviceptr);
+PointerAttrsFn pointer_attrs_fn() {
+  static PointerAttrsFn fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuPointerGetAttribute", &f, cudaEnableDefault, &q) == cudaSuccess &&
+    if (cudaGetDriverEntryPoint("cuPointerGetAttributes", &f, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PointerAttrFn>(f);
+      fn = reinterpret_cast<PointerAttrsFn>(f);
     cudaGetLastError();
   });
   return fn;
@@ -918,25 +918,23 @@ PointerAttrFn pointer_attr_fn() {
 // Device address of `bytes` of page-locked, device-mapped host memory at p, or
 // null: for pageable memory, a failed query, or a buffer that does not lie
 // inside one page-locked allocation (a kernel reading or writing past its end
-// would fault; the copy path reports the error on the host instead).
+// would fault; the copy path reports the error on the host instead).  One
+// driver query per buffer.
 void* mapped_host(const void* p, size_t bytes) {
   if (p == nullptr) return nullptr;
-  cudaPointerAttributes at{};
-  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
-    cudaGetLastError();
-    return nullptr;
-  }
-  if (at.type != cudaMemoryTypeHost || at.devicePointer == nullptr) return nullptr;
-  PointerAttrFn fn = pointer_attr_fn();
+  PointerAttrsFn fn = pointer_attrs_fn();
   if (fn == nullptr) return nullptr;
-  CUdeviceptr start = 0;
+  unsigned int type = 0;
+  CUdeviceptr dev = 0, start = 0;
   size_t size = 0;
+  CUpointer_attribute at[4] = {CU_POINTER_ATTRIBUTE_MEMORY_TYPE, CU_POINTER_ATTRIBUTE_DEVICE_POINTER,
+                               CU_POINTER_ATTRIBUTE_RANGE_START_ADDR, CU_POINTER_ATTRIBUTE_RANGE_SIZE};
+  void* data[4] = {&type, &dev, &start, &size};
   const CUdeviceptr addr = (CUdeviceptr)(uintptr_t)p;
-  if (fn(&start, CU_POINTER_ATTRIBUTE_RANGE_START_ADDR, addr) != CUDA_SUCCESS ||
-      fn(&size, CU_POINTER_ATTRIBUTE_RANGE_SIZE, addr) != CUDA_SUCCESS)
-    return nullptr;
+  if (fn(4, at, data, addr) != CUDA_SUCCESS) return nullptr;  // pageable memory: zeros and CUDA_SUCCESS
+  if (type != CU_MEMORYTYPE_HOST || dev == 0 || size == 0) return nullptr;
   if (addr < start || bytes > size || addr - start > size - bytes) return nullptr;
-  return at.devicePointer;
+  return reinterpret_cast<void*>((uintptr_t)dev);
 }
 
 // Reads `bytes` (a multiple of 16) from mapped host memory into device memory:
