@@ -99,9 +99,10 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
   P.tb = tile_bytes(c.bits);
   P.cb = tile_code_bytes(c.bits);
   P.gu_tiles = c.hidden / kGroup;
-  P.gu_chunks = (P.gu_tiles + kChunkTiles - 1) / kChunkTiles;
+  const int ct = chunk_tiles(c.bits);
+  P.gu_chunks = (P.gu_tiles + ct - 1) / ct;
   P.dn_tiles = c.inter / kGroup;
-  P.dn_chunks = (P.dn_tiles + kChunkTiles - 1) / kChunkTiles;
+  P.dn_chunks = (P.dn_tiles + ct - 1) / ct;
   P.units_per_slot = c.inter / 8;
   P.total_units = P.n_slots * P.units_per_slot;
   P.units_per_cta = (P.total_units + grid - 1) / grid;
@@ -112,8 +113,8 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
   // A router row is one task when it fits an expert stage (one copy, one warp);
   // otherwise it is split into up to 4 non-empty parts of whole 64-column groups.
   const int rgroups = c.hidden / kGroup;
-  const uint32_t expert_stage = (uint32_t)std::max(std::min(kChunkTiles, c.hidden / kGroup),
-                                                   std::min(kChunkTiles, c.inter / kGroup)) * tile_bytes(c.bits);
+  const uint32_t expert_stage = (uint32_t)std::max(std::min(ct, c.hidden / kGroup),
+                                                   std::min(ct, c.inter / kGroup)) * tile_bytes(c.bits);
   const int per_part = ((uint32_t)c.hidden * 2 <= expert_stage) ? rgroups : (rgroups + 3) / 4;
   P.router_part_cols = per_part * kGroup;
   P.router_parts = (rgroups + per_part - 1) / per_part;
@@ -124,8 +125,8 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
 
   uint32_t stage = 0;
   if (P.total_units > 0) {
-    stage = std::max<uint32_t>(stage, (uint32_t)(std::min(kChunkTiles, P.gu_tiles) * P.tb));
-    stage = std::max<uint32_t>(stage, (uint32_t)(std::min(kChunkTiles, P.dn_tiles) * P.tb));
+    stage = std::max<uint32_t>(stage, (uint32_t)(std::min(ct, P.gu_tiles) * P.tb));
+    stage = std::max<uint32_t>(stage, (uint32_t)(std::min(ct, P.dn_tiles) * P.tb));
   }
   if (router) stage = std::max<uint32_t>(stage, (uint32_t)P.router_part_cols * 2);
   P.stage_bytes = align_up(stage, 128);
@@ -152,10 +153,10 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
   const uint32_t r_tasks = region((uint32_t)kMaxTasks * 4);
   const uint32_t r_misc = region((uint32_t)sizeof(Misc));
   // Down jobs get a stage each after the ring when that leaves the ring at
-  // least kMinRingStages stages (else they share the ring, streamed last).  A
+  // least min_ring_stages(bits) stages (else they share the ring, streamed last).  A
   // ring stage turns over in about one loaded HBM round trip plus one task's
-  // processing (~1.5 + ~1.7 us), so keeping HBM busy takes ~20 stages of
-  // 9 KB per SM; a shallower ring loses more than early down weights gain.
+  // processing (~1.5 + ~1.7 us), so keeping HBM busy takes ~180 KB of stages
+  // per SM at 4-bit; a shallower ring loses more than early down weights gain.
   // The ring takes as many stages as still fit (<= 64 in all, <= its tasks).
   auto fit_ring = [&](int n_down) {
     const int ring_tasks = std::max(max_tasks - n_down, 1);
@@ -168,7 +169,7 @@ bool make_plan(const fmoe_config& c, int grid, int mode, int max_smem, DecodePla
   };
   P.n_down_max = P.n_slots > 0 ? P.rb_per_cta * P.n_slots * P.dn_chunks : 0;
   int nstage = P.n_down_max > 0 && P.n_down_max <= 32 ? fit_ring(P.n_down_max) : 0;
-  if (nstage < std::min(kMinRingStages, std::max(max_tasks - P.n_down_max, 1))) {
+  if (nstage < std::min(min_ring_stages(c.bits), std::max(max_tasks - P.n_down_max, 1))) {
     P.n_down_max = 0;
     nstage = fit_ring(0);
   }

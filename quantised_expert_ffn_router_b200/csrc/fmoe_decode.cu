@@ -712,13 +712,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             P.cache.on ? misc->slot_src[slot] : Ld.experts + (int64_t)misc->slot_e[slot] * P.blob_bytes;
         if (ty == kTaskGateUp) {
           const int u = cta + (int)idx * G, rb = u % P.units_per_slot;
-          const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
-          src = blob + ((int64_t)rb * P.gu_tiles + c * kChunkTiles) * TB;
+          const int n = min(chunk_tiles(BITS), P.gu_tiles - (int)c * chunk_tiles(BITS));
+          src = blob + ((int64_t)rb * P.gu_tiles + c * chunk_tiles(BITS)) * TB;
           bytes = (uint32_t)(n * TB);
         } else {
           const int rbg = first_rb + (int)idx * G;
-          const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
-          src = blob + packed_gu_bytes(P.H, P.I, BITS) + ((int64_t)rbg * P.dn_tiles + c * kChunkTiles) * TB;
+          const int n = min(chunk_tiles(BITS), P.dn_tiles - (int)c * chunk_tiles(BITS));
+          src = blob + packed_gu_bytes(P.H, P.I, BITS) + ((int64_t)rbg * P.dn_tiles + c * chunk_tiles(BITS)) * TB;
           bytes = (uint32_t)(n * TB);
         }
       }
@@ -972,11 +972,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           int n;
           if (ty == kTaskGateUp) {
             const int rb = (cta + (int)idx * G) % P.units_per_slot;
-            n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
-            off = ((int64_t)rb * P.gu_tiles + c * kChunkTiles) * TB;
+            n = min(chunk_tiles(BITS), P.gu_tiles - (int)c * chunk_tiles(BITS));
+            off = ((int64_t)rb * P.gu_tiles + c * chunk_tiles(BITS)) * TB;
           } else {
-            n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
-            off = packed_gu_bytes(P.H, P.I, BITS) + ((int64_t)(first_rb + (int)idx * G) * P.dn_tiles + c * kChunkTiles) * TB;
+            n = min(chunk_tiles(BITS), P.dn_tiles - (int)c * chunk_tiles(BITS));
+            off = packed_gu_bytes(P.H, P.I, BITS) + ((int64_t)(first_rb + (int)idx * G) * P.dn_tiles + c * chunk_tiles(BITS)) * TB;
           }
           bulk_store(misc->slot_dst[slot] + off, smem_u32(stage), (uint32_t)(n * TB));
         }
@@ -1031,8 +1031,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           }
         } else if (ty == kTaskGateUp) {
           if (lane == 0 && slot > 0) FMOE_TRACE_FIRST(cur, 8);
-          const int n = min(kChunkTiles, P.gu_tiles - (int)c * kChunkTiles);
-          const float2 acc = chunk_dot<BITS>(stage, n, zfrag, zinfo, (int)c * kChunkTiles, lane);
+          const int n = min(chunk_tiles(BITS), P.gu_tiles - (int)c * chunk_tiles(BITS));
+          const float2 acc = chunk_dot<BITS>(stage, n, zfrag, zinfo, (int)c * chunk_tiles(BITS), lane);
           float acc0 = acc.x, acc1 = acc.y;
           const int u = cta + (int)idx * G, rb = u % P.units_per_slot;
           bool last = true;
@@ -1151,8 +1151,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           }
           __threadfence_block();
           if (!good) break;
-          const int n = min(kChunkTiles, P.dn_tiles - (int)c * kChunkTiles);
-          const float2 acc = chunk_dot<BITS>(stage, n, af, ai, (int)c * kChunkTiles, lane);
+          const int n = min(chunk_tiles(BITS), P.dn_tiles - (int)c * chunk_tiles(BITS));
+          const float2 acc = chunk_dot<BITS>(stage, n, af, ai, (int)c * chunk_tiles(BITS), lane);
           const float acc0 = acc.x, acc1 = acc.y;
           float* y = ys + ((int)idx * P.n_slots + (int)slot) * 16;
           if (P.dn_chunks == 1) {

@@ -38,12 +38,17 @@ constexpr int kMaxSlots = kMaxTopK + 1;  // K routed + 1 shared
 constexpr int kConsumerWarps = 15;       // warps that compute (16 warps in all: 4 per SM sub-partition, 128 registers each)
 constexpr int kMaxHidden = 4096;         // largest hidden size a context accepts
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
-constexpr int kChunkTiles = 16;          // tiles per gate/up or down task
+// Tiles per gate/up or down task, one bulk copy each: 24 x 576 B = 13.5 KB at
+// 4-bit, 32 x 320 B = 10 KB at 2-bit.  Larger copies stream HBM faster; fewer
+// tasks per unit leave consumer warps idle (32 tiles at 4-bit measured slower).
+constexpr __host__ __device__ int chunk_tiles(int bits) { return bits == 4 ? 24 : 32; }
 constexpr int kMaxTasks = 96;            // task-list capacity per block (multiple of 32)
 constexpr int kStaticRouteLogits = 32768; // fp32 logits in the fixed scratch of fmoe_route_static (128 KB)
 constexpr int kStaticRouteMaxTokens = 4096;  // tokens per fmoe_route_static call
 constexpr int kMaxDevices = 64;          // devices fmoe_route_static caches a scratch address for
-constexpr int kMinRingStages = 20;       // ring stages kept when down jobs get stages of their own
+// Ring stages kept when down jobs get stages of their own (~180 KB of ring at
+// 4-bit; 100 KB at 2-bit, where the down jobs' own stages pay more).
+constexpr __host__ __device__ int min_ring_stages(int bits) { return bits == 4 ? 13 : 10; }
 constexpr int kFetchGroups = 8;          // activation groups a warp fetches per round trip
 constexpr int kTracePoints = 32;         // FMOE_TRACE builds: %globaltimer stamps per block and layer
 constexpr int kTraceLayers = 4;          // ... for the first layers of a launch
@@ -166,7 +171,7 @@ struct DecodePlan {
   int grid;                // blocks (one per SM)
   int tb, cb;              // tile bytes, code bytes per tile
   int gu_tiles;            // H/64 tiles per gate/up row block (unit)
-  int gu_chunks;           // tasks per unit (kChunkTiles tiles each, last may be shorter)
+  int gu_chunks;           // tasks per unit (chunk_tiles(bits) tiles each, last may be shorter)
   int dn_tiles;            // I/64 tiles per down row block
   int dn_chunks;           // tasks per down job
   int units_per_slot;      // I/8

@@ -92,13 +92,13 @@ int check(int H, int E, int K, int I, int bits, int G, int mode, bool must_plan)
         CHECK((int)idx < P.units_per_cta && (int)ch < P.gu_chunks && (int)slot < P.n_slots, "gate/up task");
         const int u = b + (int)idx * G;
         CHECK(u < P.total_units && u / P.units_per_slot == (int)slot, "unit %d slot %d", u, slot);
-        bytes = (uint32_t)std::min(kChunkTiles, P.gu_tiles - (int)ch * kChunkTiles) * P.tb;
+        bytes = (uint32_t)std::min(chunk_tiles(P.bits), P.gu_tiles - (int)ch * chunk_tiles(P.bits)) * P.tb;
         seen[{1, u, (int)ch}]++;
       } else {
         CHECK(ty == kTaskDown && (int)idx < P.rb_per_cta && (int)slot < P.n_slots && (int)ch < P.dn_chunks, "down task");
         const int rb = first_rb + (int)idx * G;
         CHECK(rb < P.n_rb, "row block %d", rb);
-        bytes = (uint32_t)std::min(kChunkTiles, P.dn_tiles - (int)ch * kChunkTiles) * P.tb;
+        bytes = (uint32_t)std::min(chunk_tiles(P.bits), P.dn_tiles - (int)ch * chunk_tiles(P.bits)) * P.tb;
         seen[{2, rb * 16 + (int)slot, (int)ch}]++;
       }
       CHECK(bytes > 0 && bytes <= P.stage_bytes && bytes % 16 == 0, "task bytes %u stage %u", bytes, P.stage_bytes);
