@@ -21,6 +21,7 @@
 //   combine  out = h + y_shared + sum_k w_k y_k, fp32, one bf16 rounding
 #include <cuda_bf16.h>
 #include <algorithm>
+#include <type_traits>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -474,6 +475,7 @@ struct GemvArgs {
   int bands;                 // 16-row bands of the matrix
   float* out;                // gate/up: a [P][I]; down: y [P][H]
   int ldo;
+  uint32_t* status;          // device status word (a timed-out wait sets kStatusTimeoutTc)
 };
 
 // B fragments of every small segment: one warp per (segment, group), the
@@ -522,64 +524,195 @@ __global__ void bt_gv_frag_kernel(GemvArgs g, int n_small_cap) {
   }
 }
 
-// One warp per (small segment, 16-row band): all K/64 tiles of the band.
-// Lane 4r+t accumulates rows r and r+8 of the band for positions 2t and 2t+1.
+// One block per (small segment, 8 consecutive 16-row bands): consumer warp w
+// contracts band 8o+w; lane 4r+t accumulates rows r and r+8 of the band for
+// positions 2t and 2t+1.  A producer warp streams the block's operands through
+// a ring of kBsStages shared-memory stages, each holding kBsGroups groups: per
+// band one bulk copy of its kBsGroups consecutive tiles (codes + scale/bias),
+// plus the segment's B fragments and input info for those groups, copied once
+// for all eight bands.  The block's items run as one stream of stages; one
+// block per SM (the ring takes ~180 KB of shared memory).
+constexpr int kBsWarps = 8;    // consumer warps (bands per item)
+constexpr int kBsGroups = 16;  // groups (tiles per band) per stage
+constexpr uint64_t kBsWaitNs = 500ull * 1000 * 1000;  // bounded waits: 0.5 s
+
+template <int BITS>
+struct BsLayout {
+  using Codes = typename std::conditional<BITS == 4, uint4, uint2>::type;  // one lane's codes of a tile
+  static constexpr int CODES = 16 * kGroup * BITS / 8;  // a 16-row band's codes for one group
+  static constexpr int TILE = CODES + 64;               // + the 16 rows' (scale, bias)
+  static constexpr int FRAG = kGemvTokens * 32 * 4;     // one group's B fragments (8 positions)
+  static constexpr int INFO = kGemvTokens * 8;          // (2^-sh, sum x) per position
+  static constexpr int BAND = kBsGroups * TILE;         // one band's tiles in a stage
+  static constexpr int STAGE = kBsWarps * BAND + kBsGroups * (FRAG + INFO);
+  static constexpr int STAGES = BITS == 4 ? 2 : 3;
+  static constexpr int SMEM = STAGES * STAGE + 2 * STAGES * 8 + 16;
+  static_assert(TILE % 16 == 0 && BAND % 128 == 0 && STAGE % 128 == 0, "bulk copy alignment");
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ uint32_t bs_su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ uint64_t bs_time() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ bool bs_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; false after kBsWaitNs or once the block has aborted.
+__device__ __forceinline__ bool bs_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag) {
+  if (bs_try(bar, parity)) return true;
+  const uint64_t t0 = bs_time();
+  for (uint32_t it = 0;; ++it) {
+    if (bs_try(bar, parity)) return true;
+    if ((it & 15) == 15 && (*abort_flag || bs_time() - t0 > kBsWaitNs)) return false;
+    if (it >= 8) __nanosleep(32);
+  }
+}
+__device__ __forceinline__ void bs_bulk(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 template <int BITS, bool GATE_UP>
-__global__ void __launch_bounds__(256) bt_gemv_kernel(GemvArgs g) {
-  constexpr int TB = 16 * kGroup * BITS / 8 + 64, CB = 16 * kGroup * BITS / 8;
-  const int lane = threadIdx.x & 31, r = lane >> 2, t = lane & 3;
-  const int G = g.K / kGroup, n_items = *g.n_items;
-  for (int it = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); it < n_items; it += gridDim.x * (blockDim.x / 32)) {
-    const int sr = it / g.bands, band = it % g.bands;
-    const int sg = g.small_seg[sr];
-    const int e = g.seg[sg], pos0 = g.seg[g.S + sg], n = g.seg[2 * g.S + sg];
-    const uint8_t* tiles = g.experts + (int64_t)e * g.blob + g.mat_off + (int64_t)band * G * TB;
-    const uint32_t* fr = g.frag + ((size_t)sr * G * kGemvTokens + r) * 32 + t * 8;
-    const float2* inf = g.info + (size_t)sr * G * kGemvTokens + 2 * t;
-    float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;  // (row r | r+8) x (position 2t | 2t+1)
-#pragma unroll 4
-    for (int gr = 0; gr < G; ++gr) {
-      const uint8_t* tile = tiles + (int64_t)gr * TB;
-      const uint4 f0 = *reinterpret_cast<const uint4*>(fr + (size_t)gr * kGemvTokens * 32);
-      const uint4 f1 = *reinterpret_cast<const uint4*>(fr + (size_t)gr * kGemvTokens * 32 + 4);
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-      if constexpr (BITS == 4) {
-        const uint4 qv = *reinterpret_cast<const uint4*>(tile + lane * 16);
-        const uint32_t w4[4] = {qv.x, qv.y, qv.z, qv.w};
-        const uint32_t bb[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-#pragma unroll
-        for (int sl = 0; sl < 4; ++sl) {
-          const uint32_t w = w4[sl], w8 = w >> 8;
-          gv_mma(c, gv_code2(w, 0x000F000Fu), gv_code2(w8, 0x000F000Fu), gv_code2(w, 0x00F000F0u),
-                 gv_code2(w8, 0x00F000F0u), bb[2 * sl], bb[2 * sl + 1]);
+__global__ void __launch_bounds__(32 * (kBsWarps + 1), 1) bt_gemv_kernel(GemvArgs g) {
+  using Ly = BsLayout<BITS>;
+  using Codes = typename Ly::Codes;
+  constexpr int S = Ly::STAGES;
+  extern __shared__ __align__(128) uint8_t bs_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base = bs_su32(bs_smem);
+  const uint32_t full0 = base + S * Ly::STAGE, empty0 = full0 + 8 * S;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bs_smem + S * Ly::STAGE + 16 * S);
+  const int G = g.K / kGroup;
+  const int n_small = *g.n_items / g.bands;  // GEMV items are counted as small segments x bands
+  const int octets = (g.bands + kBsWarps - 1) / kBsWarps;
+  const int n_blk_items = n_small * octets;
+  const int n_st = (G + kBsGroups - 1) / kBsGroups;  // stages per item
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full0 + 8 * s) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty0 + 8 * s), "r"(kBsWarps) : "memory");
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (warp == kBsWarps) {
+    // ---- producer: lane 0 fills stage q % S with the q-th stage of the block's stream
+    if (lane != 0) return;
+    int q = 0;
+    bool ok = true;
+    for (int bi = blockIdx.x; bi < n_blk_items && ok; bi += gridDim.x) {
+      const int sr = bi / octets, b0 = (bi % octets) * kBsWarps;
+      const int nb = min(kBsWarps, g.bands - b0);
+      const uint8_t* tiles = g.experts + (int64_t)g.seg[g.small_seg[sr]] * g.blob + g.mat_off;
+      const uint8_t* frag = reinterpret_cast<const uint8_t*>(g.frag) + (size_t)sr * G * Ly::FRAG;
+      const uint8_t* info = reinterpret_cast<const uint8_t*>(g.info) + (size_t)sr * G * Ly::INFO;
+      for (int j = 0; j < n_st; ++j, ++q) {
+        const int s = q % S, gs = j * kBsGroups, ng = min(kBsGroups, G - gs);
+        if (q >= S && !bs_wait(empty0 + 8 * s, (uint32_t)((q / S) - 1) & 1u, abort_flag)) {
+          ok = false;
+          break;
         }
-      } else {
-        const uint2 qv = *reinterpret_cast<const uint2*>(tile + lane * 8);
-        const uint32_t w2[2] = {qv.x, qv.y};
-        const uint32_t bb[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+        const uint32_t st = base + s * Ly::STAGE, full = full0 + 8 * s;
+        const uint32_t bytes = (uint32_t)(nb * ng * Ly::TILE + ng * (Ly::FRAG + Ly::INFO));
+        asm volatile("{ .reg .b64 t; mbarrier.arrive.expect_tx.shared::cta.b64 t, [%0], %1; }" ::"r"(full), "r"(bytes)
+                     : "memory");
+        for (int b = 0; b < nb; ++b)
+          bs_bulk(st + b * Ly::BAND, tiles + ((int64_t)(b0 + b) * G + gs) * Ly::TILE, (uint32_t)(ng * Ly::TILE), full);
+        bs_bulk(st + kBsWarps * Ly::BAND, frag + (size_t)gs * Ly::FRAG, (uint32_t)(ng * Ly::FRAG), full);
+        bs_bulk(st + kBsWarps * Ly::BAND + kBsGroups * Ly::FRAG, info + (size_t)gs * Ly::INFO,
+                (uint32_t)(ng * Ly::INFO), full);
+      }
+    }
+    if (!ok) {
+      if (!*abort_flag) atomicOr(g.status, kStatusTimeoutTc);
+      *abort_flag = 1;
+    }
+    // every stage issued but not yet seen complete lands before the block exits (bounded)
+    const uint64_t t0 = bs_time();
+    for (int v = max(0, q - S); v < q; ++v)
+      while (!bs_try(full0 + 8 * (v % S), (uint32_t)(v / S) & 1u) && bs_time() - t0 < kBsWaitNs) __nanosleep(64);
+    return;
+  }
+  // ---- consumers: warp w contracts band b0 + w of each item
+  const int r = lane >> 2, t = lane & 3;
+  int q = 0;
+  for (int bi = blockIdx.x; bi < n_blk_items; bi += gridDim.x) {
+    const int sr = bi / octets, band = (bi % octets) * kBsWarps + warp;
+    const int sg = g.small_seg[sr];
+    const int pos0 = g.seg[g.S + sg], n = g.seg[2 * g.S + sg];
+    const bool mine = band < g.bands;
+    float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;  // (row r | r+8) x (position 2t | 2t+1)
+    for (int j = 0; j < n_st; ++j, ++q) {
+      const int s = q % S, ng = min(kBsGroups, G - j * kBsGroups);
+      if (!__all_sync(0xffffffffu, bs_wait(full0 + 8 * s, (uint32_t)(q / S) & 1u, abort_flag))) {
+        if (lane == 0) {
+          if (!*abort_flag) atomicOr(g.status, kStatusTimeoutTc);
+          *abort_flag = 1;
+        }
+        return;
+      }
+      const uint8_t* st = bs_smem + s * Ly::STAGE;
+      const uint8_t* codes = st + warp * Ly::BAND;
+      const uint8_t* frag = st + kBsWarps * Ly::BAND + (r * 32 + t * 8) * 4;
+      const uint8_t* info = st + kBsWarps * Ly::BAND + kBsGroups * Ly::FRAG + 2 * t * 8;
+      if (mine) {
+#pragma unroll 4
+        for (int k = 0; k < ng; ++k) {
+          const uint8_t* tile = codes + k * Ly::TILE;
+          const Codes qv = *reinterpret_cast<const Codes*>(tile + lane * sizeof(Codes));
+          const uint2 sb = *reinterpret_cast<const uint2*>(tile + Ly::CODES + r * 8);
+          const uint4 f0 = *reinterpret_cast<const uint4*>(frag + k * Ly::FRAG);
+          const uint4 f1 = *reinterpret_cast<const uint4*>(frag + k * Ly::FRAG + 16);
+          const float4 iv = *reinterpret_cast<const float4*>(info + k * Ly::INFO);  // positions 2t, 2t+1
+          const uint32_t bb[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+          float c[4] = {0.f, 0.f, 0.f, 0.f};
+          if constexpr (BITS == 4) {
+            const uint32_t w4[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-        for (int wj = 0; wj < 2; ++wj) {
-          const uint32_t w = w2[wj], w8 = w >> 8;
-          gv_mma(c, gv_code2(w, 0x00030003u), gv_code2(w8, 0x00030003u), gv_code2(w, 0x000C000Cu),
-                 gv_code2(w8, 0x000C000Cu), bb[4 * wj], bb[4 * wj + 1]);
-          gv_mma(c, gv_code2(w, 0x00300030u), gv_code2(w8, 0x00300030u), gv_code2(w, 0x00C000C0u),
-                 gv_code2(w8, 0x00C000C0u), bb[4 * wj + 2], bb[4 * wj + 3]);
+            for (int sl = 0; sl < 4; ++sl) {
+              const uint32_t w = w4[sl], w8 = w >> 8;
+              gv_mma(c, gv_code2(w, 0x000F000Fu), gv_code2(w8, 0x000F000Fu), gv_code2(w, 0x00F000F0u),
+                     gv_code2(w8, 0x00F000F0u), bb[2 * sl], bb[2 * sl + 1]);
+            }
+          } else {
+            const uint32_t w2[2] = {qv.x, qv.y};
+#pragma unroll
+            for (int wj = 0; wj < 2; ++wj) {
+              const uint32_t w = w2[wj], w8 = w >> 8;
+              gv_mma(c, gv_code2(w, 0x00030003u), gv_code2(w8, 0x00030003u), gv_code2(w, 0x000C000Cu),
+                     gv_code2(w8, 0x000C000Cu), bb[4 * wj], bb[4 * wj + 1]);
+              gv_mma(c, gv_code2(w, 0x00300030u), gv_code2(w8, 0x00300030u), gv_code2(w, 0x00C000C0u),
+                     gv_code2(w8, 0x00C000C0u), bb[4 * wj + 2], bb[4 * wj + 3]);
+            }
+          }
+          const float s0 = bflo(sb.x), b0 = bfhi(sb.x), s8 = bflo(sb.y), b8 = bfhi(sb.y);
+          a00 = fmaf(s0 * iv.x, c[0], fmaf(b0, iv.y, a00));
+          a01 = fmaf(s0 * iv.z, c[1], fmaf(b0, iv.w, a01));
+          a10 = fmaf(s8 * iv.x, c[2], fmaf(b8, iv.y, a10));
+          a11 = fmaf(s8 * iv.z, c[3], fmaf(b8, iv.w, a11));
         }
       }
-      const uint2 sb = *reinterpret_cast<const uint2*>(tile + CB + r * 8);
-      const float4 iv = *reinterpret_cast<const float4*>(inf + (size_t)gr * kGemvTokens);  // positions 2t, 2t+1
-      const float s0 = bflo(sb.x), b0 = bfhi(sb.x), s8 = bflo(sb.y), b8 = bfhi(sb.y);
-      a00 = fmaf(s0 * iv.x, c[0], fmaf(b0, iv.y, a00));
-      a01 = fmaf(s0 * iv.z, c[1], fmaf(b0, iv.w, a01));
-      a10 = fmaf(s8 * iv.x, c[2], fmaf(b8, iv.y, a10));
-      a11 = fmaf(s8 * iv.z, c[3], fmaf(b8, iv.w, a11));
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty0 + 8 * s) : "memory");
     }
+    if (!mine) continue;
     const int p0 = 2 * t, p1 = 2 * t + 1;
     if constexpr (GATE_UP) {
       // band rows r (gate) and r + 8 (up) are the same activation j
-      const int j = band * 8 + r;
-      if (p0 < n) g.out[(size_t)(pos0 + p0) * g.ldo + j] = a00 / (1.0f + expf(-a00)) * a10;
-      if (p1 < n) g.out[(size_t)(pos0 + p1) * g.ldo + j] = a01 / (1.0f + expf(-a01)) * a11;
+      const int jj = band * 8 + r;
+      if (p0 < n) g.out[(size_t)(pos0 + p0) * g.ldo + jj] = a00 / (1.0f + expf(-a00)) * a10;
+      if (p1 < n) g.out[(size_t)(pos0 + p1) * g.ldo + jj] = a01 / (1.0f + expf(-a01)) * a11;
     } else {
       const int row = band * 16 + r;
       if (p0 < n) {
@@ -620,16 +753,22 @@ __global__ void bt_combine_kernel(const uint16_t* __restrict__ h, const float* _
   }
 }
 
-int launch_gemv(int bits, bool gate_up, const GemvArgs& v, int n_sm, cudaStream_t st) {
-  const dim3 grid(4 * n_sm), block(256);
-  if (bits == 4) {
-    if (gate_up) bt_gemv_kernel<4, true><<<grid, block, 0, st>>>(v);
-    else bt_gemv_kernel<4, false><<<grid, block, 0, st>>>(v);
-  } else {
-    if (gate_up) bt_gemv_kernel<2, true><<<grid, block, 0, st>>>(v);
-    else bt_gemv_kernel<2, false><<<grid, block, 0, st>>>(v);
+template <int BITS, bool GATE_UP>
+int launch_gemv_t(const GemvArgs& v, int n_sm, cudaStream_t st) {
+  static bool sized = false;  // opt in to the kernel's dynamic shared memory once
+  if (!sized) {
+    const cudaError_t e = cudaFuncSetAttribute(bt_gemv_kernel<BITS, GATE_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               BsLayout<BITS>::SMEM);
+    if (e != cudaSuccess) return (int)e;
+    sized = true;
   }
+  bt_gemv_kernel<BITS, GATE_UP><<<n_sm, 32 * (kBsWarps + 1), BsLayout<BITS>::SMEM, st>>>(v);
   return (int)cudaGetLastError();
+}
+
+int launch_gemv(int bits, bool gate_up, const GemvArgs& v, int n_sm, cudaStream_t st) {
+  if (bits == 4) return gate_up ? launch_gemv_t<4, true>(v, n_sm, st) : launch_gemv_t<4, false>(v, n_sm, st);
+  return gate_up ? launch_gemv_t<2, true>(v, n_sm, st) : launch_gemv_t<2, false>(v, n_sm, st);
 }
 
 int grid_of(int64_t work, int per_block, int cap) {
@@ -769,6 +908,7 @@ int launch_batched(const BatchArgs& a, const BatchWs& ws, int n_sm, void* stream
   v.info = ws.gv_info;
   v.experts = a.experts;
   v.blob = a.blob_bytes;
+  v.status = a.status;
   mark(0);
   v.n_items = ws.n_items + 2;
   v.src = ws.z;
