@@ -755,13 +755,10 @@ __global__ void bt_combine_kernel(const uint16_t* __restrict__ h, const float* _
 
 template <int BITS, bool GATE_UP>
 int launch_gemv_t(const GemvArgs& v, int n_sm, cudaStream_t st) {
-  static bool sized = false;  // opt in to the kernel's dynamic shared memory once
-  if (!sized) {
-    const cudaError_t e = cudaFuncSetAttribute(bt_gemv_kernel<BITS, GATE_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               BsLayout<BITS>::SMEM);
-    if (e != cudaSuccess) return (int)e;
-    sized = true;
-  }
+  // the shared-memory opt-in is per device: set it on every launch, like the other kernels
+  const cudaError_t e = cudaFuncSetAttribute(bt_gemv_kernel<BITS, GATE_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             BsLayout<BITS>::SMEM);
+  if (e != cudaSuccess) return (int)e;
   bt_gemv_kernel<BITS, GATE_UP><<<n_sm, 32 * (kBsWarps + 1), BsLayout<BITS>::SMEM, st>>>(v);
   return (int)cudaGetLastError();
 }
